@@ -1,0 +1,353 @@
+"""CPU oracle for the DualQuant dual-scale W4A4 path -- TEST INFRASTRUCTURE.
+
+Only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline / reference
+legs may import this package.  It shares no code with the CUDA library in
+w4a4_post_quantization_dual_b200 and imports nothing from it.
+
+Source: "DualQuant: Dual-scale Calibration-free Weight-and-Activation
+Quantization for LLMs" (arXiv 2610.13767).  The element-level quantisers and
+Algorithm 1 live in dq_oracle.c (fp64 accumulation, fp32 quantiser
+arguments); this module adds ctypes marshalling and the dequantised
+reference matmul of Eq. (3) / Section 4.4 in numpy fp64.
+
+The block-scale storage layout (sf_offset) is a hardware convention of the
+block-scaled tensor-core MMA, not a result of the paper: parity unpinned
+(it is checked only against its own written definition).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+INT4, MXINT4, MXFP4, NVFP4 = 0, 1, 2, 3
+FORMAT_NAMES = {"int4": INT4, "mxint4": MXINT4, "mxfp4": MXFP4, "nvfp4": NVFP4}
+NATIVE_GROUP = {INT4: 64, MXINT4: 32, MXFP4: 32, NVFP4: 16}
+
+_lib = None
+
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_i64 = ctypes.c_int64
+
+
+def lib():
+    """Load (building if needed) the C oracle."""
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        sig = {
+            "oracle_e2m1_value": (ctypes.c_double, [ctypes.c_int]),
+            "oracle_e2m1_encode": (ctypes.c_int, [ctypes.c_float]),
+            "oracle_int4_value": (ctypes.c_double, [ctypes.c_int]),
+            "oracle_int4_encode": (ctypes.c_int, [ctypes.c_float]),
+            "oracle_e4m3_value": (ctypes.c_double, [ctypes.c_int]),
+            "oracle_ue4m3_rne": (ctypes.c_int, [ctypes.c_double]),
+            "oracle_ue4m3_proj": (ctypes.c_int, [ctypes.c_double]),
+            "oracle_e8m0_value": (ctypes.c_double, [ctypes.c_int]),
+            "oracle_e8m0_proj": (ctypes.c_int, [ctypes.c_double]),
+            "oracle_bf16_value": (ctypes.c_double, [ctypes.c_int]),
+            "oracle_bf16_rne": (ctypes.c_int, [ctypes.c_double]),
+            "oracle_bf16_proj": (ctypes.c_double, [ctypes.c_double]),
+            "oracle_proj_alpha": (ctypes.c_double, [ctypes.c_int, ctypes.c_double, ctypes.c_float]),
+            "oracle_proj_beta": (ctypes.c_double, [ctypes.c_int, ctypes.c_double]),
+            "oracle_init_c": (None, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int, _f32p]),
+            "oracle_tensor_scale": (ctypes.c_float, [_f32p, _i64, _i64, _f32p]),
+            "oracle_init_r": (None, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int, _f32p,
+                                     ctypes.c_float, _f32p]),
+            "oracle_solve": (None, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    _i64p, _i64, _f32p, _f32p, _f32p, _f64p, _f64p]),
+            "oracle_error": (ctypes.c_double, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int,
+                                               _f32p, _f32p]),
+            "oracle_error_fixed_q": (ctypes.c_double, [_f32p, _u8p, _i64, _i64, ctypes.c_int,
+                                                       ctypes.c_int, _f32p, _f32p]),
+            "oracle_codes": (None, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int, _f32p, _f32p,
+                                    _u8p]),
+            "oracle_update_fixed_q": (None, [_f32p, _u8p, _i64, _i64, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_float, _f32p, _f32p, ctypes.c_int]),
+            "oracle_sf_offset": (_i64, [_i64, _i64, _i64]),
+            "oracle_sf_bytes": (_i64, [_i64, _i64]),
+            "oracle_pack_weight": (None, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int, _f32p,
+                                          _f32p, ctypes.c_float, _u8p, _u8p]),
+            "oracle_quantize_act": (None, [_f32p, _i64, _i64, _f32p, ctypes.c_int, ctypes.c_int,
+                                           _u8p, _u8p, _f32p]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _p(a, t):
+    return a.ctypes.data_as(t)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+# ---------------------------------------------------------------- formats
+def e2m1_value(code):
+    return lib().oracle_e2m1_value(int(code))
+
+
+def e2m1_encode(t):
+    return lib().oracle_e2m1_encode(float(np.float32(t)))
+
+
+def int4_value(code):
+    return lib().oracle_int4_value(int(code))
+
+
+def int4_encode(t):
+    return lib().oracle_int4_encode(float(np.float32(t)))
+
+
+def e4m3_value(b):
+    return lib().oracle_e4m3_value(int(b))
+
+
+def ue4m3_rne(x):
+    return lib().oracle_ue4m3_rne(float(x))
+
+
+def ue4m3_proj(u):
+    return lib().oracle_ue4m3_proj(float(u))
+
+
+def e8m0_value(b):
+    return lib().oracle_e8m0_value(int(b))
+
+
+def e8m0_proj(u):
+    return lib().oracle_e8m0_proj(float(u))
+
+
+def bf16_value(h):
+    return lib().oracle_bf16_value(int(h))
+
+
+def bf16_rne(x):
+    return lib().oracle_bf16_rne(float(x))
+
+
+def bf16_proj(u):
+    return lib().oracle_bf16_proj(float(u))
+
+
+def proj_alpha(fmt, u, s_T=1.0):
+    return lib().oracle_proj_alpha(fmt, float(u), float(s_T))
+
+
+def proj_beta(fmt, u):
+    return lib().oracle_proj_beta(fmt, float(u))
+
+
+def elem_value_table(fmt):
+    """Value of each of the 16 element codes."""
+    f = int4_value if fmt in (INT4, MXINT4) else e2m1_value
+    return np.array([f(k) for k in range(16)], dtype=np.float64)
+
+
+# ---------------------------------------------------------------- solver
+def init_c(W, fmt, G):
+    W = _f32(W)
+    m, n = W.shape
+    c = np.empty(n, np.float32)
+    lib().oracle_init_c(_p(W, _f32p), m, n, fmt, G, _p(c, _f32p))
+    return c
+
+
+def tensor_scale(W, c):
+    W = _f32(W)
+    m, n = W.shape
+    return float(lib().oracle_tensor_scale(_p(W, _f32p), m, n, _p(_f32(c), _f32p)))
+
+
+def init_r(W, fmt, G, c, s_T=1.0):
+    """Format-native RTN row-block scales of W * diag(c)^-1 (c = 1: plain RTN)."""
+    W = _f32(W)
+    m, n = W.shape
+    r = np.empty((m, n // G), np.float32)
+    lib().oracle_init_r(_p(W, _f32p), m, n, fmt, G, _p(_f32(c), _f32p), float(s_T), _p(r, _f32p))
+    return r
+
+
+def solve(W, fmt, G, T, tiles=None):
+    """Algorithm 1 on every (or the listed) m x G tile.
+
+    Returns dict(r (m, n/G) f32, c (n,) f32, s_T float, trace (T+1,) f64 =
+    normalised MSE ||W - W_hat||^2 / ||W||^2 over the solved tiles).
+    """
+    W = _f32(W)
+    m, n = W.shape
+    nb = n // G
+    r = np.empty((m, nb), np.float32)
+    c = np.empty(n, np.float32)
+    sT = np.zeros(1, np.float32)
+    err = np.zeros(T + 1, np.float64)
+    w2 = np.zeros(1, np.float64)
+    if tiles is None:
+        tp, nt = None, 0
+    else:
+        tarr = np.ascontiguousarray(tiles, dtype=np.int64)
+        tp, nt = _p(tarr, _i64p), len(tarr)
+    lib().oracle_solve(_p(W, _f32p), m, n, fmt, G, T, tp, nt, _p(r, _f32p), _p(c, _f32p),
+                       _p(sT, _f32p), _p(err, _f64p), _p(w2, _f64p))
+    trace = err / w2[0] if w2[0] > 0 else err
+    return {"r": r, "c": c, "s_T": float(sT[0]), "trace": trace, "err": err, "w2": float(w2[0])}
+
+
+def error(W, fmt, G, r, c):
+    W = _f32(W)
+    m, n = W.shape
+    return lib().oracle_error(_p(W, _f32p), m, n, fmt, G, _p(_f32(r), _f32p), _p(_f32(c), _f32p))
+
+
+def error_fixed_q(W, Q, fmt, G, r, c):
+    W = _f32(W)
+    m, n = W.shape
+    Q = np.ascontiguousarray(Q, np.uint8)
+    return lib().oracle_error_fixed_q(_p(W, _f32p), _p(Q, _u8p), m, n, fmt, G,
+                                      _p(_f32(r), _f32p), _p(_f32(c), _f32p))
+
+
+def codes(W, fmt, G, r, c):
+    W = _f32(W)
+    m, n = W.shape
+    Q = np.empty((m, n), np.uint8)
+    lib().oracle_codes(_p(W, _f32p), m, n, fmt, G, _p(_f32(r), _f32p), _p(_f32(c), _f32p),
+                       _p(Q, _u8p))
+    return Q
+
+
+def update_fixed_q(W, Q, fmt, G, r, c, which, s_T=1.0):
+    """One projected closed-form half-step with Q held fixed (Eq. 10 rows, Eq. 14 columns)."""
+    W = _f32(W)
+    m, n = W.shape
+    r = _f32(r).copy()
+    c = _f32(c).copy()
+    Q = np.ascontiguousarray(Q, np.uint8)
+    lib().oracle_update_fixed_q(_p(W, _f32p), _p(Q, _u8p), m, n, fmt, G, float(s_T),
+                                _p(r, _f32p), _p(c, _f32p), int(which))
+    return r, c
+
+
+# ---------------------------------------------------------------- packing
+def sf_offset(row, s, S):
+    return int(lib().oracle_sf_offset(int(row), int(s), int(S)))
+
+
+def sf_bytes(rows, S):
+    return int(lib().oracle_sf_bytes(int(rows), int(S)))
+
+
+def pack_weight(W, fmt, G, r, c, s_T=1.0):
+    """Packed codes (m, n/2) u8 and scales (GEMM layout bytes, or (m, n/G) u16 bf16 for INT4)."""
+    W = _f32(W)
+    m, n = W.shape
+    cod = np.empty((m, n // 2), np.uint8)
+    if fmt == INT4:
+        sc = np.empty((m, n // G), np.uint16)
+    else:
+        sc = np.empty(sf_bytes(m, n // G), np.uint8)
+    lib().oracle_pack_weight(_p(W, _f32p), m, n, fmt, G, _p(_f32(r), _f32p), _p(_f32(c), _f32p),
+                             float(s_T), _p(cod, _u8p), sc.ctypes.data_as(_u8p))
+    return cod, sc
+
+
+def quantize_act(X, c, fmt, G):
+    """Rescale by c and quantise.  Returns (codes (M, K/2) u8, scales, s_tok (M,) f32)."""
+    X = _f32(X)
+    M, K = X.shape
+    cod = np.empty((M, K // 2), np.uint8)
+    if fmt == INT4:
+        sc = np.empty((M, K // G), np.uint16)
+    else:
+        sc = np.empty(sf_bytes(M, K // G), np.uint8)
+    st = np.zeros(M, np.float32)
+    lib().oracle_quantize_act(_p(X, _f32p), M, K, _p(_f32(c), _f32p), fmt, G, _p(cod, _u8p),
+                              sc.ctypes.data_as(_u8p), _p(st, _f32p))
+    return cod, sc, st
+
+
+# ---------------------------------------------------------------- reference GEMM
+def unpack_codes(packed, K):
+    """(R, K/2) bytes -> (R, K) codes, element 2k in the low nibble of byte k."""
+    packed = np.asarray(packed, np.uint8)
+    out = np.empty((packed.shape[0], K), np.uint8)
+    out[:, 0::2] = packed & 0xF
+    out[:, 1::2] = packed >> 4
+    return out
+
+
+def scale_values(sf, rows, S, fmt):
+    """Decode block scales stored in the GEMM layout -> (rows, S) float64."""
+    sf = np.asarray(sf, np.uint8).reshape(-1)
+    rr = np.arange(rows)[:, None]
+    ss = np.arange(S)[None, :]
+    S4 = (S + 3) // 4
+    off = ((rr // 128) * S4 + ss // 4) * 512 + (rr % 32) * 16 + ((rr % 128) // 32) * 4 + (ss % 4)
+    b = sf[off]
+    if fmt == NVFP4:
+        tab = np.array([e4m3_value(k) for k in range(256)], np.float64)
+    else:
+        tab = np.array([e8m0_value(k) if k < 255 else np.nan for k in range(256)], np.float64)
+    return tab[b]
+
+
+def dequant(packed, sf, rows, K, fmt, G, row_scale=None):
+    """Dequantised operand (rows, K) fp64 = code value x block scale (x per-row scale)."""
+    q = elem_value_table(fmt)[unpack_codes(packed, K)]
+    s = scale_values(sf, rows, K // G, fmt)
+    v = q * np.repeat(s, G, axis=1)
+    if row_scale is not None:
+        v = v * np.asarray(row_scale, np.float64)[:, None]
+    return v
+
+
+def linear(A, sA, s_tok, B, sB, s_W, M, N, K, fmt, r_row=None):
+    """Y = dequant(A) dequant(B)^T * s_tok[t] * s_W (* r_row[n]) in fp64 (Eq. 3, Section 4.4)."""
+    G = NATIVE_GROUP[fmt]
+    a = dequant(A, sA, M, K, fmt, G, s_tok if fmt == NVFP4 else None)
+    b = dequant(B, sB, N, K, fmt, G)
+    Y = a @ b.T
+    if fmt == NVFP4:
+        Y = Y * float(s_W)
+    if r_row is not None:
+        Y = Y * np.asarray(r_row, np.float64)[None, :]
+    return Y
+
+
+def linear_rows(A, sA, s_tok, B, sB, s_W, rows, M, N, K, fmt, r_row=None):
+    """Selected output rows of linear(), for sampled checks at full size."""
+    G = NATIVE_GROUP[fmt]
+    rows = np.asarray(rows)
+    S = K // G
+    Asub = np.asarray(A).reshape(M, K // 2)[rows]
+    q = elem_value_table(fmt)[unpack_codes(Asub, K)]
+    sf = np.asarray(sA, np.uint8).reshape(-1)
+    S4 = (S + 3) // 4
+    rr = rows[:, None]
+    ss = np.arange(S)[None, :]
+    off = ((rr // 128) * S4 + ss // 4) * 512 + (rr % 32) * 16 + ((rr % 128) // 32) * 4 + (ss % 4)
+    if fmt == NVFP4:
+        tab = np.array([e4m3_value(k) for k in range(256)], np.float64)
+    else:
+        tab = np.array([e8m0_value(k) if k < 255 else np.nan for k in range(256)], np.float64)
+    a = q * np.repeat(tab[sf[off]], G, axis=1)
+    if fmt == NVFP4:
+        a = a * np.asarray(s_tok, np.float64)[rows][:, None]
+    b = dequant(B, sB, N, K, fmt, G)
+    Y = a @ b.T
+    if fmt == NVFP4:
+        Y = Y * float(s_W)
+    if r_row is not None:
+        Y = Y * np.asarray(r_row, np.float64)[None, :]
+    return Y
