@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the DualQuant dual-scale W4A4 hot path on B200.
+
+One step = the whole path over the Llama-3.1-8B-shaped attention workload
+(weights 4096x4096 and 1024x4096 bf16, NVFP4, 50 BCD rounds; activations
+M in {1, 16, 256, 4096} x 4096 bf16 with 1 % outlier channels x50):
+    for each weight : dq_solve_scales (T = 50) -> dq_quantize_weight
+    for each M, each weight : dq_quantize_act -> dq_w4a4_linear
+Inputs are resident in HBM before timing; L2 (126 MB) is flushed between
+steps by writing a 256 MiB buffer outside the timed events.
+
+`value` = W4A4 linear TFLOP/s of the inference part of the step (act quant
++ GEMM, 2*M*N*K summed over the 8 linears, divided by their device time).
+The solver is reported beside it as effective streaming GB/s
+(T * bytes(W) / time) and its own time; ms_per_step covers everything.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from w4a4_post_quantization_dual_b200 import synth  # noqa: E402
+
+WORKLOAD = "llama8b_attn_nvfp4"
+METRIC = "W4A4 linear TFLOP/s & % of FP4 peak; BCD solver GB/s & % HBM peak"
+FMT_NAME = "nvfp4"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), d.get(
+            "sm_max_mhz", 1965.0), "measured"
+    return 6650.0, 1590.0, 1400.0, 1965.0, "fallback"
+
+
+def workload_inputs():
+    wl = synth.WORKLOADS[WORKLOAD]
+    Ws = [synth.weight(WORKLOAD, i)[0] for i in range(len(wl["weights"]))]
+    K = Ws[0].shape[1]
+    Xs = {M: synth.acts(WORKLOAD, M, K)[0] for M in wl["M"]}
+    return wl, Ws, Xs
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.proc, self.lines = index, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(max(mx)) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# Reference arm / CPU baseline: the oracle as it stands, on host cores.
+# ---------------------------------------------------------------------------
+def oracle_sample(wl, Ws, Xs, rows=64):
+    """Bounded oracle run on the same workload: the inference path (act
+    quant + dequantised fp64 matmul) on `rows` token rows of the M=4096
+    activations for both weights, plus Algorithm 1 on one 4096x16 tile.
+    Returns (linear TFLOP/s, solver GB/s effective, seconds, description)."""
+    import oracle as O
+    fmt, G, T = O.NVFP4, 16, wl["T"]
+    t0 = time.perf_counter()
+    flops = 0.0
+    t_lin = 0.0
+    t_sol = 0.0
+    solved_bytes = 0.0
+    X = Xs[max(Xs)][:rows]
+    for W in Ws:
+        N, K = W.shape
+        ts = time.perf_counter()
+        res = O.solve(W, fmt, G, T, tiles=[0])
+        t_sol += time.perf_counter() - ts
+        solved_bytes += T * W.shape[0] * G * 2.0
+        tl = time.perf_counter()
+        A, sA, st = O.quantize_act(X, res["c"], fmt, G)
+        B, sB = O.pack_weight(W, fmt, G, res["r"], res["c"], res["s_T"])
+        O.linear(A, sA, st, B, sB, res["s_T"], rows, N, K, fmt)
+        t_lin += time.perf_counter() - tl
+        flops += 2.0 * rows * N * K
+    desc = (f"oracle: act quant + weight pack + fp64 dequantised matmul on {rows} of 4096 "
+            f"token rows for both weights; Algorithm 1 (T={T}) on one 4096x16 tile per weight")
+    return flops / t_lin / 1e12, solved_bytes / t_sol / 1e9, time.perf_counter() - t0, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl, Ws, Xs = workload_inputs()
+    for _ in range(args.warmup):
+        oracle_sample(wl, Ws, Xs, rows=16)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, _, _, desc = oracle_sample(wl, Ws, Xs, rows=16)
+        vals.append(v)
+    dt = time.perf_counter() - t0
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / max(args.steps, 1) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "format": FMT_NAME, "sample_rows": 16},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc.replace("64 of", "16 of")},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    from w4a4_post_quantization_dual_b200 import dq
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dq.lib()
+    wl, Ws, Xs = workload_inputs()
+    fmt, T = dq.DQ_NVFP4, wl["T"]
+    G = dq.native_group(fmt)
+    st = torch.cuda.current_stream()
+
+    # device-resident inputs and outputs
+    Wd = [torch.from_numpy(W).to(torch.bfloat16).to(dev) for W in Ws]
+    Xd = {M: torch.from_numpy(X).to(torch.bfloat16).to(dev) for M, X in Xs.items()}
+    ws = torch.empty(dq.solve_workspace_size(T), dtype=torch.uint8, device=dev)
+    Wbuf = []
+    for W in Wd:
+        m, n = W.shape
+        Wbuf.append(dict(
+            r=torch.empty((m, n // G), dtype=torch.float32, device=dev),
+            c=torch.empty(n, dtype=torch.float32, device=dev),
+            sT=torch.empty(1, dtype=torch.float32, device=dev),
+            codes=torch.empty((m, n // 2), dtype=torch.uint8, device=dev),
+            scales=torch.empty(dq.scales_bytes(m, n, fmt, G), dtype=torch.uint8, device=dev)))
+    Abuf = {}
+    for M, X in Xd.items():
+        K = X.shape[1]
+        Abuf[M] = dict(A=torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                       sA=torch.empty(dq.scales_bytes(M, K, fmt, G), dtype=torch.uint8, device=dev),
+                       st=torch.empty(M, dtype=torch.float32, device=dev),
+                       Y=[torch.empty((M, W.shape[0]), dtype=torch.bfloat16, device=dev) for W in Wd])
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    lin_flops = sum(2.0 * M * W.shape[0] * W.shape[1] for M in Xd for W in Wd)
+    prefill_M = max(Xd)
+    launches_per_step = 2 * len(Wd) + len(Wd) + 2 * len(Wd) * len(Xd)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def step(rec):
+        e0, e1, e2 = ev(), ev(), ev()
+        e0.record(st)
+        for W, b in zip(Wd, Wbuf):
+            s0, s1 = ev(), ev()
+            s0.record(st)
+            dq.dq_solve_scales(W, fmt, T, b["r"], b["c"], b["sT"], None, ws, group=G)
+            s1.record(st)
+            dq.dq_quantize_weight(W, fmt, b["r"], b["c"], b["sT"], b["codes"], b["scales"], group=G)
+            rec["solve"].append((s0, s1))
+        e1.record(st)
+        for M, X in Xd.items():
+            a = Abuf[M]
+            for j, (W, b) in enumerate(zip(Wd, Wbuf)):
+                q0, q1, g1 = ev(), ev(), ev()
+                q0.record(st)
+                dq.dq_quantize_act(X, fmt, b["c"], a["A"], a["sA"], a["st"], group=G)
+                q1.record(st)
+                dq.dq_w4a4_linear(a["A"], a["sA"], a["st"], b["codes"], b["scales"], b["sT"],
+                                  a["Y"][j], fmt)
+                g1.record(st)
+                rec["act"].append((q0, q1, M * X.shape[1]))
+                rec["gemm"].append((q1, g1, 2.0 * M * W.shape[0] * W.shape[1], M))
+        e2.record(st)
+        rec["step"].append((e0, e2))
+        rec["lin"].append((e1, e2))
+
+    if world > 1:
+        torch.distributed.barrier()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step({"solve": [], "act": [], "gemm": [], "step": [], "lin": []})
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    rec = {"solve": [], "act": [], "gemm": [], "step": [], "lin": []}
+    for _ in range(args.steps):
+        flush.fill_(rank + 1)      # L2 flush, outside the timed events
+        step(rec)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dq.dq_device_error(clear=True) != 0:
+        raise RuntimeError("device error word set during the bench")
+
+    el = lambda p: p[0].elapsed_time(p[1])  # ms
+    step_ms = sum(el(p) for p in rec["step"])
+    lin_ms = sum(el(p) for p in rec["lin"])
+    solve_ms = sum(el(p) for p in rec["solve"])
+    gemm_pre = [(el((p[0], p[1])), p[2]) for p in rec["gemm"] if p[3] == prefill_M]
+    act_pre = [(el((p[0], p[1])), p[2]) for p in rec["act"] if p[2] == prefill_M * 4096]
+    totals = torch.tensor([step_ms, lin_ms, solve_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(totals, op=torch.distributed.ReduceOp.MAX)
+    step_ms, lin_ms, solve_ms = totals.tolist()
+
+    # ---- e2e through the public API with host buffers (pinned), prefill linears
+    e2e = None
+    if rank == 0 or world > 1:
+        Xh = torch.from_numpy(Xs[prefill_M]).to(torch.bfloat16).pin_memory()
+        Yh = [torch.empty((prefill_M, W.shape[0]), dtype=torch.bfloat16).pin_memory() for W in Wd]
+        a = Abuf[prefill_M]
+        Xdev = torch.empty_like(Xd[prefill_M])
+
+        def e2e_step():
+            Xdev.copy_(Xh, non_blocking=True)
+            for j, (W, b) in enumerate(zip(Wd, Wbuf)):
+                dq.dq_quantize_act(Xdev, fmt, b["c"], a["A"], a["sA"], a["st"], group=G)
+                dq.dq_w4a4_linear(a["A"], a["sA"], a["st"], b["codes"], b["scales"], b["sT"],
+                                  a["Y"][j], fmt)
+                Yh[j].copy_(a["Y"][j], non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(max(args.steps, 5)):
+            flush.fill_(2)
+            x0, x1 = ev(), ev()
+            x0.record(st)
+            e2e_step()
+            x1.record(st)
+            x1.synchronize()
+            tot += x0.elapsed_time(x1)
+        n_e2e = max(args.steps, 5)
+        fl = sum(2.0 * prefill_M * W.shape[0] * W.shape[1] for W in Wd)
+        e2e = {"value": fl * n_e2e / (tot * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": Xh.numel() * 2,
+               "d2h_bytes_per_step": sum(y.numel() * 2 for y in Yh),
+               "what": f"host bf16 X ({prefill_M}x4096) -> device, act quant + GEMM for both "
+                       f"weights, bf16 Y -> host; prefill M={prefill_M}"}
+
+    if rank != 0:
+        return
+    hbm, bf16_tf, bf16_sus, sm_max, peak_kind = peaks()
+    fp4_peak = 4.0 * bf16_tf            # nominal fp4 : bf16 dense ratio 9 : 2.25
+    n_solve = len(rec["solve"])
+    solve_launch_ms = solve_ms / max(n_solve, 1)
+    # solver: algorithmic work = 12 fp32 ops per element per round (two
+    # quantisations, two scale products, four reduction FMAs), ALU peak =
+    # 148 SMs x 128 fp32 lanes x max SM clock.
+    elems = sum(W.numel() for W in Wd)
+    alu_peak = 148 * 128 * sm_max * 1e6 / 1e12  # T lane-ops/s
+    solve_ops = 12.0 * elems * T * args.steps
+    solver_alu = solve_ops / (solve_ms * 1e-3) / 1e12
+    solver_gbs = T * sum(W.numel() * 2 for W in Wd) * args.steps / (solve_ms * 1e-3) / 1e9
+    g_ms = sum(t for t, _ in gemm_pre) / max(len(gemm_pre), 1)
+    g_fl = sum(f for _, f in gemm_pre) / max(len(gemm_pre), 1)
+    gemm_tf = g_fl / (g_ms * 1e-3) / 1e12
+    a_ms = sum(t for t, _ in act_pre) / max(len(act_pre), 1)
+    a_bytes = prefill_M * 4096 * (2 + 0.5 + 1.0 / 16) + prefill_M * 4
+    act_gbs = a_bytes / (a_ms * 1e-3) / 1e9
+    value = lin_flops * args.steps / (lin_ms * 1e-3) / 1e12
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, sgbs, secs, desc = oracle_sample(wl, Ws, Xs, rows=64)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc, "solver_gbs_effective": sgbs, "seconds": secs}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4(e2m1)",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "format": FMT_NAME, "weights": [list(W.shape) for W in Ws],
+                   "M": sorted(Xd), "T": T, "l2": "flushed between steps (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "solve_bcd_kernel (BCD rounds)", "bound": "alu",
+                     "achieved": solver_alu, "peak": alu_peak, "unit": "Tops/s",
+                     "frac": solver_alu / alu_peak, "traffic": None,
+                     "note": "12 algorithmic fp32 ops / element / round; peak = 148 SM x 128 "
+                             "fp32 lanes x max SM clock"},
+        "roofline_gemm": {"kernel": "w4a4_gemm_kernel", "bound": "tensor", "achieved": gemm_tf,
+                          "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
+                          "traffic": None, "shape": f"M={prefill_M} x N x K=4096",
+                          "peak_kind": f"{peak_kind} bf16 burst x 4 (nominal fp4:bf16)"},
+        "roofline_act": {"kernel": "quantize_act_kernel", "bound": "hbm", "achieved": act_gbs,
+                         "peak": hbm, "unit": "GB/s", "frac": act_gbs / hbm, "traffic": None},
+        "solver": {"gbs_effective": solver_gbs, "frac_hbm": solver_gbs / hbm,
+                   "ms_per_weight_set": solve_ms / args.steps,
+                   "definition": "T * bytes(W bf16) / solver time (tile stays on chip)"},
+        "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16_tf, "kind": peak_kind},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() and args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,117 @@
+// dq_api.cu -- extern "C" entry points of include/dq.h: argument validation
+// and dispatch.  Nothing here computes; every step runs in the kernels.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dq_internal.h"
+
+namespace {
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline bool valid_group(int f, int G) {
+  switch (f) {
+    case DQ_NVFP4: return G == 16;
+    case DQ_MXFP4:
+    case DQ_MXINT4: return G == 32;
+    case DQ_INT4: return G == 32 || G == 64 || G == 128;
+  }
+  return false;
+}
+
+inline int resolve_group(int f, int group) { return group > 0 ? group : dq_native_group((dq_format)f); }
+
+inline bool valid_dtype(int t) { return t == DQ_F32 || t == DQ_BF16; }
+
+}  // namespace
+
+extern "C" {
+
+const char* dq_status_string(int s) {
+  switch (s) {
+    case DQ_OK: return "DQ_OK";
+    case DQ_ERR_ARG: return "DQ_ERR_ARG: invalid argument";
+    case DQ_ERR_UNSUPPORTED: return "DQ_ERR_UNSUPPORTED: not implemented for these arguments";
+    case DQ_ERR_CUDA: return "DQ_ERR_CUDA: CUDA launch or runtime error";
+    case DQ_ERR_DEVICE_TIMEOUT: return "DQ_ERR_DEVICE_TIMEOUT: a bounded device wait expired";
+    case DQ_ERR_WORKSPACE: return "DQ_ERR_WORKSPACE: workspace missing or too small";
+  }
+  return "unknown dq status";
+}
+
+int dq_version(void) { return 100; }
+
+int dq_native_group(dq_format f) {
+  switch (f) {
+    case DQ_INT4: return 64;
+    case DQ_MXINT4:
+    case DQ_MXFP4: return 32;
+    case DQ_NVFP4: return 16;
+  }
+  return 0;
+}
+
+size_t dq_scales_bytes(int64_t rows, int64_t k, dq_format f, int group) {
+  const int G = resolve_group(f, group);
+  if (rows < 0 || k <= 0 || !valid_group(f, G) || k % G) return 0;
+  const int64_t S = k / G;
+  if (f == DQ_INT4) return (size_t)(rows * S * 2);
+  return (size_t)(((rows + 127) / 128) * ((S + 3) / 4) * 512);
+}
+
+size_t dq_solve_workspace_size(int T) { return T < 0 ? 0 : dq::solve_workspace_bytes(T); }
+
+int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f, int group,
+                    int T, float* r, float* c, float* s_tensor, double* mse_trace,
+                    void* workspace, size_t ws_bytes, void* stream) {
+  const int G = resolve_group(f, group);
+  if (!W || !r || !c || !s_tensor || m <= 0 || n <= 0 || T < 0 || !valid_dtype(wt) ||
+      !valid_group(f, G) || n % G || !aligned(W, 16) || !aligned(r, 4) || !aligned(c, 4) ||
+      m > (int64_t)1 << 30 || n > (int64_t)1 << 30)
+    return DQ_ERR_ARG;
+  if (!workspace || ws_bytes < dq::solve_workspace_bytes(T) || !aligned(workspace, 16))
+    return DQ_ERR_WORKSPACE;
+  return dq::solve_scales(W, wt, m, n, f, G, T, r, c, s_tensor, mse_trace, workspace,
+                          (cudaStream_t)stream);
+}
+
+int dq_quantize_weight(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f, int group,
+                       const float* r, const float* c, const float* s_tensor, uint8_t* codes,
+                       void* scales, void* stream) {
+  const int G = resolve_group(f, group);
+  if (!W || !r || !c || !codes || !scales || m <= 0 || n <= 0 || !valid_dtype(wt) ||
+      !valid_group(f, G) || n % G || !aligned(W, 16) || !aligned(codes, 16) ||
+      !aligned(scales, 16) || (f == DQ_NVFP4 && !s_tensor))
+    return DQ_ERR_ARG;
+  return dq::quantize_weight(W, wt, m, n, f, G, r, c, s_tensor, codes, scales,
+                             (cudaStream_t)stream);
+}
+
+int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, const float* c,
+                    dq_format f, int group, uint8_t* codes, void* scales, float* s_tok,
+                    void* stream) {
+  const int G = resolve_group(f, group);
+  if (!X || !codes || !scales || M <= 0 || K <= 0 || !valid_dtype(xt) || !valid_group(f, G) ||
+      K % G || !aligned(X, 16) || !aligned(codes, 16) || !aligned(scales, 16) ||
+      (f == DQ_NVFP4 && !s_tok) || (f != DQ_INT4 && K % (4 * G)) || K / G > 4096)
+    return DQ_ERR_ARG;
+  return dq::quantize_act(X, xt, M, K, c, f, G, codes, scales, s_tok, (cudaStream_t)stream);
+}
+
+int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
+                   const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
+                   dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream) {
+  if (f == DQ_INT4 || f == DQ_MXINT4) return DQ_ERR_UNSUPPORTED;
+  if (f != DQ_NVFP4 && f != DQ_MXFP4) return DQ_ERR_ARG;
+  if (!A || !sA || !B || !sB || !Y || M <= 0 || N <= 0 || K <= 0 || !valid_dtype(yt) ||
+      N % 128 || K % 256 || !aligned(A, 16) || !aligned(B, 16) || !aligned(sA, 16) ||
+      !aligned(sB, 16) || !aligned(Y, 16) || (f == DQ_NVFP4 && !s_tok) ||
+      M > ((int64_t)1 << 31) - 128 || N > ((int64_t)1 << 31) || K > ((int64_t)1 << 20))
+    return DQ_ERR_ARG;
+  return dq::w4a4_linear(A, sA, s_tok, B, sB, s_w, r_row, Y, yt, M, N, K, f,
+                         (cudaStream_t)stream);
+}
+
+int dq_device_error(int clear) { return dq::read_device_error(clear); }
+
+}  // extern "C"

@@ -1,0 +1,491 @@
+// dq_gemm.cu -- block-scaled FP4 GEMM with the DualQuant epilogue (sm_100a).
+//
+// "DualQuant", Section 4.4: at inference the layer computes
+// Q(X~) What^T Diag(alpha)^-1.  The row-block scales r = alpha^-1 are the
+// weight's native block scales, so they are applied inside the tensor-core
+// MMA together with the activation block scales; the per-token (NVFP4)
+// and per-tensor scales, and an optional per-output-row factor, are applied
+// in the epilogue.
+//
+//   Y[t, o] = s_tok[t] s_w r_row[o] sum_k a[t,k] sa[t,k/G] b[o,k] sb[o,k/G]
+//
+// Design (one CTA per SM, persistent over 128 x BN output tiles):
+//   warp 0      TMA producer: A / B code tiles (128-byte swizzled K-major,
+//               BK = 256 four-bit elements) and the matching 512-byte
+//               block-scale atoms (bulk copies), into a STAGES-deep ring.
+//   warp 1      allocates tensor memory; one thread copies the scale atoms
+//               to tensor memory (tcgen05.cp 32x128b.warpx4) and issues
+//               tcgen05.mma.kind::mxf4nvf4 / kind::mxf4 .block_scale, fp32
+//               accumulation in tensor memory; commits free the ring slots.
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (each warp its 32-lane
+//               quadrant), release it to the MMA warp, scale, convert, store.
+// Every mbarrier wait is bounded (globaltimer); on expiry the kernel records
+// DQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dq_device.cuh"
+#include "dq_internal.h"
+
+namespace dq {
+
+__device__ int g_dq_device_error = 0;
+
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 256;             // four-bit elements per k-tile (128 bytes per row)
+constexpr int BKB = BK / 2;         // bytes per row per k-tile
+constexpr int NUM_THREADS = 192;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait: returns false (and raises the abort flag) if the phase does
+// not complete within WAIT_LIMIT_NS or another role already aborted.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+      *abort_flag = 1;
+      atomicExch(&g_dq_device_error, DQ_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start, leading / stride byte
+// offsets (>> 4), version 1, layout type in bits 61-63.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)(layout & 7u) << 61;
+  return d;
+}
+constexpr uint32_t LAYOUT_SW128 = 2, LAYOUT_NONE = 0;
+
+// Instruction descriptor for kind::mxf4 / kind::mxf4nvf4 with E2M1 A and B,
+// K-major operands, M = 128.
+__host__ __device__ constexpr uint32_t idesc_fp4(int N, bool e8m0_scales) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((e8m0_scales ? 1u : 0u) << 23) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+template <int FMT>
+__device__ __forceinline__ void mma_fp4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate, uint32_t tsfa,
+                                        uint32_t tsfb) {
+  if constexpr (FMT == NVFP4) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+        : "memory");
+  }
+}
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <int FMT, int BN>
+struct Cfg {
+  static constexpr int G = (FMT == NVFP4) ? 16 : 32;
+  static constexpr int SF_PER_ROW = BK / G;                   // scales per row per k-tile
+  static constexpr int SF_ATOMS = SF_PER_ROW / 4;             // 512-byte atoms per 128 rows
+  static constexpr int A_BYTES = BM * BKB;                    // 16 KB
+  static constexpr int B_BYTES = BN * BKB;
+  static constexpr int SFA_BYTES = SF_ATOMS * 512;
+  static constexpr int SFB_BYTES = (BN / 128) * SF_ATOMS * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = (227 * 1024 - 1024 - 256) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  // tensor-memory columns: accumulator, then scale factors
+  static constexpr int SFA_COL = BN;
+  static constexpr int SFB_COL = BN + 4 * SF_ATOMS;
+  static constexpr int TMEM_USED = SFB_COL + 4 * SF_ATOMS * (BN / 128);
+  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
+  static constexpr int K_STEPS = BK / 64;                     // MMAs per k-tile (K = 64 each)
+  static_assert(STAGES >= 2, "pipeline depth");
+};
+
+template <int FMT, int BN, int YT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const uint8_t* __restrict__ sfA, const uint8_t* __restrict__ sfB,
+                 const float* __restrict__ s_tok, const float* __restrict__ s_w,
+                 const float* __restrict__ r_row, void* __restrict__ Y, int M, int N, int K) {
+  using C = Cfg<FMT, BN>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* sA = smem;
+  unsigned char* sB = sA + C::STAGES * C::A_BYTES;
+  unsigned char* sSFA = sB + C::STAGES * C::B_BYTES;
+  unsigned char* sSFB = sSFA + C::STAGES * C::SFA_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + C::STAGES * C::SFB_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_m = (M + BM - 1) / BM, tiles_n = N / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int KT = K / BK;
+  const int S4 = (K / C::G) / 4;  // scale atoms along K per 128-row block
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_base_slot)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_base_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int tm = tile % tiles_m, tn = tile / tiles_m;
+        const int m0 = tm * BM, n0 = tn * BN;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kt * BKB, m0);
+          tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kt * BKB, n0);
+          bulk_load(sSFA + stage * C::SFA_BYTES,
+                    sfA + ((size_t)(m0 / 128) * S4 + (size_t)kt * C::SF_ATOMS) * 512,
+                    C::SFA_BYTES, &full[stage]);
+#pragma unroll
+          for (int g = 0; g < BN / 128; ++g)
+            bulk_load(sSFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512,
+                      sfB + ((size_t)(n0 / 128 + g) * S4 + (size_t)kt * C::SF_ATOMS) * 512,
+                      C::SF_ATOMS * 512, &full[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // drain: every issued stage must land before the CTA may exit
+      if (ok) {
+        for (int s = 0; s < C::STAGES; ++s) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      const uint32_t idesc0 = idesc_fp4(BN, FMT != NVFP4);
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        if (!mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag)) break;
+        fence_after_sync();
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          fence_after_sync();
+          const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
+          const uint32_t sfa_base = smem_u32(sSFA + stage * C::SFA_BYTES);
+          const uint32_t sfb_base = smem_u32(sSFB + stage * C::SFB_BYTES);
+          // scale atoms -> tensor memory
+#pragma unroll
+          for (int j = 0; j < C::SF_ATOMS; ++j)
+            tmem_cp_32x128b_x4(tmem + C::SFA_COL + 4 * j,
+                               smem_desc(sfa_base + j * 512, 0, 128, LAYOUT_NONE));
+#pragma unroll
+          for (int g = 0; g < BN / 128; ++g)
+#pragma unroll
+            for (int j = 0; j < C::SF_ATOMS; ++j)
+              tmem_cp_32x128b_x4(tmem + C::SFB_COL + 4 * (BN / 128) * j + 4 * g,
+                                 smem_desc(sfb_base + (g * C::SF_ATOMS + j) * 512, 0, 128,
+                                           LAYOUT_NONE));
+#pragma unroll
+          for (int kk = 0; kk < C::K_STEPS; ++kk) {
+            // K = 64 four-bit elements = 32 bytes inside the 128-byte swizzle row
+            const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, LAYOUT_SW128);
+            const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, LAYOUT_SW128);
+            uint32_t sf_id, sfa_col, sfb_col;
+            if constexpr (FMT == NVFP4) {  // 4 scales per row per MMA: one column each
+              sf_id = 0;
+              sfa_col = C::SFA_COL + 4 * kk;
+              sfb_col = C::SFB_COL + 4 * (BN / 128) * kk;
+            } else {                        // 2 scales per row per MMA: half a column
+              sf_id = 2 * (kk & 1);
+              sfa_col = C::SFA_COL + 4 * (kk >> 1);
+              sfb_col = C::SFB_COL + 4 * (BN / 128) * (kk >> 1);
+            }
+            const uint32_t idesc = idesc0 | (sf_id << 29) | (sf_id << 4);
+            mma_fp4<FMT>(tmem, ad, bd, idesc, (kt > 0 || kk > 0) ? 1u : 0u,
+                         (tmem + sfa_col) | (sf_id << 30), (tmem + sfb_col) | (sf_id << 30));
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(acc_full);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;                 // tensor-memory lane quadrant of this warp
+    const float sw = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int tm = tile % tiles_m, tn = tile / tiles_m;
+      const int row = tm * BM + quad * 32 + lane;
+      const int n0 = tn * BN;
+      // one lane waits, the warp follows (the tensor-memory loads below are
+      // warp-collective and must never run in a partial warp)
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(acc_full, it & 1, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      fence_after_sync();
+      float rs = sw;
+      if (FMT == NVFP4 && s_tok && row < M) rs = __fmul_rn(s_tok[row], sw);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
+        if (c0 + 32 == BN) {  // accumulator fully read: hand it back to the MMA warp
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty);
+        }
+        if (row < M) {
+          float f[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            f[k] = __fmul_rn(__uint_as_float(v[k]), rs);
+            if (r_row) f[k] = __fmul_rn(f[k], __ldg(r_row + n0 + c0 + k));
+          }
+          if constexpr (YT == 1) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(Y) +
+                                                  (size_t)row * N + n0 + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t w[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                __nv_bfloat162 p = __floats2bfloat162_rn(f[8 * q + 2 * h], f[8 * q + 2 * h + 1]);
+                w[h] = *reinterpret_cast<uint32_t*>(&p);
+              }
+              dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(Y) +
+                                                    (size_t)row * N + n0 + c0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a rows x (K/2) byte matrix, box = box_rows x 128 bytes, 128-byte swizzle.
+static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t kbytes,
+                     int box_rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kbytes};
+  cuuint32_t box[2] = {(cuuint32_t)BKB, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int FMT, int BN, int YT>
+static int launch(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
+                  const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int64_t M,
+                  int64_t N, int64_t K, cudaStream_t st) {
+  using C = Cfg<FMT, BN>;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K / 2, BM) || !make_map(&tb, B, N, K / 2, BN)) return DQ_ERR_CUDA;
+  auto kern = w4a4_gemm_kernel<FMT, BN, YT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return DQ_ERR_CUDA;
+  const int64_t tiles = ((M + BM - 1) / BM) * (N / BN);
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  kern<<<grid, NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, sA, sB, s_tok, s_w, r_row, Y, (int)M,
+                                                  (int)N, (int)K);
+  return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
+}
+
+}  // namespace gemm
+
+int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
+                const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int yt,
+                int64_t M, int64_t N, int64_t K, int f, cudaStream_t st) {
+  const bool n256 = (N % 256) == 0;
+#define DQ_G(FF)                                                                                 \
+  if (n256) return yt == 1 ? gemm::launch<FF, 256, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st) \
+                           : gemm::launch<FF, 256, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st); \
+  return yt == 1 ? gemm::launch<FF, 128, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)     \
+                 : gemm::launch<FF, 128, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
+  if (f == NVFP4) { DQ_G(NVFP4); }
+  if (f == MXFP4) { DQ_G(MXFP4); }
+#undef DQ_G
+  return DQ_ERR_UNSUPPORTED;
+}
+
+int read_device_error(int clear) {
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DQ_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, g_dq_device_error, sizeof(int)) != cudaSuccess) return DQ_ERR_CUDA;
+  if (clear) {
+    int z = 0;
+    cudaMemcpyToSymbol(g_dq_device_error, &z, sizeof(int));
+  }
+  return v;
+}
+
+}  // namespace dq

@@ -1,0 +1,26 @@
+// dq_internal.h -- launchers shared between the entry points (dq_api.cu) and
+// the kernel files.  Not part of the public C ABI (include/dq.h).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dq.h"
+
+namespace dq {
+
+size_t solve_workspace_bytes(int T);
+int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int T, float* r,
+                 float* c, float* sT, double* trace, void* ws, cudaStream_t st);
+int quantize_act(const void* X, int xt, int64_t M, int64_t K, const float* c, int f, int G,
+                 uint8_t* codes, void* scales, float* s_tok, cudaStream_t st);
+int quantize_weight(const void* W, int wt, int64_t m, int64_t n, int f, int G, const float* r,
+                    const float* c, const float* sT, uint8_t* codes, void* scales,
+                    cudaStream_t st);
+int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
+                const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int yt,
+                int64_t M, int64_t N, int64_t K, int f, cudaStream_t st);
+
+// Device-side error word written by kernels whose bounded waits expire.
+int read_device_error(int clear);
+
+}  // namespace dq

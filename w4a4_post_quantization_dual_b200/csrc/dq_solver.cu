@@ -1,0 +1,460 @@
+// dq_solver.cu -- DualQuant's block-coordinate-descent scale solver on sm_100a.
+//
+// "DualQuant: Dual-scale Calibration-free Weight-and-Activation Quantization
+// for LLMs", Algorithm 1 / Section 4.3 (closed-form updates Eqs. 10 and 14,
+// Appendix B), initialisation of Section 5.3.
+//
+// With the row scale alpha being the format's native block scale, every
+// m x G column-block tile of W is an independent problem: r_ib touches only
+// tile b and every column lies in one tile.  One thread-block CLUSTER owns
+// one tile; its C CTAs split the tile's rows.  The whole iteration loop runs
+// on the device:
+//   row half-step   : each thread owns 8 contiguous columns of a row; the
+//                     G/8 threads of a row-block combine <W,R> and ||R||^2
+//                     with warp shuffles; the projected update is written to
+//                     shared memory.
+//   column half-step: per-thread column partials -> transposed shared-memory
+//                     reduction in fp64 -> per-CTA sums in cluster-visible
+//                     shared memory -> every CTA reads all C partial sums
+//                     over DSMEM in rank order (identical c in every CTA).
+// W is streamed from global memory each pass (read-only path, L1/L2 hits
+// after the first round; the tile never leaves the chip in steady state).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dq_device.cuh"
+#include "dq_internal.h"
+
+namespace dq {
+
+template <int G>
+struct SolverShape {
+  static constexpr int OPB = G / 8;            // 8-column octets per row-block
+  static constexpr int NT = (G >= 64) ? 512 : 256;
+  static constexpr int NW = NT / 32;
+  static constexpr int RPW = 32 / OPB;         // rows per warp per step
+  static constexpr int RPS = NW * RPW;         // rows per CTA per step
+};
+
+// Workspace layout (bytes): [0] u32 amax bits, [8] f64 ||W||^2, [16..] f64 err[T+1].
+struct SolverWs {
+  uint32_t amax_bits;
+  uint32_t pad;
+  double w2;
+  double err[1];
+};
+
+template <typename WT>
+__device__ __forceinline__ void load8(const WT* __restrict__ W, int64_t off, float* x);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* __restrict__ W,
+                                                     int64_t off, float* x) {
+  uint4 v = __ldg(reinterpret_cast<const uint4*>(W + off));
+  bf16x8_to_f32(v, x);
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* __restrict__ W, int64_t off, float* x) {
+  float4 a = __ldg(reinterpret_cast<const float4*>(W + off));
+  float4 b = __ldg(reinterpret_cast<const float4*>(W + off) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+// Quantise 8 fp32 arguments z to grid VALUES (E2M1 or INT4).
+template <int F>
+__device__ __forceinline__ void grid8(const float* z, float* q) {
+  if constexpr (is_int_grid(F)) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) q[k] = int4_value_rn(z[k]);
+  } else {
+    uint32_t codes = e2m1x8(z);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float2 v = __half22float2(e2m1x2_to_half2((codes >> (8 * k)) & 0xFFu));
+      q[2 * k] = v.x;
+      q[2 * k + 1] = v.y;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+__device__ __forceinline__ double ld_dsmem_f64(const double* local, uint32_t rank) {
+  uint32_t a = (uint32_t)__cvta_generic_to_shared(local), ra;
+  double v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+// Reduce V fp32 partials per thread over the CTA's threads that share an
+// octet.  Thread (oct, rslot) contributes acc[v] to value gv = oct*V + v.
+// out[gv] (shared, fp64) receives the CTA total, summed in a fixed order.
+template <int G, int V>
+__device__ __forceinline__ void cta_octet_reduce(const float* acc, float* scr, double* part,
+                                                 double* out) {
+  using S = SolverShape<G>;
+  constexpr int NV = S::OPB * V;           // values per CTA
+  constexpr int P = S::NT / NV;            // parts per value
+  constexpr int SPP = S::RPS / P;          // slots per part
+  static_assert(S::NT % NV == 0 && S::RPS % P == 0, "reduction shape");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int oct = lane % S::OPB, rslot = warp * S::RPW + lane / S::OPB;
+#pragma unroll
+  for (int v = 0; v < V; ++v) scr[(oct * V + v) * (S::RPS + 1) + rslot] = acc[v];
+  __syncthreads();
+  {
+    const int gv = tid % NV, p = tid / NV;
+    double s = 0.0;
+    const float* src = scr + gv * (S::RPS + 1) + p * SPP;
+#pragma unroll 4
+    for (int i = 0; i < SPP; ++i) s += (double)src[i];
+    part[gv * P + p] = s;
+  }
+  __syncthreads();
+  if (tid < NV) {
+    double s = 0.0;
+    for (int p = 0; p < P; ++p) s += part[tid * P + p];
+    out[tid] = s;
+  }
+  __syncthreads();
+}
+
+template <int G>
+struct SolverSmem {
+  using S = SolverShape<G>;
+  float scr[S::OPB * 16 * (S::RPS + 1)];
+  double part[S::NT];                       // NV * P == NT
+  double cpart[2][2 * G];                   // cluster-visible, double-buffered
+  float c_s[G], b_s[G];
+  double l1[G];
+};
+
+// ---------------------------------------------------------------------------
+// Initialisation kernel: c0 (Section 5.3, read as the inverse column scale
+// proportional to the column l1 norm, normalised to mean 1 per tile and
+// projected onto F_beta), the NVFP4 per-tensor amax of W diag(c0)^-1, and
+// ||W||_F^2 for the trace normalisation.
+// ---------------------------------------------------------------------------
+template <int F, int G, typename WT>
+__global__ void __launch_bounds__(SolverShape<G>::NT)
+solve_init_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, float* __restrict__ c,
+                  SolverWs* ws) {
+  using S = SolverShape<G>;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SolverSmem<G>& sm = *reinterpret_cast<SolverSmem<G>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int oct = lane % S::OPB, rslot = warp * S::RPW + lane / S::OPB;
+  const uint32_t rank = cluster_ctarank(), C = gridDim.x;
+  const int64_t b = blockIdx.y;
+  const int64_t col0 = b * G + oct * 8;
+  const int64_t row0 = (int64_t)rank * steps * S::RPS;
+
+  float acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+  float w2 = 0.0f;
+  for (int s = 0; s < steps; ++s) {
+    int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+    if (i < m) {
+      float x[8];
+      load8<WT>(W, i * n + col0, x);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        acc[k] += fabsf(x[k]);
+        w2 = fmaf(x[k], x[k], w2);
+      }
+    }
+  }
+  // ||W||^2: warp sum then one fp64 atomic per warp
+#pragma unroll
+  for (int o = 16; o; o >>= 1) w2 += __shfl_xor_sync(0xffffffffu, w2, o);
+  if (lane == 0) atomicAdd(&ws->w2, (double)w2);
+
+  cta_octet_reduce<G, 8>(acc, sm.scr, sm.part, sm.cpart[0]);  // cpart[0][j] = CTA l1 of col j
+  cluster_sync_all();
+  if (tid < G) {
+    double s = 0.0;
+    for (uint32_t q = 0; q < C; ++q) s += ld_dsmem_f64(&sm.cpart[0][tid], q);
+    sm.l1[tid] = s;
+  }
+  __syncthreads();
+  if (tid < G) {
+    double mean = 0.0;
+    for (int j = 0; j < G; ++j) mean += sm.l1[j];
+    mean /= (double)G;
+    double v = sm.l1[tid];
+    float cj = (mean > 0.0 && v > 0.0) ? proj_beta<F>((float)(v / mean)) : proj_beta<F>(1.0f);
+    sm.c_s[tid] = cj;
+    sm.b_s[tid] = __frcp_rn(cj);
+    if (rank == 0) c[b * G + tid] = cj;
+  }
+  __syncthreads();
+  if constexpr (F == NVFP4) {
+    float beta[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) beta[k] = sm.b_s[oct * 8 + k];
+    float a = 0.0f;
+    for (int s = 0; s < steps; ++s) {
+      int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+      if (i < m) {
+        float x[8];
+        load8<WT>(W, i * n + col0, x);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(__fmul_rn(x[k], beta[k])));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (lane == 0) atomicMax(&ws->amax_bits, __float_as_uint(a));
+  }
+  cluster_sync_all();  // keep this CTA's shared memory alive for DSMEM readers
+}
+
+// ---------------------------------------------------------------------------
+// Main kernel: r0 and T rounds of Algorithm 1, final error, outputs.
+// ---------------------------------------------------------------------------
+template <int F, int G, typename WT>
+__global__ void __launch_bounds__(SolverShape<G>::NT)
+solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int T,
+                 float* __restrict__ r_out, float* __restrict__ c_io, float* __restrict__ sT_out,
+                 SolverWs* ws, int want_trace) {
+  using S = SolverShape<G>;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SolverSmem<G>& sm = *reinterpret_cast<SolverSmem<G>*>(smem_raw);
+  float* r_s = reinterpret_cast<float*>(smem_raw + sizeof(SolverSmem<G>));
+  float* a_s = r_s + (size_t)steps * S::RPS;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int oct = lane % S::OPB, rslot = warp * S::RPW + lane / S::OPB;
+  const uint32_t rank = cluster_ctarank(), C = gridDim.x;
+  const int64_t b = blockIdx.y, nb = n / G;
+  const int64_t col0 = b * G + oct * 8;
+  const int64_t row0 = (int64_t)rank * steps * S::RPS;
+
+  float sT = 1.0f;
+  if constexpr (F == NVFP4) {
+    float amax = __uint_as_float(*(volatile uint32_t*)&ws->amax_bits);
+    sT = (amax > 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+    if (rank == 0 && b == 0 && tid == 0) *sT_out = sT;
+  } else {
+    if (rank == 0 && b == 0 && tid == 0) *sT_out = 1.0f;
+  }
+
+  float cc[8], beta[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    cc[k] = c_io[col0 + k];
+    beta[k] = __frcp_rn(cc[k]);
+  }
+
+  // r0: format-native absmax scale of W diag(c0)^-1 per row-block
+  for (int s = 0; s < steps; ++s) {
+    int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+    float a = 0.0f;
+    if (i < m) {
+      float x[8];
+      load8<WT>(W, i * n + col0, x);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(__fmul_rn(x[k], beta[k])));
+    }
+#pragma unroll
+    for (int o = 1; o < S::OPB; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (oct == 0) {
+      float r0 = rtn_block_scale<F>(a, sT);
+      r_s[s * S::RPS + rslot] = r0;
+      a_s[s * S::RPS + rslot] = __frcp_rn(r0);
+    }
+  }
+  __syncwarp();
+
+  for (int t = 0; t <= T; ++t) {
+    // ---- row half-step (t < T) / error at the current scales (all t) ----
+    float e_acc = 0.0f;
+    for (int s = 0; s < steps; ++s) {
+      const int lr = s * S::RPS + rslot;
+      int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+      float num = 0.0f, den = 0.0f, err = 0.0f;
+      const float rr = r_s[lr], alpha = a_s[lr];
+      if (i < m) {
+        float x[8], z[8], q[8];
+        load8<WT>(W, i * n + col0, x);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) z[k] = __fmul_rn(__fmul_rn(x[k], beta[k]), alpha);
+        grid8<F>(z, q);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float R = __fmul_rn(q[k], cc[k]);
+          num = fmaf(x[k], R, num);
+          den = fmaf(R, R, den);
+          float d = fmaf(-rr, R, x[k]);
+          err = fmaf(d, d, err);
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < S::OPB; o <<= 1) {
+        num += __shfl_xor_sync(0xffffffffu, num, o);
+        den += __shfl_xor_sync(0xffffffffu, den, o);
+        err += __shfl_xor_sync(0xffffffffu, err, o);
+      }
+      if (oct == 0) e_acc += err;
+      if (t < T && oct == 0 && i < m) {
+        float rn = (den > 0.0f) ? proj_alpha<F>(__fdiv_rn(num, den), sT) : proj_alpha<F>(1.0f, sT);
+        r_s[lr] = rn;
+        a_s[lr] = __frcp_rn(rn);
+      }
+    }
+    if (want_trace) {
+#pragma unroll
+      for (int o = 16; o; o >>= 1) e_acc += __shfl_xor_sync(0xffffffffu, e_acc, o);
+      if (lane == 0) atomicAdd(&ws->err[t], (double)e_acc);
+    }
+    if (t == T) break;
+    __syncwarp();
+
+    // ---- column half-step: re-quantise with the new r, update c ----
+    float acc[16];
+#pragma unroll
+    for (int v = 0; v < 16; ++v) acc[v] = 0.0f;
+    for (int s = 0; s < steps; ++s) {
+      const int lr = s * S::RPS + rslot;
+      int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+      if (i < m) {
+        const float rr = r_s[lr], alpha = a_s[lr];
+        float x[8], z[8], q[8];
+        load8<WT>(W, i * n + col0, x);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) z[k] = __fmul_rn(__fmul_rn(x[k], beta[k]), alpha);
+        grid8<F>(z, q);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float Sv = __fmul_rn(rr, q[k]);
+          acc[2 * k] = fmaf(Sv, x[k], acc[2 * k]);
+          acc[2 * k + 1] = fmaf(Sv, Sv, acc[2 * k + 1]);
+        }
+      }
+    }
+    const int par = t & 1;
+    cta_octet_reduce<G, 16>(acc, sm.scr, sm.part, sm.cpart[par]);
+    cluster_sync_all();
+    if (tid < G) {
+      const int j = tid, o = j >> 3, k = j & 7;
+      double sn = 0.0, sd = 0.0;
+      for (uint32_t q = 0; q < C; ++q) {
+        sn += ld_dsmem_f64(&sm.cpart[par][o * 16 + 2 * k], q);
+        sd += ld_dsmem_f64(&sm.cpart[par][o * 16 + 2 * k + 1], q);
+      }
+      float cn = (sd > 0.0) ? proj_beta<F>((float)(sn / sd)) : proj_beta<F>(1.0f);
+      sm.c_s[j] = cn;
+      sm.b_s[j] = __frcp_rn(cn);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      cc[k] = sm.c_s[oct * 8 + k];
+      beta[k] = sm.b_s[oct * 8 + k];
+    }
+  }
+
+  // outputs
+  for (int s = 0; s < steps; ++s) {
+    int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+    if (oct == 0 && i < m) r_out[i * nb + b] = r_s[s * S::RPS + rslot];
+  }
+  if (rank == 0 && tid < G) c_io[b * G + tid] = (T > 0) ? sm.c_s[tid] : c_io[b * G + tid];
+  cluster_sync_all();  // no CTA leaves while a peer may still read its cpart
+}
+
+__global__ void solve_finalize_kernel(const SolverWs* ws, int T, double* mse_trace) {
+  int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t <= T) mse_trace[t] = ws->w2 > 0.0 ? ws->err[t] / ws->w2 : 0.0;
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+template <int G>
+static size_t solver_smem_bytes(int steps) {
+  return sizeof(SolverSmem<G>) + 2 * sizeof(float) * (size_t)steps * SolverShape<G>::RPS;
+}
+
+template <int F, int G, typename WT>
+static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, float* r, float* c,
+                         float* sT, double* trace, SolverWs* ws, cudaStream_t st) {
+  using S = SolverShape<G>;
+  const WT* W = reinterpret_cast<const WT*>(Wv);
+  int steps = (int)((m + (int64_t)S::RPS * 8 - 1) / ((int64_t)S::RPS * 8));
+  if (steps < 1) steps = 1;
+  int C = (int)((m + (int64_t)S::RPS * steps - 1) / ((int64_t)S::RPS * steps));
+  const size_t sm_init = sizeof(SolverSmem<G>), sm_main = solver_smem_bytes<G>(steps);
+  if (sm_main > 227 * 1024) return DQ_ERR_UNSUPPORTED;
+
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C, (unsigned)(n / G), 1);
+  cfg.blockDim = dim3(S::NT, 1, 1);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+
+  auto kinit = solve_init_kernel<F, G, WT>;
+  auto kmain = solve_bcd_kernel<F, G, WT>;
+  if (cudaFuncSetAttribute(kinit, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_init) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(kmain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_main) !=
+          cudaSuccess)
+    return DQ_ERR_CUDA;
+  cfg.dynamicSmemBytes = sm_init;
+  if (cudaLaunchKernelEx(&cfg, kinit, W, m, n, steps, c, ws) != cudaSuccess) return DQ_ERR_CUDA;
+  cfg.dynamicSmemBytes = sm_main;
+  if (cudaLaunchKernelEx(&cfg, kmain, W, m, n, steps, T, r, c, sT, ws, trace ? 1 : 0) !=
+      cudaSuccess)
+    return DQ_ERR_CUDA;
+  if (trace) {
+    solve_finalize_kernel<<<(T + 1 + 127) / 128, 128, 0, st>>>(ws, T, trace);
+    if (cudaGetLastError() != cudaSuccess) return DQ_ERR_CUDA;
+  }
+  return DQ_OK;
+}
+
+template <typename WT>
+static int dispatch_solver(const void* W, int64_t m, int64_t n, int f, int G, int T, float* r,
+                           float* c, float* sT, double* trace, SolverWs* ws, cudaStream_t st) {
+  switch (f) {
+    case NVFP4: return launch_solver<NVFP4, 16, WT>(W, m, n, T, r, c, sT, trace, ws, st);
+    case MXFP4: return launch_solver<MXFP4, 32, WT>(W, m, n, T, r, c, sT, trace, ws, st);
+    case MXINT4: return launch_solver<MXINT4, 32, WT>(W, m, n, T, r, c, sT, trace, ws, st);
+    case INT4:
+      if (G == 32) return launch_solver<INT4, 32, WT>(W, m, n, T, r, c, sT, trace, ws, st);
+      if (G == 64) return launch_solver<INT4, 64, WT>(W, m, n, T, r, c, sT, trace, ws, st);
+      return launch_solver<INT4, 128, WT>(W, m, n, T, r, c, sT, trace, ws, st);
+  }
+  return DQ_ERR_ARG;
+}
+
+size_t solve_workspace_bytes(int T) {
+  size_t b = 16 + 8 * (size_t)(T + 1);
+  return (b + 255) & ~(size_t)255;
+}
+
+int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int T, float* r,
+                 float* c, float* sT, double* trace, void* ws, cudaStream_t st) {
+  if (cudaMemsetAsync(ws, 0, solve_workspace_bytes(T), st) != cudaSuccess) return DQ_ERR_CUDA;
+  SolverWs* w = reinterpret_cast<SolverWs*>(ws);
+  if (wt == 1)
+    return dispatch_solver<__nv_bfloat16>(W, m, n, f, G, T, r, c, sT, trace, w, st);
+  return dispatch_solver<float>(W, m, n, f, G, T, r, c, sT, trace, w, st);
+}
+
+}  // namespace dq
