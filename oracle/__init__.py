@@ -325,14 +325,15 @@ def linear(A, sA, s_tok, B, sB, s_W, M, N, K, fmt, r_row=None):
     return Y
 
 
-def linear_rows(A, sA, s_tok, B, sB, s_W, rows, M, N, K, fmt, r_row=None):
-    """Selected output rows of linear(), for sampled checks at full size."""
-    G = NATIVE_GROUP[fmt]
-    rows = np.asarray(rows)
+def dequant_rows(packed, sf, row_idx, K, fmt, G=None):
+    """Dequantised rows `row_idx` (fp64, len(row_idx) x K) of an operand whose
+    codes are (R, K/2) bytes and whose scales are in the GEMM layout."""
+    G = G or NATIVE_GROUP[fmt]
+    rows = np.asarray(row_idx)
     S = K // G
-    Asub = np.asarray(A).reshape(M, K // 2)[rows]
-    q = elem_value_table(fmt)[unpack_codes(Asub, K)]
-    sf = np.asarray(sA, np.uint8).reshape(-1)
+    P = np.asarray(packed, np.uint8).reshape(-1, K // 2)[rows]
+    q = elem_value_table(fmt)[unpack_codes(P, K)]
+    sfa = np.asarray(sf, np.uint8).reshape(-1)
     S4 = (S + 3) // 4
     rr = rows[:, None]
     ss = np.arange(S)[None, :]
@@ -341,13 +342,21 @@ def linear_rows(A, sA, s_tok, B, sB, s_W, rows, M, N, K, fmt, r_row=None):
         tab = np.array([e4m3_value(k) for k in range(256)], np.float64)
     else:
         tab = np.array([e8m0_value(k) if k < 255 else np.nan for k in range(256)], np.float64)
-    a = q * np.repeat(tab[sf[off]], G, axis=1)
+    return q * np.repeat(tab[sfa[off]], G, axis=1)
+
+
+def linear_rows(A, sA, s_tok, B, sB, s_W, rows, M, N, K, fmt, r_row=None, cols=None):
+    """Output rows `rows` (and columns `cols`, default all) of linear(), for
+    sampled checks at full size."""
+    rows = np.asarray(rows)
+    cols = np.arange(N) if cols is None else np.asarray(cols)
+    a = dequant_rows(A, sA, rows, K, fmt)
     if fmt == NVFP4:
         a = a * np.asarray(s_tok, np.float64)[rows][:, None]
-    b = dequant(B, sB, N, K, fmt, G)
+    b = dequant_rows(B, sB, cols, K, fmt)
     Y = a @ b.T
     if fmt == NVFP4:
         Y = Y * float(s_W)
     if r_row is not None:
-        Y = Y * np.asarray(r_row, np.float64)[None, :]
+        Y = Y * np.asarray(r_row, np.float64)[cols][None, :]
     return Y

@@ -188,27 +188,36 @@ double oracle_bf16_proj(double u) {
 /* per-tensor fp32 scale s_T fixed at initialisation).                 */
 /* ------------------------------------------------------------------ */
 
+/* Decision precision.  The paper fixes no precision for the projection
+ * step, so the scale decision is taken on the fp32 value of the updated
+ * inverse scale (the kernel's precision): u is rounded once to fp32, and for
+ * NVFP4 the ratio u / s_T is one fp32 division.  Accumulations that produce
+ * u stay fp64. */
+
 /* Row-scale projection: returns r in F_alpha (as float; exactly
  * representable for every format). */
 static float proj_alpha(int fmt, double u, float s_T) {
+  float u32 = (float)u;
   switch (fmt) {
     case F_NVFP4: {
-      double v = oracle_e4m3_value(oracle_ue4m3_proj(u / (double)s_T));
-      return (float)((double)s_T * v) ; /* rounded once to fp32 */
+      volatile float x = u32 / s_T;
+      double v = oracle_e4m3_value(oracle_ue4m3_proj((double)x));
+      return (float)((double)s_T * v); /* one fp32 rounding of s_T * v */
     }
     case F_MXFP4:
-    case F_MXINT4: return (float)oracle_e8m0_value(oracle_e8m0_proj(u));
-    default: return (float)oracle_bf16_proj(u);
+    case F_MXINT4: return (float)oracle_e8m0_value(u32 > 0.0f ? oracle_e8m0_proj((double)u32) : 0);
+    default: return (float)oracle_bf16_proj((double)u32);
   }
 }
 
-/* Column-scale projection: c in F_beta. */
+/* Column-scale projection: c in F_beta (decision on the fp32 value of u). */
 static float proj_beta(int fmt, double u) {
+  float u32 = (float)u;
   switch (fmt) {
-    case F_NVFP4: return (float)oracle_e4m3_value(oracle_ue4m3_proj(u));
+    case F_NVFP4: return (float)oracle_e4m3_value(oracle_ue4m3_proj((double)u32));
     case F_MXFP4:
-    case F_MXINT4: return (float)oracle_e8m0_value(oracle_e8m0_proj(u));
-    default: return (float)oracle_bf16_proj(u);
+    case F_MXINT4: return (float)oracle_e8m0_value(u32 > 0.0f ? oracle_e8m0_proj((double)u32) : 0);
+    default: return (float)oracle_bf16_proj((double)u32);
   }
 }
 
@@ -276,7 +285,10 @@ float oracle_tensor_scale(const float* W, int64_t m, int64_t n, const float* c) 
 static float rtn_block_scale(int fmt, float a, float s_T) {
   if (a == 0.0f) return proj_alpha(fmt, 1.0, s_T);  /* degenerate convention */
   switch (fmt) {
-    case F_NVFP4: return proj_alpha(fmt, (double)a / 6.0, s_T);
+    case F_NVFP4: {
+      volatile float q = a / 6.0f;
+      return proj_alpha(fmt, (double)q, s_T);
+    }
     case F_MXFP4:
     case F_MXINT4: {
       /* OCP MX: X = 2^(floor(log2 amax) - emax_elem), emax_elem = 2. */
@@ -287,7 +299,10 @@ static float rtn_block_scale(int fmt, float a, float s_T) {
       if (k > 127) k = 127;
       return (float)ldexp(1.0, k);
     }
-    default: return (float)oracle_bf16_proj((double)a / 7.0);
+    default: {
+      volatile float q = a / 7.0f;
+      return proj_alpha(fmt, (double)q, s_T);
+    }
   }
 }
 
