@@ -19,7 +19,6 @@ The solver is reported beside it as effective streaming GB/s
 import argparse
 import json
 import os
-import subprocess
 import sys
 import threading
 import time
@@ -55,88 +54,112 @@ def workload_inputs():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock and clock-event reasons sampled through NVML (read-only)
+    every 5 ms while the timed region runs."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, index):
-        self.index, self.proc, self.lines = index, None, []
+    def __init__(self, cuda_index):
+        self.samples, self.reasons, self.err = [], set(), None
+        self.stop_ev = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(cuda_index).uuid).lower().replace("gpu-", "")
+            self.h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = (u.decode() if isinstance(u, bytes) else u).lower().replace("gpu-", "")
+                if u == uuid:
+                    self.h = h
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 -- no NVML: report it, never fail the bench
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception as e:  # noqa: BLE001
+                self.err = repr(e)
+                return
+            time.sleep(0.005)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+        if self.err is None:
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": float(np.median(sm)) if sm else None,
-                "sm_max_mhz": float(max(mx)) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.err is not None and not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        self.stop_ev.set()
+        self.t.join(timeout=2)
+        return {"sm_mhz": float(np.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": float(self.max_mhz), "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "NVML"}
 
 
 # ---------------------------------------------------------------------------
 # Reference arm / CPU baseline: the oracle as it stands, on host cores.
 # ---------------------------------------------------------------------------
-def oracle_sample(wl, Ws, Xs, rows=64):
-    """Bounded oracle run on the same workload: the inference path (act
-    quant + dequantised fp64 matmul) on `rows` token rows of the M=4096
-    activations for both weights, plus Algorithm 1 on one 4096x16 tile.
-    Returns (linear TFLOP/s, solver GB/s effective, seconds, description)."""
+_ORACLE_PACKED = {}
+
+
+def oracle_prepare(wl, Ws):
+    """Offline part for the oracle legs: Algorithm 1 initial scales of every
+    tile (T = 0) and the packed weights, computed once and cached."""
     import oracle as O
-    fmt, G, T = O.NVFP4, 16, wl["T"]
-    t0 = time.perf_counter()
-    flops = 0.0
-    t_lin = 0.0
-    t_sol = 0.0
-    solved_bytes = 0.0
+    if not _ORACLE_PACKED:
+        for i, W in enumerate(Ws):
+            res = O.solve(W, O.NVFP4, 16, 0)
+            B, sB = O.pack_weight(W, O.NVFP4, 16, res["r"], res["c"], res["s_T"])
+            _ORACLE_PACKED[i] = (res, B, sB)
+    return _ORACLE_PACKED
+
+
+def oracle_linear_sample(wl, Ws, Xs, rows):
+    """The oracle's inference path -- activation rescale+quantise and the
+    dequantised fp64 matmul -- on `rows` token rows of the M=4096 activations,
+    for both weights.  Returns (TFLOP/s, seconds)."""
+    import oracle as O
+    packed = oracle_prepare(wl, Ws)
     X = Xs[max(Xs)][:rows]
-    for W in Ws:
+    flops, t0 = 0.0, time.perf_counter()
+    for i, W in enumerate(Ws):
         N, K = W.shape
-        ts = time.perf_counter()
-        res = O.solve(W, fmt, G, T, tiles=[0])
-        t_sol += time.perf_counter() - ts
-        solved_bytes += T * W.shape[0] * G * 2.0
-        tl = time.perf_counter()
-        A, sA, st = O.quantize_act(X, res["c"], fmt, G)
-        B, sB = O.pack_weight(W, fmt, G, res["r"], res["c"], res["s_T"])
-        O.linear(A, sA, st, B, sB, res["s_T"], rows, N, K, fmt)
-        t_lin += time.perf_counter() - tl
+        res, B, sB = packed[i]
+        A, sA, st = O.quantize_act(X, res["c"], O.NVFP4, 16)
+        O.linear(A, sA, st, B, sB, res["s_T"], rows, N, K, O.NVFP4)
         flops += 2.0 * rows * N * K
-    desc = (f"oracle: act quant + weight pack + fp64 dequantised matmul on {rows} of 4096 "
-            f"token rows for both weights; Algorithm 1 (T={T}) on one 4096x16 tile per weight")
-    return flops / t_lin / 1e12, solved_bytes / t_sol / 1e9, time.perf_counter() - t0, desc
+    dt = time.perf_counter() - t0
+    return flops / dt / 1e12, dt
+
+
+def oracle_solver_sample(wl, Ws):
+    """Algorithm 1 (T = 50) on one 4096 x 16 tile of the first weight.
+    Returns effective GB/s (T * tile bytes / time) and seconds."""
+    import oracle as O
+    W, T = Ws[0], wl["T"]
+    t0 = time.perf_counter()
+    O.solve(W, O.NVFP4, 16, T, tiles=[0])
+    dt = time.perf_counter() - t0
+    return T * W.shape[0] * 16 * 2.0 / dt / 1e9, dt
+
+
+LINEAR_SAMPLE_DESC = ("oracle (C + numpy fp64): activation rescale+quantise and dequantised "
+                      "matmul on {rows} of the 4096 token rows, both weights (weights packed once "
+                      "beforehand, outside the timing)")
 
 
 def blas_threads():
@@ -151,15 +174,16 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     wl, Ws, Xs = workload_inputs()
+    oracle_prepare(wl, Ws)
     for _ in range(args.warmup):
-        oracle_sample(wl, Ws, Xs, rows=16)
-    vals = []
-    t0 = time.perf_counter()
+        oracle_linear_sample(wl, Ws, Xs, rows=16)
+    flops_t, dt = 0.0, 0.0
     for _ in range(args.steps):
-        v, _, _, desc = oracle_sample(wl, Ws, Xs, rows=16)
-        vals.append(v)
-    dt = time.perf_counter() - t0
-    value = float(np.mean(vals))
+        v, d = oracle_linear_sample(wl, Ws, Xs, rows=16)
+        flops_t += v * d
+        dt += d
+    value = flops_t / dt
+    desc = LINEAR_SAMPLE_DESC.format(rows=16)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -167,7 +191,7 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "format": FMT_NAME, "sample_rows": 16},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
-                         "kind": "oracle", "sample": desc.replace("64 of", "16 of")},
+                         "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -337,9 +361,13 @@ def run_ours(args, rank, world, local_rank):
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, sgbs, secs, desc = oracle_sample(wl, Ws, Xs, rows=64)
+        oracle_prepare(wl, Ws)
+        v, secs = oracle_linear_sample(wl, Ws, Xs, rows=64)
+        sgbs, ssecs = oracle_solver_sample(wl, Ws)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": desc, "solver_gbs_effective": sgbs, "seconds": secs}
+               "sample": LINEAR_SAMPLE_DESC.format(rows=64), "seconds": secs,
+               "solver": {"gbs_effective": sgbs, "seconds": ssecs,
+                          "sample": "Algorithm 1, T=50, one 4096x16 tile, single thread"}}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -375,7 +403,7 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

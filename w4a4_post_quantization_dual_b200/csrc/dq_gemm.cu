@@ -188,6 +188,42 @@ struct Cfg {
   static_assert(STAGES >= 2, "pipeline depth");
 };
 
+// bf16 epilogue of one 128 x BN tile for one thread (one accumulator row):
+// drain the whole row from tensor memory into packed bf16 registers, hand the
+// accumulator back to the MMA warp, then store.
+template <int BN, bool ROWF>
+__device__ __forceinline__ void epilogue_bf16(uint32_t tmem, int quad, int lane, int row, int M,
+                                              int N, int n0, float rs,
+                                              const float* __restrict__ r_row, void* Y,
+                                              uint64_t* acc_empty) {
+  uint32_t pk[BN / 2];
+#pragma unroll
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
+#pragma unroll
+    for (int k = 0; k < 32; k += 2) {
+      float f0 = __fmul_rn(__uint_as_float(v[k]), rs);
+      float f1 = __fmul_rn(__uint_as_float(v[k + 1]), rs);
+      if constexpr (ROWF) {
+        f0 = __fmul_rn(f0, __ldg(r_row + n0 + c0 + k));
+        f1 = __fmul_rn(f1, __ldg(r_row + n0 + c0 + k + 1));
+      }
+      __nv_bfloat162 p2 = __floats2bfloat162_rn(f0, f1);
+      pk[(c0 + k) / 2] = *reinterpret_cast<uint32_t*>(&p2);
+    }
+  }
+  fence_before_sync();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(acc_empty);
+  if (row < M) {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(Y) + (size_t)row * N + n0);
+#pragma unroll
+    for (int q = 0; q < BN / 8; ++q)
+      dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  }
+}
+
 template <int FMT, int BN, int YT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -345,36 +381,28 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       fence_after_sync();
       float rs = sw;
       if (FMT == NVFP4 && s_tok && row < M) rs = __fmul_rn(s_tok[row], sw);
+      if constexpr (YT == 1) {
+        if (r_row)
+          epilogue_bf16<BN, true>(tmem, quad, lane, row, M, N, n0, rs, r_row, Y, acc_empty);
+        else
+          epilogue_bf16<BN, false>(tmem, quad, lane, row, M, N, n0, rs, r_row, Y, acc_empty);
+      } else {
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
-        if (c0 + 32 == BN) {  // accumulator fully read: hand it back to the MMA warp
-          fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
-        }
-        if (row < M) {
-          float f[32];
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            f[k] = __fmul_rn(__uint_as_float(v[k]), rs);
-            if (r_row) f[k] = __fmul_rn(f[k], __ldg(r_row + n0 + c0 + k));
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
+          if (c0 + 32 == BN) {  // accumulator fully read: hand it back to the MMA warp
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
           }
-          if constexpr (YT == 1) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(Y) +
-                                                  (size_t)row * N + n0 + c0);
+          if (row < M) {
+            float f[32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t w[4];
-#pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                __nv_bfloat162 p = __floats2bfloat162_rn(f[8 * q + 2 * h], f[8 * q + 2 * h + 1]);
-                w[h] = *reinterpret_cast<uint32_t*>(&p);
-              }
-              dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int k = 0; k < 32; ++k) {
+              f[k] = __fmul_rn(__uint_as_float(v[k]), rs);
+              if (r_row) f[k] = __fmul_rn(f[k], __ldg(r_row + n0 + c0 + k));
             }
-          } else {
             float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(Y) +
                                                     (size_t)row * N + n0 + c0);
 #pragma unroll

@@ -156,6 +156,139 @@ quantize_act_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int64_t K
 }
 
 // ---------------------------------------------------------------------------
+// Activation quantiser for the tensor-core formats (G <= 32).  Each thread
+// owns BPT column blocks for the whole launch (their column scales c stay in
+// registers); a CTA iteration covers R rows, so R rows of loads are in flight
+// per thread and the per-token reduction costs one barrier per R rows.
+// ---------------------------------------------------------------------------
+template <int F, int G, typename XT, int BPT, int R>
+__global__ void __launch_bounds__(512)
+quantize_act_rows_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int64_t K,
+                         const float* __restrict__ c, uint8_t* __restrict__ codes,
+                         uint8_t* __restrict__ scales, float* __restrict__ s_tok) {
+  constexpr int PIECES = G * (int)sizeof(XT) / 16;   // 16-byte loads per block
+  __shared__ float red[2][R][16];
+  const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int NWARP = (NT + 31) >> 5;
+  const int64_t S = K / G;
+  float cv[BPT][G];
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    const int64_t s = tid + (int64_t)j * NT;
+#pragma unroll
+    for (int k = 0; k < G; k += 4) {
+      float4 v = (c && s < S) ? __ldg(reinterpret_cast<const float4*>(c + s * G + k))
+                              : make_float4(1.f, 1.f, 1.f, 1.f);
+      cv[j][k] = v.x; cv[j][k + 1] = v.y; cv[j][k + 2] = v.z; cv[j][k + 3] = v.w;
+    }
+  }
+  // element k of a block held as raw 16-byte pieces
+  auto elem = [&](const uint4 (&raw)[PIECES], int k) -> float {
+    if constexpr (sizeof(XT) == 2) {
+      const uint4& v = raw[k / 8];
+      const int w = (k % 8) / 2;
+      const uint32_t u = w == 0 ? v.x : (w == 1 ? v.y : (w == 2 ? v.z : v.w));
+      return (k & 1) ? __uint_as_float(u & 0xFFFF0000u) : __uint_as_float(u << 16);
+    } else {
+      const uint4& v = raw[k / 4];
+      const int w = k % 4;
+      return __uint_as_float(w == 0 ? v.x : (w == 1 ? v.y : (w == 2 ? v.z : v.w)));
+    }
+  };
+  int it = 0;
+  for (int64_t t0 = (int64_t)blockIdx.x * R; t0 < Mpad; t0 += (int64_t)gridDim.x * R, ++it) {
+    uint4 raw[R][BPT][PIECES];
+    float ab[R][BPT];
+    float amax[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t t = t0 + r;
+#pragma unroll
+      for (int j = 0; j < BPT; ++j) {
+        const int64_t s = tid + (int64_t)j * NT;
+#pragma unroll
+        for (int u = 0; u < PIECES; ++u)
+          raw[r][j][u] = (t < M && s < S)
+                             ? __ldcs(reinterpret_cast<const uint4*>(X + t * K + s * G) + u)
+                             : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      amax[r] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < BPT; ++j) {
+        float a = 0.0f;
+#pragma unroll
+        for (int k = 0; k < G; ++k) a = fmaxf(a, fabsf(__fmul_rn(elem(raw[r][j], k), cv[j][k])));
+        ab[r][j] = a;
+        amax[r] = fmaxf(amax[r], a);
+      }
+    }
+    float st[R];
+    if constexpr (F == NVFP4) {
+      const int par = it & 1;  // double-buffered: one barrier per iteration
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float v = amax[r];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) red[par][r][warp] = v;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float v = 0.0f;
+        for (int w = 0; w < NWARP; ++w) v = fmaxf(v, red[par][r][w]);
+        st[r] = __fdiv_rn(v, 2688.0f);
+        if (tid == 0 && t0 + r < M) s_tok[t0 + r] = st[r];
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t t = t0 + r;
+#pragma unroll
+      for (int j = 0; j < BPT; ++j) {
+        const int64_t s = tid + (int64_t)j * NT;
+        uint32_t byte = 0;
+        if (t < M && s < S) {
+          float inv = 0.0f;
+          bool zero = true;
+          if constexpr (F == NVFP4) {
+            if (st[r] > 0.0f) byte = ue4m3_rn(__fdiv_rn(ab[r][j], __fmul_rn(6.0f, st[r])));
+            const float sblk = __fmul_rn(ue4m3_value(byte), st[r]);
+            zero = (sblk == 0.0f);
+            inv = zero ? 0.0f : __frcp_rn(sblk);
+          } else {
+            int e = -127;
+            if (ab[r][j] > 0.0f) {
+              e = ilog2f(ab[r][j]) - 2;
+              e = e < -127 ? -127 : (e > 127 ? 127 : e);
+              zero = false;
+            }
+            byte = (uint32_t)(e + 127);
+            inv = pow2f(-e);
+          }
+          float z[G];
+#pragma unroll
+          for (int k = 0; k < G; ++k)
+            z[k] = zero ? 0.0f : __fmul_rn(__fmul_rn(elem(raw[r][j], k), cv[j][k]), inv);
+          store_codes<F, G>(codes + t * (K / 2) + s * (G / 2), z);
+        }
+        // scale bytes of 4 consecutive blocks share one 32-bit word of the
+        // layout: gather them in the lane whose block index is a multiple of 4
+        const uint32_t b1 = __shfl_down_sync(0xffffffffu, byte, 1);
+        const uint32_t b2 = __shfl_down_sync(0xffffffffu, byte, 2);
+        const uint32_t b3 = __shfl_down_sync(0xffffffffu, byte, 3);
+        if ((s & 3) == 0 && s < S && t < Mpad)
+          *reinterpret_cast<uint32_t*>(scales + sf_offset(t, s, S)) =
+              byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Weight packer: one thread per (row, block).
 // ---------------------------------------------------------------------------
 template <int F, int G, typename WT>
@@ -224,9 +357,27 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
   int NT = (int)((S < 1024 ? S : 1024) + 31) / 32 * 32;
   const int bpt = (int)((S + NT - 1) / NT);
   const int64_t Mpad = (F == INT4) ? M : ((M + 127) / 128) * 128;
+  const XT* Xp = reinterpret_cast<const XT*>(X);
+  if constexpr (F != INT4) {
+    // rows kernel: R rows per CTA iteration, BPT blocks per thread
+    constexpr int R = (G == 16) ? 4 : 2;
+    NT = (int)((S < 512 ? S : 512) + 31) / 32 * 32;
+    const int bpt = (int)((S + NT - 1) / NT);
+    int64_t grid = (int64_t)num_sms() * (2048 / NT);
+    const int64_t groups = (Mpad + R - 1) / R;
+    if (grid > groups) grid = groups;
+    if (bpt == 1)
+      quantize_act_rows_kernel<F, G, XT, 1, R><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
+    else if (bpt == 2)
+      quantize_act_rows_kernel<F, G, XT, 2, R / 2><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
+    else if (bpt <= 4)
+      quantize_act_rows_kernel<F, G, XT, 4, 1><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
+    else
+      return DQ_ERR_UNSUPPORTED;
+    return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
+  }
   int64_t grid = (int64_t)num_sms() * (2048 / NT);
   if (grid > Mpad) grid = Mpad;
-  const XT* Xp = reinterpret_cast<const XT*>(X);
   switch (bpt) {
     case 1: quantize_act_kernel<F, G, XT, 1><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok); break;
     case 2: quantize_act_kernel<F, G, XT, 2><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok); break;

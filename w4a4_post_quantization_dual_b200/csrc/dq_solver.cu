@@ -17,8 +17,10 @@
 //                     reduction in fp64 -> per-CTA sums in cluster-visible
 //                     shared memory -> every CTA reads all C partial sums
 //                     over DSMEM in rank order (identical c in every CTA).
-// W is streamed from global memory each pass (read-only path, L1/L2 hits
-// after the first round; the tile never leaves the chip in steady state).
+// Each CTA stages its rows of the tile in shared memory once (clusters of up
+// to 16 CTAs keep the share <= 96 KB) and reads them from there in every
+// pass; tiles too tall for that stream their rows through the read-only
+// global path (L1 / L2 hits after the first round).  HBM sees W about once.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -220,17 +222,108 @@ solve_init_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, flo
 
 // ---------------------------------------------------------------------------
 // Main kernel: r0 and T rounds of Algorithm 1, final error, outputs.
+//
+// WSMEM: the CTA's rows of the tile are staged once in shared memory and
+// every pass reads them from there; otherwise they are re-read through the
+// read-only global path (L1 / L2).  Element arithmetic uses the packed
+// fp32x2 instructions of sm_100 (each lane of a pair is an ordinary
+// correctly-rounded fp32 operation, so the quantiser argument
+// (w * beta) * alpha is bit-identical to the scalar definition).
+// TRACE: accumulate the reconstruction error for the MSE trace.
 // ---------------------------------------------------------------------------
-template <int F, int G, typename WT>
+template <int F>
+struct RowProj {
+  // projected row scale r in F_alpha and alpha = fl(1/r) for an update u
+  __device__ __forceinline__ static void apply(float u, float inv_sT, const float* rtab,
+                                               const float* atab, float sT, float& r, float& a) {
+    if constexpr (F == NVFP4) {
+      uint32_t b = ue4m3_rn(u * inv_sT);
+      b = b ? b : 1u;
+      r = rtab[b];
+      a = atab[b];
+    } else if constexpr (F == MXFP4 || F == MXINT4) {
+      uint32_t bits = __float_as_uint(u);
+      int e = (int)((bits >> 23) & 0xFFu);
+      int k = e ? e - 127 + ((bits & 0x7FFFFFu) >= 0x400000u ? 1 : 0)
+                : ((u >= 8.816207631167156e-39f) ? -126 : -127);
+      k = k < -127 ? -127 : (k > 127 ? 127 : k);
+      r = pow2f(k);
+      a = pow2f(-k);
+    } else {
+      r = proj_bf16(u);
+      a = __frcp_rn(r);
+    }
+  }
+};
+
+template <int F>
+__device__ __forceinline__ void grid8_packed(const float2* z, float2* q) {
+  if constexpr (is_int_grid(F)) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      q[k].x = rintf(fminf(fmaxf(z[k].x, -8.0f), 7.0f));
+      q[k].y = rintf(fminf(fmaxf(z[k].y, -8.0f), 7.0f));
+    }
+  } else {
+    uint32_t codes;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(codes)
+        : "f"(z[0].x), "f"(z[0].y), "f"(z[1].x), "f"(z[1].y), "f"(z[2].x), "f"(z[2].y),
+          "f"(z[3].x), "f"(z[3].y));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) q[k] = __half22float2(e2m1x2_to_half2((codes >> (8 * k)) & 0xFFu));
+  }
+}
+
+template <typename WT>
+__device__ __forceinline__ void unpack8(const WT* p, float2* x);
+template <>
+__device__ __forceinline__ void unpack8<__nv_bfloat16>(const __nv_bfloat16* p, float2* x) {
+  uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+template <>
+__device__ __forceinline__ void unpack8<float>(const float* p, float2* x) {
+  float4 a = reinterpret_cast<const float4*>(p)[0];
+  float4 b = reinterpret_cast<const float4*>(p)[1];
+  x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w);
+  x[2] = make_float2(b.x, b.y); x[3] = make_float2(b.z, b.w);
+}
+template <typename WT>
+__device__ __forceinline__ void unpack8_global(const WT* __restrict__ p, float2* x) {
+  if constexpr (sizeof(WT) == 2) {
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+  } else {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w);
+    x[2] = make_float2(b.x, b.y); x[3] = make_float2(b.z, b.w);
+  }
+}
+
+template <int F, int G, typename WT, bool WSMEM, bool TRACE>
 __global__ void __launch_bounds__(SolverShape<G>::NT)
 solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int T,
                  float* __restrict__ r_out, float* __restrict__ c_io, float* __restrict__ sT_out,
-                 SolverWs* ws, int want_trace) {
+                 SolverWs* ws) {
   using S = SolverShape<G>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SolverSmem<G>& sm = *reinterpret_cast<SolverSmem<G>*>(smem_raw);
   float* r_s = reinterpret_cast<float*>(smem_raw + sizeof(SolverSmem<G>));
   float* a_s = r_s + (size_t)steps * S::RPS;
+  float* rtab = a_s + (size_t)steps * S::RPS;       // NVFP4: r and alpha of every scale byte
+  float* atab = rtab + 128;
+  WT* wch = reinterpret_cast<WT*>(atab + 128);      // staged rows (WSMEM)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int oct = lane % S::OPB, rslot = warp * S::RPW + lane / S::OPB;
@@ -238,32 +331,60 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
   const int64_t b = blockIdx.y, nb = n / G;
   const int64_t col0 = b * G + oct * 8;
   const int64_t row0 = (int64_t)rank * steps * S::RPS;
+  const int rows_cta = steps * S::RPS;
 
   float sT = 1.0f;
   if constexpr (F == NVFP4) {
     float amax = __uint_as_float(*(volatile uint32_t*)&ws->amax_bits);
     sT = (amax > 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
-    if (rank == 0 && b == 0 && tid == 0) *sT_out = sT;
-  } else {
-    if (rank == 0 && b == 0 && tid == 0) *sT_out = 1.0f;
+    if (tid < 128) {
+      float rv = __fmul_rn(sT, ue4m3_value(tid ? (uint32_t)tid : 1u));
+      rtab[tid] = rv;
+      atab[tid] = __frcp_rn(rv);
+    }
   }
+  if (rank == 0 && b == 0 && tid == 0) *sT_out = sT;
+  const float inv_sT = __frcp_rn(sT);
 
-  float cc[8], beta[8];
+  if constexpr (WSMEM) {
+    // stage rows [row0, row0 + rows_cta) x columns [b*G, b*G+G) (zeros past m)
+    constexpr int V = 16 / sizeof(WT);                // elements per 16-byte piece
+    constexpr int PPR = G / V;                        // pieces per row
+    for (int p = tid; p < rows_cta * PPR; p += S::NT) {
+      const int lr = p / PPR, pc = p % PPR;
+      const int64_t i = row0 + lr;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (i < m) v = __ldg(reinterpret_cast<const uint4*>(W + i * n + b * G) + pc);
+      reinterpret_cast<uint4*>(wch + (size_t)lr * G)[pc] = v;
+    }
+    __syncthreads();
+  }
+  auto load_x = [&](int s, float2* x) {
+    const int lr = s * S::RPS + rslot;
+    if constexpr (WSMEM) unpack8<WT>(wch + (size_t)lr * G + oct * 8, x);
+    else unpack8_global<WT>(W + (row0 + lr) * n + col0, x);
+  };
+
+  float2 cc[4], beta[4];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    cc[k] = c_io[col0 + k];
-    beta[k] = __frcp_rn(cc[k]);
+  for (int k = 0; k < 4; ++k) {
+    cc[k] = make_float2(c_io[col0 + 2 * k], c_io[col0 + 2 * k + 1]);
+    beta[k] = make_float2(__frcp_rn(cc[k].x), __frcp_rn(cc[k].y));
   }
 
-  // r0: format-native absmax scale of W diag(c0)^-1 per row-block
+  // r0: format-native absmax scale of W diag(c0)^-1 per row-block (IEEE
+  // arithmetic: the same fp32 decisions as the oracle's initialisation)
   for (int s = 0; s < steps; ++s) {
-    int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+    const int64_t i = row0 + (int64_t)s * S::RPS + rslot;
     float a = 0.0f;
     if (i < m) {
-      float x[8];
-      load8<WT>(W, i * n + col0, x);
+      float2 x[4];
+      load_x(s, x);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(__fmul_rn(x[k], beta[k])));
+      for (int k = 0; k < 4; ++k) {
+        float2 p = __fmul2_rn(x[k], beta[k]);
+        a = fmaxf(a, fmaxf(fabsf(p.x), fabsf(p.y)));
+      }
     }
 #pragma unroll
     for (int o = 1; o < S::OPB; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
@@ -276,42 +397,50 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
   __syncwarp();
 
   for (int t = 0; t <= T; ++t) {
-    // ---- row half-step (t < T) / error at the current scales (all t) ----
+    // ---- row half-step (t < T) / error at the current scales ----
     float e_acc = 0.0f;
-    for (int s = 0; s < steps; ++s) {
-      const int lr = s * S::RPS + rslot;
-      int64_t i = row0 + (int64_t)s * S::RPS + rslot;
-      float num = 0.0f, den = 0.0f, err = 0.0f;
-      const float rr = r_s[lr], alpha = a_s[lr];
-      if (i < m) {
-        float x[8], z[8], q[8];
-        load8<WT>(W, i * n + col0, x);
+    if (t < T || TRACE) {
+      for (int s = 0; s < steps; ++s) {
+        const int lr = s * S::RPS + rslot;
+        const int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+        float2 num2 = make_float2(0.f, 0.f), den2 = num2, err2 = num2;
+        const float rr = r_s[lr], alpha = a_s[lr];
+        if (i < m) {
+          float2 x[4], z[4], q[4];
+          load_x(s, x);
+          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) z[k] = __fmul_rn(__fmul_rn(x[k], beta[k]), alpha);
-        grid8<F>(z, q);
+          for (int k = 0; k < 4; ++k) z[k] = __fmul2_rn(__fmul2_rn(x[k], beta[k]), a2);
+          grid8_packed<F>(z, q);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float R = __fmul_rn(q[k], cc[k]);
-          num = fmaf(x[k], R, num);
-          den = fmaf(R, R, den);
-          float d = fmaf(-rr, R, x[k]);
-          err = fmaf(d, d, err);
+          for (int k = 0; k < 4; ++k) {
+            float2 R = __fmul2_rn(q[k], cc[k]);
+            num2 = __ffma2_rn(x[k], R, num2);
+            den2 = __ffma2_rn(R, R, den2);
+            if constexpr (TRACE) {
+              float2 d = __ffma2_rn(make_float2(-rr, -rr), R, x[k]);
+              err2 = __ffma2_rn(d, d, err2);
+            }
+          }
+        }
+        float num = num2.x + num2.y, den = den2.x + den2.y, err = err2.x + err2.y;
+#pragma unroll
+        for (int o = 1; o < S::OPB; o <<= 1) {
+          num += __shfl_xor_sync(0xffffffffu, num, o);
+          den += __shfl_xor_sync(0xffffffffu, den, o);
+          if constexpr (TRACE) err += __shfl_xor_sync(0xffffffffu, err, o);
+        }
+        if (TRACE && oct == 0) e_acc += err;
+        if (t < T && oct == 0 && i < m) {
+          float rn, an;
+          if (den > 0.0f) RowProj<F>::apply(__fdividef(num, den), inv_sT, rtab, atab, sT, rn, an);
+          else RowProj<F>::apply(1.0f, inv_sT, rtab, atab, sT, rn, an);
+          r_s[lr] = rn;
+          a_s[lr] = an;
         }
       }
-#pragma unroll
-      for (int o = 1; o < S::OPB; o <<= 1) {
-        num += __shfl_xor_sync(0xffffffffu, num, o);
-        den += __shfl_xor_sync(0xffffffffu, den, o);
-        err += __shfl_xor_sync(0xffffffffu, err, o);
-      }
-      if (oct == 0) e_acc += err;
-      if (t < T && oct == 0 && i < m) {
-        float rn = (den > 0.0f) ? proj_alpha<F>(__fdiv_rn(num, den), sT) : proj_alpha<F>(1.0f, sT);
-        r_s[lr] = rn;
-        a_s[lr] = __frcp_rn(rn);
-      }
     }
-    if (want_trace) {
+    if constexpr (TRACE) {
 #pragma unroll
       for (int o = 16; o; o >>= 1) e_acc += __shfl_xor_sync(0xffffffffu, e_acc, o);
       if (lane == 0) atomicAdd(&ws->err[t], (double)e_acc);
@@ -320,29 +449,39 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
     __syncwarp();
 
     // ---- column half-step: re-quantise with the new r, update c ----
-    float acc[16];
+    float2 acc[8];
 #pragma unroll
-    for (int v = 0; v < 16; ++v) acc[v] = 0.0f;
+    for (int v = 0; v < 8; ++v) acc[v] = make_float2(0.f, 0.f);
     for (int s = 0; s < steps; ++s) {
       const int lr = s * S::RPS + rslot;
-      int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+      const int64_t i = row0 + (int64_t)s * S::RPS + rslot;
       if (i < m) {
         const float rr = r_s[lr], alpha = a_s[lr];
-        float x[8], z[8], q[8];
-        load8<WT>(W, i * n + col0, x);
+        float2 x[4], z[4], q[4];
+        load_x(s, x);
+        const float2 a2 = make_float2(alpha, alpha), r2 = make_float2(rr, rr);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) z[k] = __fmul_rn(__fmul_rn(x[k], beta[k]), alpha);
-        grid8<F>(z, q);
+        for (int k = 0; k < 4; ++k) z[k] = __fmul2_rn(__fmul2_rn(x[k], beta[k]), a2);
+        grid8_packed<F>(z, q);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float Sv = __fmul_rn(rr, q[k]);
-          acc[2 * k] = fmaf(Sv, x[k], acc[2 * k]);
-          acc[2 * k + 1] = fmaf(Sv, Sv, acc[2 * k + 1]);
+        for (int k = 0; k < 4; ++k) {
+          float2 Sv = __fmul2_rn(r2, q[k]);
+          acc[2 * k] = __ffma2_rn(Sv, x[k], acc[2 * k]);        // (num_j, num_j+1)
+          acc[2 * k + 1] = __ffma2_rn(Sv, Sv, acc[2 * k + 1]);  // (den_j, den_j+1)
         }
       }
     }
+    // reorder to [column][num, den] for the reduction
+    float accv[16];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      accv[4 * k + 0] = acc[2 * k].x;       // num of column 2k
+      accv[4 * k + 1] = acc[2 * k + 1].x;   // den of column 2k
+      accv[4 * k + 2] = acc[2 * k].y;       // num of column 2k+1
+      accv[4 * k + 3] = acc[2 * k + 1].y;   // den of column 2k+1
+    }
     const int par = t & 1;
-    cta_octet_reduce<G, 16>(acc, sm.scr, sm.part, sm.cpart[par]);
+    cta_octet_reduce<G, 16>(accv, sm.scr, sm.part, sm.cpart[par]);
     cluster_sync_all();
     if (tid < G) {
       const int j = tid, o = j >> 3, k = j & 7;
@@ -357,18 +496,18 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
     }
     __syncthreads();
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      cc[k] = sm.c_s[oct * 8 + k];
-      beta[k] = sm.b_s[oct * 8 + k];
+    for (int k = 0; k < 4; ++k) {
+      cc[k] = make_float2(sm.c_s[oct * 8 + 2 * k], sm.c_s[oct * 8 + 2 * k + 1]);
+      beta[k] = make_float2(sm.b_s[oct * 8 + 2 * k], sm.b_s[oct * 8 + 2 * k + 1]);
     }
   }
 
   // outputs
   for (int s = 0; s < steps; ++s) {
-    int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+    const int64_t i = row0 + (int64_t)s * S::RPS + rslot;
     if (oct == 0 && i < m) r_out[i * nb + b] = r_s[s * S::RPS + rslot];
   }
-  if (rank == 0 && tid < G) c_io[b * G + tid] = (T > 0) ? sm.c_s[tid] : c_io[b * G + tid];
+  if (rank == 0 && tid < G && T > 0) c_io[b * G + tid] = sm.c_s[tid];
   cluster_sync_all();  // no CTA leaves while a peer may still read its cpart
 }
 
@@ -380,9 +519,42 @@ __global__ void solve_finalize_kernel(const SolverWs* ws, int T, double* mse_tra
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int G>
-static size_t solver_smem_bytes(int steps) {
-  return sizeof(SolverSmem<G>) + 2 * sizeof(float) * (size_t)steps * SolverShape<G>::RPS;
+template <int G, typename WT>
+static size_t solver_smem_bytes(int steps, bool wsmem) {
+  const size_t rows = (size_t)steps * SolverShape<G>::RPS;
+  return sizeof(SolverSmem<G>) + 2 * sizeof(float) * rows + 2 * 128 * sizeof(float) +
+         (wsmem ? rows * G * sizeof(WT) : 0);
+}
+
+// Launch geometry: the tile's rows are split over C CTAs of one cluster,
+// `steps` row-steps of RPS rows per CTA.  Prefer staging the CTA's rows in
+// shared memory (<= 96 KB of rows, clusters of up to 16 CTAs); otherwise
+// stream them through the read-only global path with clusters of 8.
+template <int G, typename WT>
+static void solver_geometry(int64_t m, int& steps, int& C, bool& wsmem) {
+  using S = SolverShape<G>;
+  const size_t row_bytes = (size_t)G * sizeof(WT);
+  for (int cmax : {8, 16}) {
+    int st = (int)((m + (int64_t)S::RPS * cmax - 1) / ((int64_t)S::RPS * cmax));
+    if (st < 1) st = 1;
+    if ((size_t)st * S::RPS * row_bytes <= 96 * 1024) {
+      steps = st;
+      C = (int)((m + (int64_t)S::RPS * st - 1) / ((int64_t)S::RPS * st));
+      wsmem = true;
+      return;
+    }
+  }
+  steps = (int)((m + (int64_t)S::RPS * 8 - 1) / ((int64_t)S::RPS * 8));
+  C = (int)((m + (int64_t)S::RPS * steps - 1) / ((int64_t)S::RPS * steps));
+  wsmem = false;
+}
+
+template <typename K>
+static bool allow_big_cluster(K kern, size_t smem) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+             cudaSuccess &&
+         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+             cudaSuccess;
 }
 
 template <int F, int G, typename WT>
@@ -390,10 +562,10 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, float* r, 
                          float* sT, double* trace, SolverWs* ws, cudaStream_t st) {
   using S = SolverShape<G>;
   const WT* W = reinterpret_cast<const WT*>(Wv);
-  int steps = (int)((m + (int64_t)S::RPS * 8 - 1) / ((int64_t)S::RPS * 8));
-  if (steps < 1) steps = 1;
-  int C = (int)((m + (int64_t)S::RPS * steps - 1) / ((int64_t)S::RPS * steps));
-  const size_t sm_init = sizeof(SolverSmem<G>), sm_main = solver_smem_bytes<G>(steps);
+  int steps, C;
+  bool wsmem;
+  solver_geometry<G, WT>(m, steps, C, wsmem);
+  const size_t sm_init = sizeof(SolverSmem<G>), sm_main = solver_smem_bytes<G, WT>(steps, wsmem);
   if (sm_main > 227 * 1024) return DQ_ERR_UNSUPPORTED;
 
   cudaLaunchAttribute attr[1];
@@ -409,18 +581,25 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, float* r, 
   cfg.numAttrs = 1;
 
   auto kinit = solve_init_kernel<F, G, WT>;
-  auto kmain = solve_bcd_kernel<F, G, WT>;
-  if (cudaFuncSetAttribute(kinit, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_init) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(kmain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_main) !=
-          cudaSuccess)
-    return DQ_ERR_CUDA;
+  if (!allow_big_cluster(kinit, sm_init)) return DQ_ERR_CUDA;
   cfg.dynamicSmemBytes = sm_init;
   if (cudaLaunchKernelEx(&cfg, kinit, W, m, n, steps, c, ws) != cudaSuccess) return DQ_ERR_CUDA;
+
   cfg.dynamicSmemBytes = sm_main;
-  if (cudaLaunchKernelEx(&cfg, kmain, W, m, n, steps, T, r, c, sT, ws, trace ? 1 : 0) !=
-      cudaSuccess)
-    return DQ_ERR_CUDA;
+  cudaError_t e;
+#define DQ_MAIN(WS, TR)                                                                     \
+  {                                                                                         \
+    auto km = solve_bcd_kernel<F, G, WT, WS, TR>;                                          \
+    if (!allow_big_cluster(km, sm_main)) return DQ_ERR_CUDA;                               \
+    e = cudaLaunchKernelEx(&cfg, km, W, m, n, steps, T, r, c, sT, ws);                      \
+  }
+  if (wsmem) {
+    if (trace) DQ_MAIN(true, true) else DQ_MAIN(true, false)
+  } else {
+    if (trace) DQ_MAIN(false, true) else DQ_MAIN(false, false)
+  }
+#undef DQ_MAIN
+  if (e != cudaSuccess) return DQ_ERR_CUDA;
   if (trace) {
     solve_finalize_kernel<<<(T + 1 + 127) / 128, 128, 0, st>>>(ws, T, trace);
     if (cudaGetLastError() != cudaSuccess) return DQ_ERR_CUDA;
