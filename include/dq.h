@@ -186,6 +186,34 @@ DQ_API int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_to
                    const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                    dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream);
 
+/* ------------------------------------------------------------------------
+ * dq_solve_scales_noalloc -- dq_solve_scales for callers that cannot
+ * allocate device memory (the paper has no counterpart: this is a library
+ * convenience).  Some callers have no way to provide the workspace: a
+ * serving process that has handed all free device memory to its own pool
+ * and may not call cudaMalloc around it, or a latency-critical path that
+ * must never wait in the driver's allocator.  This entry point takes the
+ * same inputs and outputs but no workspace: its scratch is a fixed array of
+ * DQ_NOALLOC_SCRATCH_BYTES compiled into the library, present on every GPU
+ * that loads the library until the process exits.  It never calls
+ * cudaMalloc, cudaFree or any allocating routine.
+ *  - T may be at most DQ_NOALLOC_MAX_ROUNDS; larger T returns
+ *    DQ_ERR_WORKSPACE before anything is enqueued.
+ *  - The first call on each device looks up the array's device address with
+ *    that device current (a host-side step); make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the one array, which keeps the contents
+ *    of the last call (each call clears what it uses first).  Calls whose
+ *    execution overlaps on the GPU (different streams, no ordering between
+ *    them) race on the array and may corrupt each other's trace and NVFP4
+ *    tensor scale; serialise them.
+ * ---------------------------------------------------------------------- */
+#define DQ_NOALLOC_SCRATCH_BYTES 16384
+#define DQ_NOALLOC_MAX_ROUNDS 2045
+DQ_API int dq_solve_scales_noalloc(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f,
+                                   int group, int T, float* r, float* c, float* s_tensor,
+                                   double* mse_trace, void* stream);
+
 /* Device-side error word set by a kernel whose bounded wait expired
  * (0 = none).  Synchronises the current device; clear != 0 resets it. */
 DQ_API int dq_device_error(int clear);

@@ -35,6 +35,8 @@ SIGNATURES = {
     "dq_quantize_act": (_int, [_vp, _int, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp, _vp]),
     "dq_w4a4_linear": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64,
                               _int, _vp]),
+    "dq_solve_scales_noalloc": (_int, [_vp, _int, _i64, _i64, _int, _int, _int, _vp, _vp, _vp,
+                                       _vp, _vp]),
     "dq_device_error": (_int, [_int]),
     "dq_version": (_int, []),
 }
@@ -112,6 +114,16 @@ def dq_solve_scales(W, fmt, T, r, c, s_tensor, mse_trace=None, workspace=None, g
                                  _ptr(s_tensor), _ptr(mse_trace), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)),
            "dq_solve_scales")
+
+
+def dq_solve_scales_noalloc(W, fmt, T, r, c, s_tensor, mse_trace=None, group=0, stream=None):
+    """dq_solve_scales without a workspace: the library's fixed scratch array
+    is used instead (T <= 2045; calls on one device must not overlap)."""
+    m, n = W.shape
+    _check(lib().dq_solve_scales_noalloc(_ptr(W), _dtype(W), m, n, _fmt(fmt), group, T, _ptr(r),
+                                         _ptr(c), _ptr(s_tensor), _ptr(mse_trace),
+                                         _stream(stream)),
+           "dq_solve_scales_noalloc")
 
 
 def dq_quantize_weight(W, fmt, r, c, s_tensor, codes, scales, group=0, stream=None):
