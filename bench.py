@@ -45,6 +45,22 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, 1965.0, "fallback"
 
 
+def measured_traffic(key, files):
+    """DRAM bytes per launch from the committed ncu capture of this kernel,
+    or None when the kernel's source changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(key)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "w4a4_post_quantization_dual_b200", "csrc", f), "rb").read())
+    return rec["dram_bytes"] if h.hexdigest()[:16] == rec["source_hash"] else None
+
+
 def workload_inputs():
     wl = synth.WORKLOADS[WORKLOAD]
     Ws = [synth.weight(WORKLOAD, i)[0] for i in range(len(wl["weights"]))]
@@ -248,7 +264,7 @@ def run_ours(args, rank, world, local_rank):
             dq.dq_solve_scales(W, fmt, T, b["r"], b["c"], b["sT"], None, ws, group=G)
             s1.record(st)
             dq.dq_quantize_weight(W, fmt, b["r"], b["c"], b["sT"], b["codes"], b["scales"], group=G)
-            rec["solve"].append((s0, s1))
+            rec["solve"].append((s0, s1, W.numel()))
         e1.record(st)
         for M, X in Xd.items():
             a = Abuf[M]
@@ -293,7 +309,9 @@ def run_ours(args, rank, world, local_rank):
     el = lambda p: p[0].elapsed_time(p[1])  # ms
     step_ms = sum(el(p) for p in rec["step"])
     lin_ms = sum(el(p) for p in rec["lin"])
-    solve_ms = sum(el(p) for p in rec["solve"])
+    solve_ms = sum(el(p[:2]) for p in rec["solve"])
+    big = max(p[2] for p in rec["solve"])
+    solve_big = [el(p[:2]) for p in rec["solve"] if p[2] == big]
     gemm_pre = [(el((p[0], p[1])), p[2]) for p in rec["gemm"] if p[3] == prefill_M]
     act_pre = [(el((p[0], p[1])), p[2]) for p in rec["act"] if p[2] == prefill_M * 4096]
     totals = torch.tensor([step_ms, lin_ms, solve_ms], dtype=torch.float64, device=dev)
@@ -341,15 +359,13 @@ def run_ours(args, rank, world, local_rank):
         return
     hbm, bf16_tf, bf16_sus, sm_max, peak_kind = peaks()
     fp4_peak = 4.0 * bf16_tf            # nominal fp4 : bf16 dense ratio 9 : 2.25
-    n_solve = len(rec["solve"])
-    solve_launch_ms = solve_ms / max(n_solve, 1)
-    # solver: algorithmic work = 12 fp32 ops per element per round (two
-    # quantisations, two scale products, four reduction FMAs), ALU peak =
+    # solver roofline on the largest weight (one dq_solve_scales call: init +
+    # BCD launches).  Algorithmic work = 12 fp32 ops per element per round
+    # (two quantisations, two scale products, four reduction FMAs); ALU peak =
     # 148 SMs x 128 fp32 lanes x max SM clock.
-    elems = sum(W.numel() for W in Wd)
     alu_peak = 148 * 128 * sm_max * 1e6 / 1e12  # T lane-ops/s
-    solve_ops = 12.0 * elems * T * args.steps
-    solver_alu = solve_ops / (solve_ms * 1e-3) / 1e12
+    big_ms = sum(solve_big) / len(solve_big)
+    solver_alu = 12.0 * big * T / (big_ms * 1e-3) / 1e12
     solver_gbs = T * sum(W.numel() * 2 for W in Wd) * args.steps / (solve_ms * 1e-3) / 1e9
     g_ms = sum(t for t, _ in gemm_pre) / max(len(gemm_pre), 1)
     g_fl = sum(f for _, f in gemm_pre) / max(len(gemm_pre), 1)
@@ -377,17 +393,25 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD, "format": FMT_NAME, "weights": [list(W.shape) for W in Ws],
                    "M": sorted(Xd), "T": T, "l2": "flushed between steps (256 MiB write)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "solve_bcd_kernel (BCD rounds)", "bound": "alu",
-                     "achieved": solver_alu, "peak": alu_peak, "unit": "Tops/s",
-                     "frac": solver_alu / alu_peak, "traffic": None,
+        "roofline": {"kernel": "solve_bcd_kernel (+ solve_init_kernel), 4096x4096 bf16, T=50",
+                     "bound": "alu", "achieved": solver_alu, "peak": alu_peak, "unit": "Tops/s",
+                     "frac": solver_alu / alu_peak, "ms_per_launch": big_ms,
+                     "traffic": measured_traffic("solver_4096x4096_nvfp4_T50",
+                                                 ["dq_solver.cu", "dq_device.cuh"]),
+                     "algorithmic_bytes": big * 2 + big // 16 * 4 + 4096 * 4,
                      "note": "12 algorithmic fp32 ops / element / round; peak = 148 SM x 128 "
-                             "fp32 lanes x max SM clock"},
+                             "fp32 lanes x max SM clock (derived, not measured)"},
         "roofline_gemm": {"kernel": "w4a4_gemm_kernel", "bound": "tensor", "achieved": gemm_tf,
                           "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
-                          "traffic": None, "shape": f"M={prefill_M} x N x K=4096",
+                          "traffic": measured_traffic("gemm_nvfp4_4096x4096x4096",
+                                                      ["dq_gemm.cu", "dq_device.cuh"]),
+                          "shape": f"M={prefill_M} x N x K=4096",
                           "peak_kind": f"{peak_kind} bf16 burst x 4 (nominal fp4:bf16)"},
-        "roofline_act": {"kernel": "quantize_act_kernel", "bound": "hbm", "achieved": act_gbs,
-                         "peak": hbm, "unit": "GB/s", "frac": act_gbs / hbm, "traffic": None},
+        "roofline_act": {"kernel": "quantize_act_rows_kernel", "bound": "hbm", "achieved": act_gbs,
+                         "peak": hbm, "unit": "GB/s", "frac": act_gbs / hbm,
+                         "traffic": measured_traffic("act_nvfp4_4096x4096",
+                                                     ["dq_quant.cu", "dq_device.cuh"]),
+                         "shape": f"M={prefill_M} x K=4096"},
         "solver": {"gbs_effective": solver_gbs, "frac_hbm": solver_gbs / hbm,
                    "ms_per_weight_set": solve_ms / args.steps,
                    "definition": "T * bytes(W bf16) / solver time (tile stays on chip)"},
