@@ -13,12 +13,16 @@
 //   warp 0      TMA producer: A / B code tiles (128-byte swizzled K-major,
 //               BK = 256 four-bit elements) and the matching 512-byte
 //               block-scale atoms (bulk copies), into a STAGES-deep ring.
-//   warp 1      allocates tensor memory; one thread copies the scale atoms
-//               to tensor memory (tcgen05.cp 32x128b.warpx4) and issues
+//   warp 1      allocates tensor memory; one thread issues
 //               tcgen05.mma.kind::mxf4nvf4 / kind::mxf4 .block_scale, fp32
 //               accumulation in tensor memory; commits free the ring slots.
 //   warps 2..5  epilogue: tcgen05.ld the accumulator (each warp its 32-lane
 //               quadrant), release it to the MMA warp, scale, convert, store.
+//   warp 6      copies each stage's scale atoms into that stage's own slot of
+//               tensor memory (tcgen05.cp 32x128b.warpx4) and signals the MMA
+//               warp, so the copies for later stages run while the MMAs of
+//               the current stage execute (issued by the MMA thread itself,
+//               the copies serialise with the MMAs).
 // Every mbarrier wait is bounded (globaltimer); on expiry the kernel records
 // DQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
 #include <cuda.h>
@@ -37,7 +41,7 @@ namespace gemm {
 constexpr int BM = 128;
 constexpr int BK = 256;             // four-bit elements per k-tile (128 bytes per row)
 constexpr int BKB = BK / 2;         // bytes per row per k-tile
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 224;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -179,13 +183,16 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = (227 * 1024 - 1024 - 256) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  // tensor-memory columns: accumulator, then scale factors
-  static constexpr int SFA_COL = BN;
-  static constexpr int SFB_COL = BN + 4 * SF_ATOMS;
-  static constexpr int TMEM_USED = SFB_COL + 4 * SF_ATOMS * (BN / 128);
+  static_assert(3 * STAGES * 8 + 32 <= 256, "barrier area");
+  // tensor-memory columns: accumulator, then one scale slot per stage
+  // (SFA: 4 columns per atom; SFB: 4 columns per atom and 128-row group)
+  static constexpr int SF_COLS = 4 * SF_ATOMS * (1 + BN / 128);
+  static constexpr int SF_BASE = BN;
+  static constexpr int TMEM_USED = SF_BASE + STAGES * SF_COLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static constexpr int K_STEPS = BK / 64;                     // MMAs per k-tile (K = 64 each)
   static_assert(STAGES >= 2, "pipeline depth");
+  static_assert(TMEM_USED <= 512, "tensor memory budget");
 };
 
 // bf16 epilogue of one 128 x BN tile for one thread (one accumulator row):
@@ -241,7 +248,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   unsigned char* sSFB = sSFA + C::STAGES * C::SFA_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + C::STAGES * C::SFB_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* sfready = empty + C::STAGES;
+  uint64_t* acc_full = sfready + C::STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
@@ -256,6 +264,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sfready[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
@@ -319,24 +328,13 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (!mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag)) break;
         fence_after_sync();
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&full[stage], phase, abort_flag) ||
+              !mbar_wait(&sfready[stage], phase, abort_flag)) { ok = false; break; }
           fence_after_sync();
           const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
-          const uint32_t sfa_base = smem_u32(sSFA + stage * C::SFA_BYTES);
-          const uint32_t sfb_base = smem_u32(sSFB + stage * C::SFB_BYTES);
-          // scale atoms -> tensor memory
-#pragma unroll
-          for (int j = 0; j < C::SF_ATOMS; ++j)
-            tmem_cp_32x128b_x4(tmem + C::SFA_COL + 4 * j,
-                               smem_desc(sfa_base + j * 512, 0, 128, LAYOUT_NONE));
-#pragma unroll
-          for (int g = 0; g < BN / 128; ++g)
-#pragma unroll
-            for (int j = 0; j < C::SF_ATOMS; ++j)
-              tmem_cp_32x128b_x4(tmem + C::SFB_COL + 4 * (BN / 128) * j + 4 * g,
-                                 smem_desc(sfb_base + (g * C::SF_ATOMS + j) * 512, 0, 128,
-                                           LAYOUT_NONE));
+          const uint32_t sfa0 = C::SF_BASE + stage * C::SF_COLS;
+          const uint32_t sfb0 = sfa0 + 4 * C::SF_ATOMS;
 #pragma unroll
           for (int kk = 0; kk < C::K_STEPS; ++kk) {
             // K = 64 four-bit elements = 32 bytes inside the 128-byte swizzle row
@@ -345,12 +343,12 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t sf_id, sfa_col, sfb_col;
             if constexpr (FMT == NVFP4) {  // 4 scales per row per MMA: one column each
               sf_id = 0;
-              sfa_col = C::SFA_COL + 4 * kk;
-              sfb_col = C::SFB_COL + 4 * (BN / 128) * kk;
+              sfa_col = sfa0 + 4 * kk;
+              sfb_col = sfb0 + 4 * (BN / 128) * kk;
             } else {                        // 2 scales per row per MMA: half a column
               sf_id = 2 * (kk & 1);
-              sfa_col = C::SFA_COL + 4 * (kk >> 1);
-              sfb_col = C::SFB_COL + 4 * (BN / 128) * (kk >> 1);
+              sfa_col = sfa0 + 4 * (kk >> 1);
+              sfb_col = sfb0 + 4 * (BN / 128) * (kk >> 1);
             }
             const uint32_t idesc = idesc0 | (sf_id << 29) | (sf_id << 4);
             mma_fp4<FMT>(tmem, ad, bd, idesc, (kt > 0 || kk > 0) ? 1u : 0u,
@@ -361,6 +359,35 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         if (!ok) break;
         mma_commit(acc_full);
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ scale copier
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          fence_after_sync();
+          const uint32_t sfa_base = smem_u32(sSFA + stage * C::SFA_BYTES);
+          const uint32_t sfb_base = smem_u32(sSFB + stage * C::SFB_BYTES);
+          const uint32_t sfa0 = C::SF_BASE + stage * C::SF_COLS;
+          const uint32_t sfb0 = sfa0 + 4 * C::SF_ATOMS;
+#pragma unroll
+          for (int j = 0; j < C::SF_ATOMS; ++j)
+            tmem_cp_32x128b_x4(tmem + sfa0 + 4 * j, smem_desc(sfa_base + j * 512, 0, 128, LAYOUT_NONE));
+#pragma unroll
+          for (int g = 0; g < BN / 128; ++g)
+#pragma unroll
+            for (int j = 0; j < C::SF_ATOMS; ++j)
+              tmem_cp_32x128b_x4(tmem + sfb0 + 4 * (BN / 128) * j + 4 * g,
+                                 smem_desc(sfb_base + (g * C::SF_ATOMS + j) * 512, 0, 128,
+                                           LAYOUT_NONE));
+          mma_commit(&sfready[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
       }
     }
   } else {
