@@ -276,7 +276,7 @@ def run_ours(args, rank, world, local_rank):
                 dq.dq_w4a4_linear(a["A"], a["sA"], a["st"], b["codes"], b["scales"], b["sT"],
                                   a["Y"][j], fmt)
                 g1.record(st)
-                rec["act"].append((q0, q1, M * X.shape[1]))
+                rec["act"].append((q0, q1, M * X.shape[1], M))
                 rec["gemm"].append((q1, g1, 2.0 * M * W.shape[0] * W.shape[1], M))
         e2.record(st)
         rec["step"].append((e0, e2))
@@ -374,6 +374,11 @@ def run_ours(args, rank, world, local_rank):
     a_bytes = prefill_M * 4096 * (2 + 0.5 + 1.0 / 16) + prefill_M * 4
     act_gbs = a_bytes / (a_ms * 1e-3) / 1e9
     value = lin_flops * args.steps / (lin_ms * 1e-3) / 1e12
+    per_m = {}
+    for M in sorted(Xd):
+        ga = [el((p[0], p[1])) for p in rec["gemm"] if p[3] == M]
+        aa = [el((p[0], p[1])) for p in rec["act"] if p[3] == M]
+        per_m[str(M)] = {"act_quant": 1e3 * sum(aa) / len(aa), "gemm": 1e3 * sum(ga) / len(ga)}
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -412,6 +417,7 @@ def run_ours(args, rank, world, local_rank):
                          "traffic": measured_traffic("act_nvfp4_4096x4096",
                                                      ["dq_quant.cu", "dq_device.cuh"]),
                          "shape": f"M={prefill_M} x K=4096"},
+        "per_M_us": per_m,
         "solver": {"gbs_effective": solver_gbs, "frac_hbm": solver_gbs / hbm,
                    "ms_per_weight_set": solve_ms / args.steps,
                    "definition": "T * bytes(W bf16) / solver time (tile stays on chip)"},

@@ -31,7 +31,8 @@ def operands(M, N, K, fmt, seed=0, T=0, x_outliers=0.01, x_scale=50.0):
 
 @pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
 @pytest.mark.parametrize("M,N,K", [(16, 256, 256), (1, 512, 4096), (300, 512, 768),
-                                   (128, 128, 256), (257, 384, 512), (1000, 1024, 1024)])
+                                   (128, 128, 256), (257, 384, 512), (1000, 1024, 1024),
+                                   (64, 4096, 4096), (8, 1024, 5120)])
 def test_gemm_small_parity(fmt, M, N, K):
     A, sA, st, B, sB, sW = operands(M, N, K, fmt, seed=M + N)
     ref = O.linear(A, sA, st, B, sB, sW, M, N, K, fmt)
@@ -54,7 +55,8 @@ def test_gemm_row_factor_epilogue():
 
 @pytest.mark.parametrize("fmt,M,N,K", [
     (O.NVFP4, 4096, 4096, 4096),    # Llama-3.1-8B q/o projection, prefill
-    (O.NVFP4, 1, 1024, 4096),       # k/v projection, decode
+    (O.NVFP4, 1, 1024, 4096),       # k/v projection, decode (split-K over a cluster)
+    (O.NVFP4, 8, 27648, 5120),      # Qwen-32B up projection, decode
     (O.MXFP4, 2048, 14336, 4096),   # gate/up, MX
     (O.NVFP4, 8192, 5120, 27648),   # Qwen-32B down projection, prefill
 ])

@@ -3,7 +3,48 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 #include "dq_internal.h"
+
+namespace dq {
+
+bool ensure_kernel_attrs(const void* kernel, int smem_bytes, bool big_cluster) {
+  struct Done {
+    const void* k;
+    int dev, smem;
+    bool cluster;
+  };
+  static std::mutex mu;
+  static std::vector<Done> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    for (const Done& d : done)
+      if (d.k == kernel && d.dev == dev && d.smem >= smem_bytes && (d.cluster || !big_cluster))
+        return true;
+  }
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+      cudaSuccess)
+    return false;
+  // Every kernel of the library asks for the same L1 / shared-memory split
+  // (all shared), so consecutive kernels (act quant -> GEMM -> ...) never
+  // make the SMs re-partition their on-chip memory between launches.
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return false;
+  if (big_cluster &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess)
+    return false;
+  std::lock_guard<std::mutex> g(mu);
+  done.push_back({kernel, dev, smem_bytes, big_cluster});
+  return true;
+}
+
+}  // namespace dq
 
 namespace {
 

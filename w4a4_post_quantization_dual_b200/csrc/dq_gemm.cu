@@ -171,7 +171,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* v) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-template <int FMT, int BN>
+template <int FMT, int BN, int RESERVE = 0>
 struct Cfg {
   static constexpr int G = (FMT == NVFP4) ? 16 : 32;
   static constexpr int SF_PER_ROW = BK / G;                   // scales per row per k-tile
@@ -181,8 +181,8 @@ struct Cfg {
   static constexpr int SFA_BYTES = SF_ATOMS * 512;
   static constexpr int SFB_BYTES = (BN / 128) * SF_ATOMS * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = (227 * 1024 - 1024 - 256) / STAGE_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int STAGES = (227 * 1024 - 1024 - 256 - RESERVE) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + RESERVE;
   static_assert(3 * STAGES * 8 + 32 <= 256, "barrier area");
   // tensor-memory columns: accumulator, then one scale slot per stage
   // (SFA: 4 columns per atom; SFB: 4 columns per atom and 128-row group)
@@ -452,6 +452,218 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------
+// Split-K variant for problems with few output tiles (small M): the S CTAs
+// of a thread-block cluster compute K-slices of the same 128 x 128 tile with
+// the same TMA / scale-copy / tcgen05 pipeline, drain their fp32 partial
+// tiles into shared memory, and after a cluster barrier each CTA sums one
+// column slice of the tile over DSMEM (in rank order), applies the epilogue
+// scales and stores.  No global workspace.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
+  uint32_t a = smem_u32(local), ra;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+constexpr int SK_BN = 128;
+constexpr int SK_LD = SK_BN + 4;                  // padded row of the partial tile (floats)
+constexpr int SK_PART_BYTES = BM * SK_LD * 4;
+
+template <int FMT, int YT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const uint8_t* __restrict__ sfA,
+                        const uint8_t* __restrict__ sfB, const float* __restrict__ s_tok,
+                        const float* __restrict__ s_w, const float* __restrict__ r_row,
+                        void* __restrict__ Y, int M, int N, int K, int kt_per_slice) {
+  constexpr int BN = SK_BN;
+  using C = Cfg<FMT, BN, SK_PART_BYTES>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* sA = smem;
+  unsigned char* sB = sA + C::STAGES * C::A_BYTES;
+  unsigned char* sSFA = sB + C::STAGES * C::B_BYTES;
+  unsigned char* sSFB = sSFA + C::STAGES * C::SFA_BYTES;
+  float* part = reinterpret_cast<float*>(sSFB + C::STAGES * C::SFB_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(part) + SK_PART_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* sfready = empty + C::STAGES;
+  uint64_t* acc_full = sfready + C::STAGES;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank(), S = gridDim.x;
+  const int n0 = blockIdx.y * BN, m0 = blockIdx.z * BM;
+  const int kt0 = (int)rank * kt_per_slice;
+  const int S4 = (K / C::G) / 4;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sfready[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_base_slot)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_base_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = 0; kt < kt_per_slice; ++kt) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+        mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+        tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], (kt0 + kt) * BKB, m0);
+        tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], (kt0 + kt) * BKB, n0);
+        bulk_load(sSFA + stage * C::SFA_BYTES,
+                  sfA + ((size_t)(m0 / 128) * S4 + (size_t)(kt0 + kt) * C::SF_ATOMS) * 512,
+                  C::SFA_BYTES, &full[stage]);
+        bulk_load(sSFB + stage * C::SFB_BYTES,
+                  sfB + ((size_t)(n0 / 128) * S4 + (size_t)(kt0 + kt) * C::SF_ATOMS) * 512,
+                  C::SFB_BYTES, &full[stage]);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+      for (int s = 0; s < C::STAGES; ++s) {  // drain: every issued stage lands before exit
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      const uint32_t idesc0 = idesc_fp4(BN, FMT != NVFP4);
+      for (int kt = 0; kt < kt_per_slice; ++kt) {
+        if (!mbar_wait(&full[stage], phase, abort_flag) ||
+            !mbar_wait(&sfready[stage], phase, abort_flag)) { ok = false; break; }
+        fence_after_sync();
+        const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
+        const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
+        const uint32_t sfa0 = C::SF_BASE + stage * C::SF_COLS;
+        const uint32_t sfb0 = sfa0 + 4 * C::SF_ATOMS;
+#pragma unroll
+        for (int kk = 0; kk < C::K_STEPS; ++kk) {
+          const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, LAYOUT_SW128);
+          const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, LAYOUT_SW128);
+          uint32_t sf_id, sfa_col, sfb_col;
+          if constexpr (FMT == NVFP4) {
+            sf_id = 0;
+            sfa_col = sfa0 + 4 * kk;
+            sfb_col = sfb0 + 4 * kk;
+          } else {
+            sf_id = 2 * (kk & 1);
+            sfa_col = sfa0 + 4 * (kk >> 1);
+            sfb_col = sfb0 + 4 * (kk >> 1);
+          }
+          const uint32_t idesc = idesc0 | (sf_id << 29) | (sf_id << 4);
+          mma_fp4<FMT>(tmem, ad, bd, idesc, (kt > 0 || kk > 0) ? 1u : 0u,
+                       (tmem + sfa_col) | (sf_id << 30), (tmem + sfb_col) | (sf_id << 30));
+        }
+        mma_commit(&empty[stage]);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (ok) mma_commit(acc_full);
+    }
+  } else if (warp == 6) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = 0; kt < kt_per_slice; ++kt) {
+        if (!mbar_wait(&full[stage], phase, abort_flag)) break;
+        fence_after_sync();
+        const uint32_t sfa_base = smem_u32(sSFA + stage * C::SFA_BYTES);
+        const uint32_t sfb_base = smem_u32(sSFB + stage * C::SFB_BYTES);
+        const uint32_t sfa0 = C::SF_BASE + stage * C::SF_COLS;
+        const uint32_t sfb0 = sfa0 + 4 * C::SF_ATOMS;
+#pragma unroll
+        for (int j = 0; j < C::SF_ATOMS; ++j) {
+          tmem_cp_32x128b_x4(tmem + sfa0 + 4 * j, smem_desc(sfa_base + j * 512, 0, 128, LAYOUT_NONE));
+          tmem_cp_32x128b_x4(tmem + sfb0 + 4 * j, smem_desc(sfb_base + j * 512, 0, 128, LAYOUT_NONE));
+        }
+        mma_commit(&sfready[stage]);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else {
+    // drain this CTA's partial tile (rows that exist) into shared memory
+    const int quad = warp & 3;
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(acc_full, 0, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok && m0 + quad * 32 < M) {
+      fence_after_sync();
+      float* dst = part + (size_t)(quad * 32 + lane) * SK_LD;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
+#pragma unroll
+        for (int k = 0; k < 32; k += 4)
+          *reinterpret_cast<float4*>(dst + c0 + k) =
+              make_float4(__uint_as_float(v[k]), __uint_as_float(v[k + 1]),
+                          __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+      }
+    }
+  }
+
+  fence_before_sync();
+  cluster_barrier();   // every CTA's partial tile is in its shared memory
+  {
+    // this CTA reduces columns [rank * BN / S, (rank + 1) * BN / S) of the tile
+    const int cols = BN / (int)S, c_begin = (int)rank * cols;
+    const int rows = (M - m0) < BM ? (M - m0) : BM;
+    const float sw = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
+    for (int idx = threadIdx.x; idx < rows * cols; idx += NUM_THREADS) {
+      const int r = idx / cols, c = c_begin + idx % cols;
+      float acc = 0.0f;
+      for (uint32_t q = 0; q < S; ++q) acc += ld_dsmem_f32(part + (size_t)r * SK_LD + c, q);
+      float rs = sw;
+      if (FMT == NVFP4 && s_tok) rs = __fmul_rn(s_tok[m0 + r], sw);
+      float f = __fmul_rn(acc, rs);
+      if (r_row) f = __fmul_rn(f, __ldg(r_row + n0 + c));
+      const size_t o = (size_t)(m0 + r) * N + n0 + c;
+      if constexpr (YT == 1) reinterpret_cast<__nv_bfloat16*>(Y)[o] = __float2bfloat16_rn(f);
+      else reinterpret_cast<float*>(Y)[o] = f;
+    }
+  }
+  cluster_barrier();   // no CTA leaves while a peer may still read its partial tile
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -473,17 +685,41 @@ static PFN_encodeTiled get_encode() {
 }
 
 // 2-D map over a rows x (K/2) byte matrix, box = box_rows x 128 bytes, 128-byte swizzle.
+// Encoding a map is host work comparable to a small kernel, so the maps of
+// recent operands are kept in a small per-thread cache (a map only encodes
+// the base pointer, sizes and strides, so a hit is always valid).
+struct MapEntry {
+  const void* base;
+  int64_t rows, kbytes;
+  int box_rows;
+  CUtensorMap map;
+};
 static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t kbytes,
                      int box_rows) {
+  constexpr int kEntries = 16;
+  thread_local MapEntry cache[kEntries];
+  thread_local int used = 0, next = 0;
+  for (int i = 0; i < used; ++i)
+    if (cache[i].base == base && cache[i].rows == rows && cache[i].kbytes == kbytes &&
+        cache[i].box_rows == box_rows) {
+      *map = cache[i].map;
+      return true;
+    }
   PFN_encodeTiled enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kbytes};
   cuuint32_t box[2] = {(cuuint32_t)BKB, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  MapEntry& e = cache[next];
+  e.base = base; e.rows = rows; e.kbytes = kbytes; e.box_rows = box_rows; e.map = *map;
+  next = (next + 1) % kEntries;
+  if (used < kEntries) ++used;
+  return true;
 }
 
 static int num_sms() {
@@ -505,9 +741,7 @@ static int launch(const uint8_t* A, const uint8_t* sA, const float* s_tok, const
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, M, K / 2, BM) || !make_map(&tb, B, N, K / 2, BN)) return DQ_ERR_CUDA;
   auto kern = w4a4_gemm_kernel<FMT, BN, YT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-      cudaSuccess)
-    return DQ_ERR_CUDA;
+  if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
   const int64_t tiles = ((M + BM - 1) / BM) * (N / BN);
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
   kern<<<grid, NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, sA, sB, s_tok, s_w, r_row, Y, (int)M,
@@ -515,20 +749,65 @@ static int launch(const uint8_t* A, const uint8_t* sA, const float* s_tok, const
   return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
 }
 
+template <int FMT, int YT>
+static int launch_splitk(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
+                         const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
+                         int64_t M, int64_t N, int64_t K, int S, cudaStream_t st) {
+  using C = Cfg<FMT, SK_BN, SK_PART_BYTES>;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K / 2, BM) || !make_map(&tb, B, N, K / 2, SK_BN)) return DQ_ERR_CUDA;
+  auto kern = w4a4_gemm_splitk_kernel<FMT, YT>;
+  if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S, (unsigned)(N / SK_BN), (unsigned)((M + BM - 1) / BM));
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int kt_per_slice = (int)(K / BK) / S;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, sA, sB, s_tok, s_w, r_row, Y, (int)M, (int)N,
+                         (int)K, kt_per_slice) != cudaSuccess)
+    return DQ_ERR_CUDA;
+  return DQ_OK;
+}
+
+// Tile-shape policy: 128 x 256 persistent tiles when they fill the machine,
+// else 128 x 128 persistent tiles, else split-K over a cluster of S CTAs.
+template <int FMT, int YT>
+static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
+                    const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int64_t M,
+                    int64_t N, int64_t K, cudaStream_t st) {
+  const int64_t tm = (M + BM - 1) / BM, sms = num_sms();
+  if (N % 256 == 0 && tm * (N / 256) >= sms)
+    return launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
+  const int64_t t128 = tm * (N / 128);
+  const int KT = (int)(K / BK);
+  int S = 1;
+  for (int cand : {8, 4, 2})
+    if (S == 1 && KT % cand == 0 && t128 * cand <= 2 * sms && t128 * 2 <= sms) S = cand;
+  if (S > 1) return launch_splitk<FMT, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, S, st);
+  if (N % 256 == 0 && tm * (N / 256) * 2 > t128)  // few tiles either way: keep the wide tile
+    return launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
+  return launch<FMT, 128, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
+}
+
 }  // namespace gemm
 
 int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                 const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int yt,
                 int64_t M, int64_t N, int64_t K, int f, cudaStream_t st) {
-  const bool n256 = (N % 256) == 0;
-#define DQ_G(FF)                                                                                 \
-  if (n256) return yt == 1 ? gemm::launch<FF, 256, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st) \
-                           : gemm::launch<FF, 256, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st); \
-  return yt == 1 ? gemm::launch<FF, 128, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)     \
-                 : gemm::launch<FF, 128, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
-  if (f == NVFP4) { DQ_G(NVFP4); }
-  if (f == MXFP4) { DQ_G(MXFP4); }
-#undef DQ_G
+  if (f == NVFP4)
+    return yt == 1 ? gemm::dispatch<NVFP4, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
+                   : gemm::dispatch<NVFP4, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
+  if (f == MXFP4)
+    return yt == 1 ? gemm::dispatch<MXFP4, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
+                   : gemm::dispatch<MXFP4, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
   return DQ_ERR_UNSUPPORTED;
 }
 

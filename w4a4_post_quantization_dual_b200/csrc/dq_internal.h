@@ -20,6 +20,12 @@ int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const u
                 const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int yt,
                 int64_t M, int64_t N, int64_t K, int f, cudaStream_t st);
 
+// Set the function attributes a launch needs (dynamic shared memory bytes,
+// the all-shared L1 carveout, and optionally non-portable cluster sizes)
+// once per kernel, device and size: they persist, and setting them on every call costs host time
+// comparable to a small kernel.  Keyed by the kernel's address.
+bool ensure_kernel_attrs(const void* kernel, int smem_bytes, bool big_cluster);
+
 // Device-side error word written by kernels whose bounded waits expire.
 int read_device_error(int clear);
 

@@ -366,14 +366,21 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
     int64_t grid = (int64_t)num_sms() * (2048 / NT);
     const int64_t groups = (Mpad + R - 1) / R;
     if (grid > groups) grid = groups;
-    if (bpt == 1)
-      quantize_act_rows_kernel<F, G, XT, 1, R><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
-    else if (bpt == 2)
-      quantize_act_rows_kernel<F, G, XT, 2, R / 2><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
-    else if (bpt <= 4)
-      quantize_act_rows_kernel<F, G, XT, 4, 1><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
-    else
+    if (bpt == 1) {
+      auto k = quantize_act_rows_kernel<F, G, XT, 1, R>;
+      if (!ensure_kernel_attrs((const void*)k, 0, false)) return DQ_ERR_CUDA;
+      k<<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
+    } else if (bpt == 2) {
+      auto k = quantize_act_rows_kernel<F, G, XT, 2, R / 2>;
+      if (!ensure_kernel_attrs((const void*)k, 0, false)) return DQ_ERR_CUDA;
+      k<<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
+    } else if (bpt <= 4) {
+      auto k = quantize_act_rows_kernel<F, G, XT, 4, 1>;
+      if (!ensure_kernel_attrs((const void*)k, 0, false)) return DQ_ERR_CUDA;
+      k<<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
+    } else {
       return DQ_ERR_UNSUPPORTED;
+    }
     return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
   }
   int64_t grid = (int64_t)num_sms() * (2048 / NT);
@@ -419,6 +426,7 @@ static int launch_pack(const void* W, int64_t m, int64_t n, const float* r, cons
     }
   }
   int64_t total = m * nb;
+  if (!ensure_kernel_attrs((const void*)pack_weight_kernel<F, G, WT>, 0, false)) return DQ_ERR_CUDA;
   pack_weight_kernel<F, G, WT><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
       reinterpret_cast<const WT*>(W), m, n, r, c, sT, codes, scales);
   return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;

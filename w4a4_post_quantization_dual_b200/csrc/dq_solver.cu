@@ -551,10 +551,7 @@ static void solver_geometry(int64_t m, int& steps, int& C, bool& wsmem) {
 
 template <typename K>
 static bool allow_big_cluster(K kern, size_t smem) {
-  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
-             cudaSuccess &&
-         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-             cudaSuccess;
+  return ensure_kernel_attrs((const void*)kern, (int)smem, true);
 }
 
 template <int F, int G, typename WT>
