@@ -177,8 +177,10 @@ DQ_API int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, con
  *           a per-row alpha outside the block scales.
  *  Y        out, M x N, dtype yt (DQ_BF16: round to nearest even; DQ_F32).
  * Formats: DQ_NVFP4 (kind::mxf4nvf4, UE4M3 scales, 16-blocks), DQ_MXFP4
- * (kind::mxf4, E8M0, 32-blocks); DQ_MXINT4 and DQ_INT4 return
- * DQ_ERR_UNSUPPORTED (no 4-bit integer tensor-core MMA on sm_100a).
+ * (kind::mxf4, E8M0, 32-blocks), DQ_MXINT4 (integer codes widened on chip to
+ * E4M3, exact for -8..7, kind::mxf8f6f4 with E8M0 32-block scales);
+ * DQ_INT4 returns DQ_ERR_UNSUPPORTED (bf16 group scales have no
+ * block-scaled tensor-core form on sm_100a).
  * Sizes: M >= 1, N % 128 == 0, K % 256 == 0; A, B, sA, sB 16-byte aligned.
  * FP32 accumulation in tensor memory.
  * ---------------------------------------------------------------------- */

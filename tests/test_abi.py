@@ -66,9 +66,7 @@ def test_invalid_arguments_rejected_without_launch(L):
     # NVFP4 activations need s_tok; K must be a multiple of 4*G for the MMA layout
     assert L.dq_quantize_act(fake, 1, 4, 64, None, 3, 16, fake, fake, None, None) == 1
     assert L.dq_quantize_act(fake, 1, 4, 48, None, 3, 16, fake, fake, fake, None) == 1
-    # GEMM: integer formats have no 4-bit tensor-core MMA on sm_100a
-    assert L.dq_w4a4_linear(fake, fake, fake, fake, fake, fake, None, fake, 1, 16, 128, 256,
-                            1, None) == 2
+    # GEMM: INT4 (bf16 group scales) has no block-scaled tensor-core form on sm_100a
     assert L.dq_w4a4_linear(fake, fake, fake, fake, fake, fake, None, fake, 1, 16, 128, 256,
                             0, None) == 2
     # GEMM shape rules: N % 128, K % 256, 16-byte alignment

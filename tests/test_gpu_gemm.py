@@ -29,7 +29,7 @@ def operands(M, N, K, fmt, seed=0, T=0, x_outliers=0.01, x_scale=50.0):
     return A, sA, st, B, sB, res["s_T"]
 
 
-@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4, O.MXINT4])
 @pytest.mark.parametrize("M,N,K", [(16, 256, 256), (1, 512, 4096), (300, 512, 768),
                                    (128, 128, 256), (257, 384, 512), (1000, 1024, 1024),
                                    (64, 4096, 4096), (8, 1024, 5120)])
@@ -58,6 +58,8 @@ def test_gemm_row_factor_epilogue():
     (O.NVFP4, 1, 1024, 4096),       # k/v projection, decode (split-K over a cluster)
     (O.NVFP4, 8, 27648, 5120),      # Qwen-32B up projection, decode
     (O.MXFP4, 2048, 14336, 4096),   # gate/up, MX
+    (O.MXINT4, 2048, 14336, 4096),  # gate/up, MXINT4 (widened on chip to E4M3)
+    (O.MXINT4, 2048, 4096, 14336),  # down, MXINT4
     (O.NVFP4, 8192, 5120, 27648),   # Qwen-32B down projection, prefill
 ])
 def test_gemm_full_size_sampled(fmt, M, N, K):

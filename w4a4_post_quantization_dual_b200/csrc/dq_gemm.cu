@@ -664,6 +664,277 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
 }
 
 // ---------------------------------------------------------------------------
+// MXINT4 linear.  sm_100a has no 4-bit integer tensor-core MMA, so the
+// integer codes (-8..7, exact in E4M3) are widened on chip: TMA stages the
+// packed codes, four converter warps turn each two's-complement nibble into
+// its E4M3 byte (byte-permute table lookups) and write the 128-byte-swizzled
+// K-major operand tiles, and tcgen05.mma.kind::mxf8f6f4 with E8M0 scales per
+// 32 elements (one scale byte per MMA, K = 32) accumulates in tensor memory.
+// Tiles 128 x 128, BK = 128 elements per stage, persistent.
+//   warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, warp 6 scale copies,
+//   warps 7..10 converters.
+// ---------------------------------------------------------------------------
+namespace i4 {
+constexpr int BN = 128, BKE = 128;                   // elements per k-tile
+constexpr int THREADS = 352;
+constexpr int STG_A = BM * BKE / 2, STG_B = BN * BKE / 2;      // packed staging (8 KB each)
+constexpr int OP_A = BM * BKE, OP_B = BN * BKE;                // E4M3 operands (16 KB each)
+constexpr int SF_A = 512, SF_B = 512;                          // one 128 x 4 atom each
+constexpr int STAGE = STG_A + STG_B + OP_A + OP_B + SF_A + SF_B;
+constexpr int STAGES = 4;
+constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+constexpr int SF_COLS = 8;                                     // 4 (A) + 4 (B) columns per slot
+constexpr int TMEM_COLS = 256;
+static_assert(BN + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
+static_assert(SMEM <= 227 * 1024, "shared memory budget");
+
+// Eight two's-complement INT4 codes (one 32-bit word, element k in nibble k)
+// -> eight E4M3 bytes (two words, element k in byte k).
+__device__ __forceinline__ uint2 widen8(uint32_t w) {
+  // E4M3 of 0..7 and of -8..-1 (indexed by the low three bits of the code)
+  constexpr uint32_t POS_LO = 0x44403800u, POS_HI = 0x4E4C4A48u;
+  constexpr uint32_t NEG_LO = 0xCACCCED0u, NEG_HI = 0xB8C0C4C8u;
+  uint32_t out[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t sel = (w >> (16 * h)) & 0xFFFFu;
+    const uint32_t pos = __byte_perm(POS_LO, POS_HI, sel);
+    const uint32_t neg = __byte_perm(NEG_LO, NEG_HI, sel);
+    // byte i from pos (selector i) or neg (selector 4 + i) by bit 3 of code i
+    const uint32_t pick = ((sel >> 1) & 0x4444u) | 0x3210u;
+    out[h] = __byte_perm(pos, neg, pick);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+__device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate, uint32_t tsfa,
+                                       uint32_t tsfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+}  // namespace i4
+
+template <int YT>
+__global__ void __launch_bounds__(i4::THREADS, 1)
+w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const uint8_t* __restrict__ sfA,
+                        const uint8_t* __restrict__ sfB, const float* __restrict__ r_row,
+                        void* __restrict__ Y, int M, int N, int K) {
+  using namespace i4;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* opA = smem;                              // 1024-aligned operand tiles
+  unsigned char* opB = opA + STAGES * OP_A;
+  unsigned char* stA = opB + STAGES * OP_B;
+  unsigned char* stB = stA + STAGES * STG_A;
+  unsigned char* sSFA = stB + STAGES * STG_B;
+  unsigned char* sSFB = sSFA + STAGES * SF_A;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SF_B);
+  uint64_t* empty = full + STAGES;
+  uint64_t* sfready = empty + STAGES;
+  uint64_t* conv = sfready + STAGES;
+  uint64_t* acc_full = conv + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_m = (M + BM - 1) / BM, tiles_n = N / BN, num_tiles = tiles_m * tiles_n;
+  const int KT = K / BKE;
+  const int S4 = (K / 32) / 4;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sfready[s], 1);
+      mbar_init(&conv[s], 4);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_base_slot)), "r"((uint32_t)TMEM_COLS) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_base_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&full[stage], STG_A + STG_B + SF_A + SF_B);
+          tma_load_2d(stA + stage * STG_A, &tmA, &full[stage], kt * (BKE / 2), m0);
+          tma_load_2d(stB + stage * STG_B, &tmB, &full[stage], kt * (BKE / 2), n0);
+          bulk_load(sSFA + stage * SF_A, sfA + ((size_t)(m0 / 128) * S4 + kt) * 512, SF_A,
+                    &full[stage]);
+          bulk_load(sSFB + stage * SF_B, sfB + ((size_t)(n0 / 128) * S4 + kt) * 512, SF_B,
+                    &full[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (ok)
+        for (int s = 0; s < STAGES; ++s) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      // kind::mxf8f6f4: E4M3 A and B (format 0), E8M0 scales, K-major, M = 128
+      const uint32_t idesc0 = ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24);
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        if (!mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag)) break;
+        fence_after_sync();
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&conv[stage], phase, abort_flag) ||
+              !mbar_wait(&sfready[stage], phase, abort_flag)) { ok = false; break; }
+          fence_after_sync();
+          const uint32_t a_base = smem_u32(opA + stage * OP_A);
+          const uint32_t b_base = smem_u32(opB + stage * OP_B);
+          const uint32_t sfa_col = BN + stage * SF_COLS, sfb_col = sfa_col + 4;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {      // K = 32 bytes per MMA in the 128-byte row
+            const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, LAYOUT_SW128);
+            const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, LAYOUT_SW128);
+            const uint32_t sf_id = (uint32_t)kk;  // scale byte kk of the 32-bit column
+            const uint32_t idesc = idesc0 | (sf_id << 29) | (sf_id << 4);
+            mma_f8(tmem, ad, bd, idesc, (kt > 0 || kk > 0) ? 1u : 0u,
+                   (tmem + sfa_col) | (sf_id << 30), (tmem + sfb_col) | (sf_id << 30));
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(acc_full);
+      }
+    }
+  } else if (warp == 6) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        bool ok = true;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          fence_after_sync();
+          const uint32_t sfa_col = BN + stage * SF_COLS;
+          tmem_cp_32x128b_x4(tmem + sfa_col, smem_desc(smem_u32(sSFA + stage * SF_A), 0, 128, LAYOUT_NONE));
+          tmem_cp_32x128b_x4(tmem + sfa_col + 4, smem_desc(smem_u32(sSFB + stage * SF_B), 0, 128, LAYOUT_NONE));
+          mma_commit(&sfready[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp >= 7) {
+    // converters: packed INT4 staging -> swizzled E4M3 operand tiles
+    const int ct = threadIdx.x - 7 * 32;        // 0..127
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int kt = 0; kt < KT; ++kt) {
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&full[stage], phase, abort_flag) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        // 16-byte packed chunks: A rows 0..127 (4 chunks each), then B rows
+#pragma unroll 2
+        for (int c = ct; c < (BM + BN) * 4; c += 128) {
+          const bool isB = c >= BM * 4;
+          const int cc = isB ? c - BM * 4 : c;
+          const int r = cc >> 2, kc = cc & 3;
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              (isB ? stB + stage * STG_B : stA + stage * STG_A) + r * 64 + kc * 16);
+          const uint2 w0 = widen8(v.x), w1 = widen8(v.y), w2 = widen8(v.z), w3 = widen8(v.w);
+          unsigned char* rowp = (isB ? opB + stage * OP_B : opA + stage * OP_A) + r * 128;
+          const int sw = r & 7;
+          *reinterpret_cast<uint4*>(rowp + (((2 * kc) ^ sw) << 4)) = make_uint4(w0.x, w0.y, w1.x, w1.y);
+          *reinterpret_cast<uint4*>(rowp + (((2 * kc + 1) ^ sw) << 4)) = make_uint4(w2.x, w2.y, w3.x, w3.y);
+        }
+        // make the generic-proxy writes visible to the tensor core (async proxy)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&conv[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else {
+    // epilogue (warps 2..5)
+    const int quad = warp & 3;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int row = (tile % tiles_m) * BM + quad * 32 + lane, n0 = (tile / tiles_m) * BN;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(acc_full, it & 1, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      fence_after_sync();
+      if constexpr (YT == 1) {
+        if (r_row)
+          epilogue_bf16<BN, true>(tmem, quad, lane, row, M, N, n0, 1.0f, r_row, Y, acc_empty);
+        else
+          epilogue_bf16<BN, false>(tmem, quad, lane, row, M, N, n0, 1.0f, r_row, Y, acc_empty);
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
+          if (c0 + 32 == BN) {
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          if (row < M) {
+            float* dst = reinterpret_cast<float*>(Y) + (size_t)row * N + n0 + c0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              float4 f = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                     __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+              if (r_row) {
+                f.x = __fmul_rn(f.x, __ldg(r_row + n0 + c0 + 4 * q));
+                f.y = __fmul_rn(f.y, __ldg(r_row + n0 + c0 + 4 * q + 1));
+                f.z = __fmul_rn(f.z, __ldg(r_row + n0 + c0 + 4 * q + 2));
+                f.w = __fmul_rn(f.w, __ldg(r_row + n0 + c0 + 4 * q + 3));
+              }
+              reinterpret_cast<float4*>(dst)[q] = f;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)TMEM_COLS) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -691,17 +962,17 @@ static PFN_encodeTiled get_encode() {
 struct MapEntry {
   const void* base;
   int64_t rows, kbytes;
-  int box_rows;
+  int box_rows, box_bytes;
   CUtensorMap map;
 };
 static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t kbytes,
-                     int box_rows) {
+                     int box_rows, int box_bytes = BKB) {
   constexpr int kEntries = 16;
   thread_local MapEntry cache[kEntries];
   thread_local int used = 0, next = 0;
   for (int i = 0; i < used; ++i)
     if (cache[i].base == base && cache[i].rows == rows && cache[i].kbytes == kbytes &&
-        cache[i].box_rows == box_rows) {
+        cache[i].box_rows == box_rows && cache[i].box_bytes == box_bytes) {
       *map = cache[i].map;
       return true;
     }
@@ -709,14 +980,17 @@ static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t k
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kbytes};
-  cuuint32_t box[2] = {(cuuint32_t)BKB, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw =
+      box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
   if (enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   MapEntry& e = cache[next];
-  e.base = base; e.rows = rows; e.kbytes = kbytes; e.box_rows = box_rows; e.map = *map;
+  e.base = base; e.rows = rows; e.kbytes = kbytes; e.box_rows = box_rows;
+  e.box_bytes = box_bytes; e.map = *map;
   next = (next + 1) % kEntries;
   if (used < kEntries) ++used;
   return true;
@@ -788,13 +1062,30 @@ static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, con
     return launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
   const int64_t t128 = tm * (N / 128);
   const int KT = (int)(K / BK);
+  // largest split that still fits one wave (one CTA per SM: the CTAs hold
+  // ~210 KB of shared memory each)
   int S = 1;
   for (int cand : {8, 4, 2})
-    if (S == 1 && KT % cand == 0 && t128 * cand <= 2 * sms && t128 * 2 <= sms) S = cand;
+    if (S == 1 && KT % cand == 0 && t128 * cand <= sms) S = cand;
   if (S > 1) return launch_splitk<FMT, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, S, st);
   if (N % 256 == 0 && tm * (N / 256) * 2 > t128)  // few tiles either way: keep the wide tile
     return launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
   return launch<FMT, 128, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
+}
+
+template <int YT>
+static int launch_mxint4(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB,
+                         const float* r_row, void* Y, int64_t M, int64_t N, int64_t K,
+                         cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K / 2, BM, i4::BKE / 2) || !make_map(&tb, B, N, K / 2, i4::BN, i4::BKE / 2))
+    return DQ_ERR_CUDA;
+  auto kern = w4a4_gemm_mxint4_kernel<YT>;
+  if (!ensure_kernel_attrs((const void*)kern, i4::SMEM, false)) return DQ_ERR_CUDA;
+  const int64_t tiles = ((M + BM - 1) / BM) * (N / i4::BN);
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  kern<<<grid, i4::THREADS, i4::SMEM, st>>>(ta, tb, sA, sB, r_row, Y, (int)M, (int)N, (int)K);
+  return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
 }
 
 }  // namespace gemm
@@ -808,6 +1099,9 @@ int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const u
   if (f == MXFP4)
     return yt == 1 ? gemm::dispatch<MXFP4, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
                    : gemm::dispatch<MXFP4, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
+  if (f == MXINT4)
+    return yt == 1 ? gemm::launch_mxint4<1>(A, sA, B, sB, r_row, Y, M, N, K, st)
+                   : gemm::launch_mxint4<0>(A, sA, B, sB, r_row, Y, M, N, K, st);
   return DQ_ERR_UNSUPPORTED;
 }
 
