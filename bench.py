@@ -29,7 +29,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from w4a4_post_quantization_dual_b200 import synth  # noqa: E402
+from w4a4_post_quantization_dual_b200 import dist, synth  # noqa: E402
 
 WORKLOAD = "llama8b_attn_nvfp4"
 METRIC = "W4A4 linear TFLOP/s & % of FP4 peak; BCD solver GB/s & % HBM peak"
@@ -282,14 +282,12 @@ def run_ours(args, rank, world, local_rank):
         rec["step"].append((e0, e2))
         rec["lin"].append((e1, e2))
 
-    if world > 1:
-        torch.distributed.barrier()
+    dist.barrier()
     for _ in range(args.warmup):
         flush.fill_(1)
         step({"solve": [], "act": [], "gemm": [], "step": [], "lin": []})
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    dist.barrier()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local_rank)
@@ -299,8 +297,7 @@ def run_ours(args, rank, world, local_rank):
         flush.fill_(rank + 1)      # L2 flush, outside the timed events
         step(rec)
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    dist.barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if dq.dq_device_error(clear=True) != 0:
@@ -314,10 +311,7 @@ def run_ours(args, rank, world, local_rank):
     solve_big = [el(p[:2]) for p in rec["solve"] if p[2] == big]
     gemm_pre = [(el((p[0], p[1])), p[2]) for p in rec["gemm"] if p[3] == prefill_M]
     act_pre = [(el((p[0], p[1])), p[2]) for p in rec["act"] if p[2] == prefill_M * 4096]
-    totals = torch.tensor([step_ms, lin_ms, solve_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(totals, op=torch.distributed.ReduceOp.MAX)
-    step_ms, lin_ms, solve_ms = totals.tolist()
+    step_ms, lin_ms, solve_ms = dist.max_over_ranks([step_ms, lin_ms, solve_ms], device=dev)
 
     # ---- e2e through the public API with host buffers (pinned), prefill linears
     e2e = None
@@ -373,7 +367,9 @@ def run_ours(args, rank, world, local_rank):
     a_ms = sum(t for t, _ in act_pre) / max(len(act_pre), 1)
     a_bytes = prefill_M * 4096 * (2 + 0.5 + 1.0 / 16) + prefill_M * 4
     act_gbs = a_bytes / (a_ms * 1e-3) / 1e9
-    value = lin_flops * args.steps / (lin_ms * 1e-3) / 1e12
+    # whole-job throughput: every rank runs the same per-GPU workload (weak
+    # scaling); the time is the slowest rank's
+    value = world * lin_flops * args.steps / (lin_ms * 1e-3) / 1e12
     per_m = {}
     for M in sorted(Xd):
         ga = [el((p[0], p[1])) for p in rec["gemm"] if p[3] == M]
@@ -438,25 +434,18 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local_rank = dist.env_ranks()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    if world > 1:
-        import datetime
-        backend = "nccl" if torch.cuda.is_available() and args.impl == "ours" else "gloo"
-        if backend == "nccl":
-            torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    backend = "nccl" if torch.cuda.is_available() and args.impl == "ours" else "gloo"
+    dist.init(backend, timeout_s=300)
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_ours(args, rank, world, local_rank)
     finally:
-        if world > 1:
-            torch.distributed.destroy_process_group()
+        dist.finalize()
 
 
 if __name__ == "__main__":
