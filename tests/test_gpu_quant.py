@@ -28,7 +28,8 @@ def _pad_expectation(sc_oracle, M, K, G, fmt):
 @pytest.mark.parametrize("fmt,G", FMTS)
 @pytest.mark.parametrize("M,K,xdt", [(16, 256, torch.float32), (1, 4096, torch.bfloat16),
                                      (17, 4096, torch.bfloat16), (300, 5120, torch.bfloat16),
-                                     (129, 14336, torch.bfloat16), (40, 27648, torch.bfloat16)])
+                                     (129, 14336, torch.bfloat16), (40, 27648, torch.bfloat16),
+                                     (4100, 4096, torch.bfloat16)])
 def test_act_quant_bit_exact(fmt, G, M, K, xdt):
     X, _ = synth.activations(M, K, 100 + M, n_outliers=max(1, K // 100), outlier_scale=50.0,
                              bf16=(xdt == torch.bfloat16))
@@ -63,6 +64,38 @@ def test_act_quant_rounding_boundaries():
         ocod, osc, ost = O.quantize_act(X, np.ones(K, np.float32), fmt, G)
         assert np.array_equal(cod, ocod), fmt
         assert np.array_equal(sc, osc), fmt
+
+
+@pytest.mark.parametrize("fmt,G", FMTS[:3])
+def test_act_quant_rounding_boundaries_bf16(fmt, G):
+    """The bf16 path: every E2M1 / INT4 midpoint in block-scale units (exact
+    in bf16), one bf16 ulp either side, saturation, signed zeros, zero blocks
+    and a block whose values all round to zero, in rows that span several
+    32-lane groups of blocks."""
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 7.0, 7.5, 0.0], np.float32)
+    up = torch.from_numpy(mids).to(torch.bfloat16)
+    nxt = lambda d: (up.view(torch.int16) + d).view(torch.bfloat16).float().numpy()
+    vals = np.concatenate([mids, nxt(1), nxt(-1)[mids > 0]])
+    row = np.concatenate([vals, -vals])
+    K = 2048
+    X = np.zeros((6, K), np.float32)
+    for off in range(0, K, 512):
+        X[0, off:off + row.size] = row
+    X[0, 31::64] = 7.96875       # MX block exponent floor(log2 7.97) - 2 = 0: unit scale
+    X[0, 63::64] = -7.96875
+    X[1] = X[0] * np.float32(2.0 ** -40)
+    X[2, 700:716] = np.float32(1e-3)  # a tiny block in a row whose token max is large
+    X[2, 5] = 1000.0
+    # rows 3..5 stay zero
+    X = torch.from_numpy(X).to(torch.bfloat16).float().numpy()
+    c = np.ones(K, np.float32)
+    c[100:140] = 2.0
+    cod, sc, st = gpu_act(X, c, fmt, G, torch.bfloat16)
+    ocod, osc, ost = O.quantize_act(X, c, fmt, G)
+    assert np.array_equal(cod, ocod)
+    assert np.array_equal(sc, osc)
+    if fmt == O.NVFP4:
+        assert np.array_equal(st.view(np.uint32), ost.view(np.uint32))
 
 
 @pytest.mark.parametrize("fmt,G", FMTS)

@@ -1113,7 +1113,8 @@ int read_device_error(int clear) {
     int z = 0;
     cudaMemcpyToSymbol(g_dq_device_error, &z, sizeof(int));
   }
-  return v;
+  const int q = read_quant_error(clear);
+  return v ? v : q;
 }
 
 }  // namespace dq

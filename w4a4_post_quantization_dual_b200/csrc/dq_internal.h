@@ -26,7 +26,9 @@ int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const u
 // comparable to a small kernel.  Keyed by the kernel's address.
 bool ensure_kernel_attrs(const void* kernel, int smem_bytes, bool big_cluster);
 
-// Device-side error word written by kernels whose bounded waits expire.
+// Device-side error words written by kernels whose bounded waits expire
+// (one per translation unit); read_device_error combines them.
 int read_device_error(int clear);
+int read_quant_error(int clear);
 
 }  // namespace dq

@@ -36,6 +36,20 @@ __device__ __forceinline__ void load_block(const XT* __restrict__ p, float* x) {
   }
 }
 
+template <typename XT, int G>
+__device__ __forceinline__ void load_block_smem(const XT* p, float* x) {
+  if constexpr (sizeof(XT) == 2) {
+#pragma unroll
+    for (int u = 0; u < G / 8; ++u) bf16x8_to_f32(reinterpret_cast<const uint4*>(p)[u], x + 8 * u);
+  } else {
+#pragma unroll
+    for (int u = 0; u < G / 4; ++u) {
+      float4 v = reinterpret_cast<const float4*>(p)[u];
+      x[4 * u] = v.x; x[4 * u + 1] = v.y; x[4 * u + 2] = v.z; x[4 * u + 3] = v.w;
+    }
+  }
+}
+
 // Codes of G grid arguments z -> G/2 bytes written to dst (16-byte aligned for G >= 32).
 template <int F, int G>
 __device__ __forceinline__ void store_codes(uint8_t* dst, const float* z) {
@@ -289,6 +303,334 @@ quantize_act_rows_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int6
 }
 
 // ---------------------------------------------------------------------------
+// Ring-buffered activation quantiser for the tensor-core formats, bf16 input.
+//
+// Rows of X are contiguous, so a group of RT rows is one bulk copy
+// (cp.async.bulk) into a ring of NST shared-memory stages that thread 0 keeps
+// in flight.  Row slot rt of a stage is handled by NTS threads; thread tl owns
+// blocks tl + j*NTS (j < BPT) of that row and keeps their column scales c and
+// the rescaled values x~ = x*c (Eq. 3) in registers.  A stage is therefore
+// read from shared memory exactly once, and is refilled right after the
+// barrier of the per-token reduction, while the codes are still being made.
+//
+// Conflict-free reads: a block is P = G/8 pieces of 16 bytes and lanes own
+// consecutive blocks; lane l starts at piece (l / (8/P)) mod P, so the 8 lanes
+// of each 128-byte shared-memory wavefront touch 8 distinct bank groups.  The
+// values stay in that rotated order (block maximum and scaling do not depend
+// on it) and the packed code words are rotated back before the store.
+// ---------------------------------------------------------------------------
+__device__ int g_dq_quant_error = 0;
+
+namespace aq {
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity) {
+  const uint64_t limit = 2000000000ull;  // 2 s, far beyond any legitimate wait
+  uint64_t t0 = 0;
+  for (int i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    if (ok) return true;
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (i == 0) t0 = t;
+    else if (t - t0 > limit) {
+      atomicExch(&g_dq_quant_error, DQ_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ float2 bf16pair(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ float absmax2(float2 v) { return fmaxf(fabsf(v.x), fabsf(v.y)); }
+// Eight values (four pairs) -> 32 bits of E2M1 codes, element k in nibble k.
+__device__ __forceinline__ uint32_t e2m1x8_pairs(const float2* z) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(z[0].x), "f"(z[0].y), "f"(z[1].x), "f"(z[1].y), "f"(z[2].x), "f"(z[2].y),
+        "f"(z[3].x), "f"(z[3].y));
+  return out;
+}
+// Eight values -> 32 bits of INT4 codes (round to nearest even, clip to
+// [-8, 7]), element k in nibble k.  |z| < 2^22 here, so adding 1.5 * 2^23
+// rounds to the nearest integer (ties to even) and leaves it in the low
+// mantissa bits; cvt.pack.sat.s4 clips and packs two integers per step.
+__device__ __forceinline__ uint32_t int4x8_pairs(const float2* z) {
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  int n[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __fadd2_rn(z[i], magic);
+    n[2 * i] = (int)__float_as_uint(t.x) - 0x4B400000;
+    n[2 * i + 1] = (int)__float_as_uint(t.y) - 0x4B400000;
+  }
+  uint32_t d = 0;
+#pragma unroll
+  for (int i = 3; i >= 0; --i)  // d = (d << 8) | sat(n[2i+1]) << 4 | sat(n[2i])
+    asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(n[2 * i + 1]), "r"(n[2 * i]), "r"(d));
+  return d;
+}
+}  // namespace aq
+
+// Block scale (byte of the layout) and reciprocal for one block of
+// block maximum ab; st is the per-token scale (NVFP4 only).
+template <int F>
+__device__ __forceinline__ void act_block_scale(float ab, float st, float d6, uint32_t& byte,
+                                                float& inv, bool& zero) {
+  if constexpr (F == NVFP4) {
+    byte = st > 0.0f ? ue4m3_rn(__fdiv_rn(ab, d6)) : 0u;
+    const float sblk = __fmul_rn(ue4m3_value(byte), st);
+    zero = (sblk == 0.0f);
+    inv = zero ? 0.0f : __frcp_rn(sblk);
+  } else {  // OCP MX rule: 2^(floor(log2 amax) - 2), E8M0 byte e + 127
+    int e = -127;
+    zero = !(ab > 0.0f);
+    if (!zero) {
+      e = ilog2f(ab) - 2;
+      e = e < -127 ? -127 : (e > 127 ? 127 : e);
+    }
+    byte = (uint32_t)(e + 127);
+    inv = pow2f(-e);
+  }
+}
+
+// Codes of one block (values xt in the rotated piece order), rotated back
+// and stored; all-zero codes when the block scale is zero.
+template <int F, int G>
+__device__ __forceinline__ void act_block_codes(const float2* xt, float inv, bool zero, int rot,
+                                                uint8_t* dst) {
+  constexpr int P = G / 8;
+  const float2 inv2 = make_float2(inv, inv);
+  uint32_t wv[P];
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    float2 z[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) z[h] = __fmul2_rn(xt[4 * p + h], inv2);
+    if constexpr (F == MXINT4) wv[p] = aq::int4x8_pairs(z);
+    else wv[p] = aq::e2m1x8_pairs(z);
+    if (zero) wv[p] = 0u;
+  }
+  // undo the piece rotation: code word q comes from wv[(q - rot) mod P]
+  if (rot & 1) {
+    const uint32_t last = wv[P - 1];
+#pragma unroll
+    for (int q = P - 1; q > 0; --q) wv[q] = wv[q - 1];
+    wv[0] = last;
+  }
+  if constexpr (P == 4) {
+    if (rot & 2) {
+      const uint32_t a0 = wv[0], a1 = wv[1];
+      wv[0] = wv[2]; wv[1] = wv[3]; wv[2] = a0; wv[3] = a1;
+    }
+  }
+  if constexpr (P == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(wv[0], wv[1]);
+  else *reinterpret_cast<uint4*>(dst) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+}
+
+// x~ = x*c for one block read from shared memory, and its absolute maximum.
+template <int G>
+__device__ __forceinline__ float act_block_load(const unsigned char* bp, const float2* cv, int rot,
+                                                float2* xt) {
+  constexpr int P = G / 8, H = G / 2;
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    const uint4 v = *reinterpret_cast<const uint4*>(bp + 16 * ((p + rot) & (P - 1)));
+    xt[4 * p + 0] = __fmul2_rn(aq::bf16pair(v.x), cv[4 * p + 0]);
+    xt[4 * p + 1] = __fmul2_rn(aq::bf16pair(v.y), cv[4 * p + 1]);
+    xt[4 * p + 2] = __fmul2_rn(aq::bf16pair(v.z), cv[4 * p + 2]);
+    xt[4 * p + 3] = __fmul2_rn(aq::bf16pair(v.w), cv[4 * p + 3]);
+  }
+  float m[H / 2];
+#pragma unroll
+  for (int h = 0; h < H / 2; ++h) m[h] = fmaxf(aq::absmax2(xt[2 * h]), aq::absmax2(xt[2 * h + 1]));
+#pragma unroll
+  for (int w = H / 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int h = 0; h < w; ++h) m[h] = fmaxf(m[h], m[h + w]);
+  return m[0];
+}
+
+template <int F, int G, int BPT, int MAXT, int MINB>
+__global__ void __launch_bounds__(MAXT, MINB)
+quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t Mpad, int64_t K,
+                         const float* __restrict__ c, uint8_t* __restrict__ codes,
+                         uint8_t* __restrict__ scales, float* __restrict__ s_tok, int NTS, int RT,
+                         int NST) {
+  constexpr int P = G / 8;   // 16-byte pieces per block
+  constexpr int LG = 8 / P;  // consecutive lanes sharing one piece rotation
+  constexpr int H = G / 2;   // value pairs per block
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const uint32_t row_bytes = (uint32_t)K * 2;
+  const uint32_t stage_bytes = row_bytes * (uint32_t)RT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + (size_t)stage_bytes * NST);
+  uint32_t* rowmax = reinterpret_cast<uint32_t*>(full + NST);  // [3][16] fp32 bits, >= 0
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(rowmax + 48);
+
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int rt = tid / NTS, tl = tid - rt * NTS;
+  const int rot = (lane / LG) % P;
+  const int S = (int)(K / G), S4 = S >> 2;
+
+  // per-thread constants of the owned blocks s = tl + j * NTS
+  bool own[BPT], sfw[BPT];
+  uint32_t boff[BPT], coff[BPT], sfo[BPT];
+  float2 cv[BPT][H];  // column scales, in the rotated piece order
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    const int s = tl + j * NTS;
+    own[j] = s < S;
+    sfw[j] = own[j] && (s & 3) == 0;
+    boff[j] = (uint32_t)rt * row_bytes + (uint32_t)s * (G * 2);
+    coff[j] = (uint32_t)s * (G / 2);
+    sfo[j] = ((uint32_t)(s >> 2) << 9) | (uint32_t)(s & 3);
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      const int q = (p + rot) & (P - 1);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float4 v = (c && own[j])
+                             ? __ldg(reinterpret_cast<const float4*>(c + (int64_t)s * G + q * 8) + h)
+                             : make_float4(1.f, 1.f, 1.f, 1.f);
+        cv[j][4 * p + 2 * h] = make_float2(v.x, v.y);
+        cv[j][4 * p + 2 * h + 1] = make_float2(v.z, v.w);
+      }
+    }
+  }
+  if (tid < 48) rowmax[tid] = 0u;
+  if (tid == 0) {
+    for (int i = 0; i < NST; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(aq::smem_u32(&full[i])));
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  const int64_t step = (int64_t)gridDim.x * RT;  // rows between consecutive groups of a CTA
+  auto issue = [&](int64_t t0, int stg) {         // rows t0.. -> stage stg
+    uint64_t* bar = &full[stg];
+    if (t0 < M) {
+      const int64_t rows = (M - t0) < RT ? (M - t0) : RT;
+      const uint32_t bytes = (uint32_t)rows * row_bytes;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                       aq::smem_u32(bar)), "r"(bytes) : "memory");
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+              "r"(aq::smem_u32(smem_raw + (size_t)stg * stage_bytes)),
+          "l"(X + t0 * K), "r"(bytes), "r"(aq::smem_u32(bar))
+          : "memory");
+    } else {  // padding rows only: nothing to load
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(aq::smem_u32(bar)) : "memory");
+    }
+  };
+  const int64_t first = (int64_t)blockIdx.x * RT;
+  if (tid == 0)
+    for (int k = 0; k < NST; ++k) issue(first + k * step, k);
+
+  int stg = 0, rb = 0;
+  uint32_t phase = 0;
+  int64_t t0 = first;
+  for (; t0 < Mpad; t0 += step) {
+    const int64_t t = t0 + rt;
+    const bool rowv = t < M, rowp = t < Mpad;  // both uniform over a warp
+    if (!aq::wait_parity(&full[stg], phase)) *abort_flag = 1;
+    const unsigned char* sp = smem_raw + (size_t)stg * stage_bytes;
+    uint8_t* crow = codes + t * (K / 2);
+    uint8_t* sfrow = scales + ((((t >> 7) * S4) << 9) + ((t & 31) << 4) + (((t & 127) >> 5) << 2));
+
+    if constexpr (F == NVFP4) {
+      // pass 1: x~ into registers, block maxima, per-token maximum
+      float2 xt[BPT][H];
+      float ab[BPT];
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < BPT; ++j) {
+        ab[j] = 0.0f;
+        if (rowv && own[j]) ab[j] = act_block_load<G>(sp + boff[j], cv[j], rot, xt[j]);
+        amax = fmaxf(amax, ab[j]);
+      }
+      // maxima are >= 0, so their bit patterns order like the values
+      const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+      if (lane == 0) atomicMax(&rowmax[rb * 16 + rt], wmax);
+      __syncthreads();  // the stage is consumed; per-token maxima are complete
+      if (*abort_flag) break;
+      if (tid == 0) issue(t0 + NST * step, stg);
+      const int rz = rb == 0 ? 2 : rb - 1;  // buffer last read one iteration ago
+      if (tid < 16) rowmax[rz * 16 + tid] = 0u;
+      // pass 2: block scales and codes
+      if (rowp) {
+        const float st = __fdiv_rn(__uint_as_float(rowmax[rb * 16 + rt]), 2688.0f);
+        const float d6 = __fmul_rn(6.0f, st);
+        if (tl == 0 && rowv) s_tok[t] = st;  // s_tok = amax / (6 * 448)
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) {
+          uint32_t byte = 0;
+          if (rowv && own[j]) {
+            float inv;
+            bool zero;
+            act_block_scale<F>(ab[j], st, d6, byte, inv, zero);
+            act_block_codes<F, G>(xt[j], inv, zero, rot, crow + coff[j]);
+          }
+          // the scale bytes of 4 consecutive blocks form one 32-bit word of
+          // the layout; gather them in the lane whose block index is a multiple of 4
+          const uint32_t b2 = byte | (__shfl_down_sync(0xffffffffu, byte, 1) << 8);
+          const uint32_t b4 = b2 | (__shfl_down_sync(0xffffffffu, b2, 2) << 16);
+          if (sfw[j]) *reinterpret_cast<uint32_t*>(sfrow + sfo[j]) = b4;
+        }
+      }
+      rb = rb == 2 ? 0 : rb + 1;
+    } else {
+      // MX: blocks are independent, one pass
+      if (rowp) {
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) {
+          uint32_t byte = 0;
+          if (rowv && own[j]) {
+            float2 xt[H];
+            const float ab = act_block_load<G>(sp + boff[j], cv[j], rot, xt);
+            float inv;
+            bool zero;
+            act_block_scale<F>(ab, 0.0f, 0.0f, byte, inv, zero);
+            act_block_codes<F, G>(xt, inv, zero, rot, crow + coff[j]);
+          }
+          const uint32_t b2 = byte | (__shfl_down_sync(0xffffffffu, byte, 1) << 8);
+          const uint32_t b4 = b2 | (__shfl_down_sync(0xffffffffu, b2, 2) << 16);
+          if (sfw[j]) *reinterpret_cast<uint32_t*>(sfrow + sfo[j]) = b4;
+        }
+      }
+      __syncthreads();  // the stage is consumed
+      if (*abort_flag) break;
+      if (tid == 0) issue(t0 + NST * step, stg);
+    }
+    if (++stg == NST) {
+      stg = 0;
+      phase ^= 1u;
+    }
+  }
+  if (*abort_flag && tid == 0) {
+    // a bounded wait expired: the group being processed and the NST - 1
+    // after it may still have copies in flight; let each land (each wait is
+    // bounded as well) before the CTA exits
+    for (int k = 0; k < NST; ++k) {
+      const int sk = stg + k < NST ? stg + k : stg + k - NST;
+      const uint32_t pk = stg + k < NST ? phase : phase ^ 1u;
+      if (t0 + k * step < M) aq::wait_parity(&full[sk], pk);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Weight packer: one thread per (row, block).
 // ---------------------------------------------------------------------------
 template <int F, int G, typename WT>
@@ -359,7 +701,38 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
   const int64_t Mpad = (F == INT4) ? M : ((M + 127) / 128) * 128;
   const XT* Xp = reinterpret_cast<const XT*>(X);
   if constexpr (F != INT4) {
-    // rows kernel: R rows per CTA iteration, BPT blocks per thread
+    if constexpr (sizeof(XT) == 2) {
+      // ring kernel: NTS threads per row, BPT blocks per thread, at most MAXT
+      // threads and MINB CTAs per SM (the register budget of each variant)
+      auto ring = [&](auto kern, int bpt2, int maxt, int minb) -> int {
+        const int NTS = (int)((S + bpt2 - 1) / bpt2 + 31) / 32 * 32;
+        int RT = maxt / NTS;
+        RT = RT > 16 ? 16 : RT;
+        const size_t stage = (size_t)K * sizeof(XT) * RT;
+        int NST = (int)((minb == 2 ? 100 * 1024 : 200 * 1024) / stage);
+        NST = NST > 8 ? 8 : NST;
+        if (RT < 1 || NST < 2) return -1;
+        const size_t smem = stage * NST + 8 * NST + 48 * 4 + 16;
+        int64_t grid = (Mpad + RT - 1) / RT;
+        if (grid > (int64_t)num_sms() * minb) grid = (int64_t)num_sms() * minb;
+        if (!ensure_kernel_attrs((const void*)kern, (int)smem, false)) return (int)DQ_ERR_CUDA;
+        kern<<<(unsigned)grid, NTS * RT, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(X), M,
+                                                     Mpad, K, c, codes, scales, s_tok, NTS, RT,
+                                                     NST);
+        return cudaGetLastError() == cudaSuccess ? (int)DQ_OK : (int)DQ_ERR_CUDA;
+      };
+      int rc = -1;
+      if constexpr (F == NVFP4) {
+        if (S <= 512) rc = ring(quantize_act_ring_kernel<F, G, 1, 512, 2>, 1, 512, 2);
+        else if (S <= 1024) rc = ring(quantize_act_ring_kernel<F, G, 2, 512, 1>, 2, 512, 1);
+      } else {
+        if (S <= 384) rc = ring(quantize_act_ring_kernel<F, G, 1, 384, 2>, 1, 384, 2);
+        else if (S <= 512) rc = ring(quantize_act_ring_kernel<F, G, 1, 512, 1>, 1, 512, 1);
+      }
+      if (rc >= 0) return rc;
+    }
+    // rows kernel (fp32 input, or rows too long for the register-resident ring):
+    // R rows per CTA iteration, BPT blocks per thread
     constexpr int R = (G == 16) ? 4 : 2;
     NT = (int)((S < 512 ? S : 512) + 31) / 32 * 32;
     const int bpt = (int)((S + NT - 1) / NT);
@@ -393,6 +766,16 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
     default: return DQ_ERR_UNSUPPORTED;
   }
   return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
+}
+
+int read_quant_error(int clear) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dq_quant_error, sizeof(int)) != cudaSuccess) return DQ_ERR_CUDA;
+  if (clear) {
+    int z = 0;
+    cudaMemcpyToSymbol(g_dq_quant_error, &z, sizeof(int));
+  }
+  return v;
 }
 
 int quantize_act(const void* X, int xt, int64_t M, int64_t K, const float* c, int f, int G,
