@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <stdlib.h>
+
 #include <mutex>
 #include <vector>
 
@@ -42,6 +44,14 @@ bool ensure_kernel_attrs(const void* kernel, int smem_bytes, bool big_cluster) {
   std::lock_guard<std::mutex> g(mu);
   done.push_back({kernel, dev, smem_bytes, big_cluster});
   return true;
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("DQ_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
 }
 
 }  // namespace dq

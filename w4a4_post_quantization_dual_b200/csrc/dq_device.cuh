@@ -72,12 +72,17 @@ __device__ __forceinline__ uint32_t ue4m3_rn(float x) {
       : "=r"(out) : "f"(x), "f"(0.0f));
   return out & 0xFFu;
 }
-// Value of a UE4M3 byte (0..126).
+// Value of a UE4M3 byte (0..126): every E4M3 value is exact in fp16, so the
+// hardware conversion e4m3 -> f16 followed by f16 -> f32 is exact.
 __device__ __forceinline__ float ue4m3_value(uint32_t b) {
-  uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
-  // normal: (1 + m/8) 2^(e-7) -> fp32 exponent e + 120, mantissa m << 20
-  // subnormal: m 2^-9
-  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
+  float f;
+  asm("{\n\t.reg .b16 t;\n\t.reg .b32 h;\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.u16.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h, t;\n\t"
+      "mov.b32 {lo, hi}, h;\n\t"
+      "cvt.f32.f16 %0, lo;\n\t}"
+      : "=f"(f) : "r"(b & 0xFFu));
+  return f;
 }
 
 // ---------------------------------------------------------------- E8M0
@@ -164,6 +169,13 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float* x) {
     x[2 * i] = __uint_as_float(w[i] << 16);
     x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
+}
+
+// Programmatic dependent launch (see pdl_enabled in dq_internal.h): wait for
+// the previous kernel of the stream to complete, and let the next one launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Block-scale layout of the block-scaled tensor-core MMA (see include/dq.h).

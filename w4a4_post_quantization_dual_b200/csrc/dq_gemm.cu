@@ -87,6 +87,10 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
   }
 }
 
+// Fetch a tensor map's descriptor ahead of its first use.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y) {
   asm volatile(
@@ -255,6 +259,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
   const int tiles_m = (M + BM - 1) / BM, tiles_n = N / BN;
   const int num_tiles = tiles_m * tiles_n;
   const int KT = K / BK;
@@ -282,6 +290,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_base_slot;
+  pdl_wait();     // operands and output may belong to the previous kernel of the stream
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -454,10 +464,12 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 // ---------------------------------------------------------------------------
 // Split-K variant for problems with few output tiles (small M): the S CTAs
 // of a thread-block cluster compute K-slices of the same 128 x 128 tile with
-// the same TMA / scale-copy / tcgen05 pipeline, drain their fp32 partial
-// tiles into shared memory, and after a cluster barrier each CTA sums one
-// column slice of the tile over DSMEM (in rank order), applies the epilogue
-// scales and stores.  No global workspace.
+// the same TMA / scale-copy / tcgen05 pipeline.  Each CTA owns one column
+// slice of the tile: while draining its fp32 partial tile from tensor memory
+// it stores every slice straight into the owner's shared memory (DSMEM);
+// after one cluster barrier each CTA sums its S partial slices from local
+// shared memory (in rank order), applies the epilogue scales and stores.
+// No global workspace.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -468,17 +480,21 @@ __device__ __forceinline__ void cluster_barrier() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
 }
-__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
-  uint32_t a = smem_u32(local), ra;
-  float v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
-  return v;
+// Store four floats at a shared-memory offset of CTA `rank` of the cluster
+// (16-byte aligned).  Ordered before the peers' reads by the cluster barrier
+// (release / acquire).
+__device__ __forceinline__ void st_dsmem_f32x4(uint32_t local_addr, uint32_t rank, uint32_t a,
+                                               uint32_t b, uint32_t c, uint32_t d) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ra), "r"(a), "r"(b),
+               "r"(c), "r"(d)
+               : "memory");
 }
 
 constexpr int SK_BN = 128;
-constexpr int SK_LD = SK_BN + 4;                  // padded row of the partial tile (floats)
-constexpr int SK_PART_BYTES = BM * SK_LD * 4;
+// partial slices received from the S CTAs of the cluster: [S][BM][BN / S] floats
+constexpr int SK_PART_BYTES = BM * SK_BN * 4;
 
 template <int FMT, int YT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -505,6 +521,10 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
   const uint32_t rank = cluster_rank(), S = gridDim.x;
   const int n0 = blockIdx.y * BN, m0 = blockIdx.z * BM;
   const int kt0 = (int)rank * kt_per_slice;
@@ -531,6 +551,8 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_base_slot;
+  pdl_wait();     // operands and output may belong to the previous kernel of the stream
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -612,48 +634,67 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
   } else {
-    // drain this CTA's partial tile (rows that exist) into shared memory
+    // drain this CTA's partial tile (rows that exist) straight into the
+    // shared memory of the CTA that reduces each column slice: owner q keeps
+    // slice [q * cols, (q + 1) * cols) of every rank, at part[rank][row][.]
     const int quad = warp & 3;
+    const int cols = BN / (int)S;
     int ok = 1;
     if (lane == 0) ok = mbar_wait(acc_full, 0, abort_flag) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok && m0 + quad * 32 < M) {
       fence_after_sync();
-      float* dst = part + (size_t)(quad * 32 + lane) * SK_LD;
+      const int row = quad * 32 + lane;
+      const uint32_t mine = smem_u32(part + ((size_t)rank * BM + row) * cols);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
 #pragma unroll
-        for (int k = 0; k < 32; k += 4)
-          *reinterpret_cast<float4*>(dst + c0 + k) =
-              make_float4(__uint_as_float(v[k]), __uint_as_float(v[k + 1]),
-                          __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+        for (int k = 0; k < 32; k += 4) {
+          const int c = c0 + k, q = c / cols;
+          st_dsmem_f32x4(mine + (uint32_t)(c - q * cols) * 4, (uint32_t)q, v[k], v[k + 1], v[k + 2],
+                         v[k + 3]);
+        }
       }
     }
   }
 
   fence_before_sync();
-  cluster_barrier();   // every CTA's partial tile is in its shared memory
+  cluster_barrier();   // every partial slice has landed in its owner's shared memory
   {
-    // this CTA reduces columns [rank * BN / S, (rank + 1) * BN / S) of the tile
-    const int cols = BN / (int)S, c_begin = (int)rank * cols;
+    // this CTA owns columns [rank * cols, (rank + 1) * cols) of the tile:
+    // sum the S partial slices (local shared memory, rank order), scale, store
+    const int cols = BN / (int)S, c4 = cols / 4, c_begin = (int)rank * cols;
     const int rows = (M - m0) < BM ? (M - m0) : BM;
+    const int total = rows * c4;
     const float sw = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
-    for (int idx = threadIdx.x; idx < rows * cols; idx += NUM_THREADS) {
-      const int r = idx / cols, c = c_begin + idx % cols;
-      float acc = 0.0f;
-      for (uint32_t q = 0; q < S; ++q) acc += ld_dsmem_f32(part + (size_t)r * SK_LD + c, q);
+    for (int idx = threadIdx.x; idx < total; idx += NUM_THREADS) {
+      const int r = idx / c4, cc = (idx % c4) * 4, c = c_begin + cc;
+      float4 acc = *reinterpret_cast<const float4*>(part + (size_t)r * cols + cc);
+      for (uint32_t q = 1; q < S; ++q) {
+        const float4 p = *reinterpret_cast<const float4*>(part + ((size_t)q * BM + r) * cols + cc);
+        acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+      }
       float rs = sw;
       if (FMT == NVFP4 && s_tok) rs = __fmul_rn(s_tok[m0 + r], sw);
-      float f = __fmul_rn(acc, rs);
-      if (r_row) f = __fmul_rn(f, __ldg(r_row + n0 + c));
+      float f[4] = {__fmul_rn(acc.x, rs), __fmul_rn(acc.y, rs), __fmul_rn(acc.z, rs),
+                    __fmul_rn(acc.w, rs)};
+      if (r_row) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) f[k] = __fmul_rn(f[k], __ldg(r_row + n0 + c + k));
+      }
       const size_t o = (size_t)(m0 + r) * N + n0 + c;
-      if constexpr (YT == 1) reinterpret_cast<__nv_bfloat16*>(Y)[o] = __float2bfloat16_rn(f);
-      else reinterpret_cast<float*>(Y)[o] = f;
+      if constexpr (YT == 1) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(f[0], f[1]), hi = __floats2bfloat162_rn(f[2], f[3]);
+        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(Y) + o) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+      } else {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(Y) + o) = make_float4(f[0], f[1], f[2], f[3]);
+      }
     }
   }
-  cluster_barrier();   // no CTA leaves while a peer may still read its partial tile
+  // no peer touches this CTA's shared memory after the barrier above
   __syncthreads();
   if (warp == 1) {
     fence_after_sync();
@@ -769,6 +810,8 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_base_slot;
+  pdl_wait();     // operands and output may belong to the previous kernel of the stream
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -1018,9 +1061,9 @@ static int launch(const uint8_t* A, const uint8_t* sA, const float* s_tok, const
   if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
   const int64_t tiles = ((M + BM - 1) / BM) * (N / BN);
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  kern<<<grid, NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, sA, sB, s_tok, s_w, r_row, Y, (int)M,
-                                                  (int)N, (int)K);
-  return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
+  const cudaError_t e = launch_ex(kern, dim3(grid), dim3(NUM_THREADS), C::SMEM_BYTES, st, 1, ta, tb,
+                                  sA, sB, s_tok, s_w, r_row, Y, (int)M, (int)N, (int)K);
+  return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
 }
 
 template <int FMT, int YT>
@@ -1032,23 +1075,44 @@ static int launch_splitk(const uint8_t* A, const uint8_t* sA, const float* s_tok
   if (!make_map(&ta, A, M, K / 2, BM) || !make_map(&tb, B, N, K / 2, SK_BN)) return DQ_ERR_CUDA;
   auto kern = w4a4_gemm_splitk_kernel<FMT, YT>;
   if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(S, (unsigned)(N / SK_BN), (unsigned)((M + BM - 1) / BM));
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   const int kt_per_slice = (int)(K / BK) / S;
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, sA, sB, s_tok, s_w, r_row, Y, (int)M, (int)N,
-                         (int)K, kt_per_slice) != cudaSuccess)
+  if (launch_ex(kern, dim3(S, (unsigned)(N / SK_BN), (unsigned)((M + BM - 1) / BM)),
+                dim3(NUM_THREADS), C::SMEM_BYTES, st, (unsigned)S, ta, tb, sA, sB, s_tok, s_w,
+                r_row, Y, (int)M, (int)N, (int)K, kt_per_slice) != cudaSuccess)
     return DQ_ERR_CUDA;
   return DQ_OK;
+}
+
+// How many clusters of S split-K CTAs the device runs at once (each CTA
+// takes one SM's shared memory; a cluster must fit inside one GPC).
+template <int FMT, int YT>
+static int splitk_max_clusters(int S) {
+  static int cache[16][9];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16 || S < 1 || S > 8) return 0;
+  if (cache[dev][S]) return cache[dev][S] > 0 ? cache[dev][S] : 0;
+  using C = Cfg<FMT, SK_BN, SK_PART_BYTES>;
+  auto kern = w4a4_gemm_splitk_kernel<FMT, YT>;
+  int n = 0;
+  if (ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void*)kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+  }
+  cache[dev][S] = n > 0 ? n : -1;
+  return n > 0 ? n : 0;
 }
 
 // Tile-shape policy: 128 x 256 persistent tiles when they fill the machine,
@@ -1062,11 +1126,12 @@ static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, con
     return launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
   const int64_t t128 = tm * (N / 128);
   const int KT = (int)(K / BK);
-  // largest split that still fits one wave (one CTA per SM: the CTAs hold
-  // ~210 KB of shared memory each)
+  // largest split whose clusters (one per output tile) all run in one wave
   int S = 1;
   for (int cand : {8, 4, 2})
-    if (S == 1 && KT % cand == 0 && t128 * cand <= sms) S = cand;
+    if (S == 1 && KT % cand == 0 && t128 * cand <= sms &&
+        t128 <= splitk_max_clusters<FMT, YT>(cand))
+      S = cand;
   if (S > 1) return launch_splitk<FMT, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, S, st);
   if (N % 256 == 0 && tm * (N / 256) * 2 > t128)  // few tiles either way: keep the wide tile
     return launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
@@ -1084,8 +1149,9 @@ static int launch_mxint4(const uint8_t* A, const uint8_t* sA, const uint8_t* B, 
   if (!ensure_kernel_attrs((const void*)kern, i4::SMEM, false)) return DQ_ERR_CUDA;
   const int64_t tiles = ((M + BM - 1) / BM) * (N / i4::BN);
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  kern<<<grid, i4::THREADS, i4::SMEM, st>>>(ta, tb, sA, sB, r_row, Y, (int)M, (int)N, (int)K);
-  return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
+  const cudaError_t e = launch_ex(kern, dim3(grid), dim3(i4::THREADS), i4::SMEM, st, 1, ta, tb, sA,
+                                  sB, r_row, Y, (int)M, (int)N, (int)K);
+  return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
 }
 
 }  // namespace gemm

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/dq.h"
 
 namespace dq {
@@ -25,6 +27,44 @@ int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const u
 // once per kernel, device and size: they persist, and setting them on every call costs host time
 // comparable to a small kernel.  Keyed by the kernel's address.
 bool ensure_kernel_attrs(const void* kernel, int smem_bytes, bool big_cluster);
+
+// Programmatic dependent launch for the inference kernels (activation
+// quantiser, GEMMs).  Launched with programmatic stream serialisation, a
+// kernel may begin while the previous kernel of the stream is still
+// finishing; each such kernel therefore runs only its prologue (barrier
+// set-up, tensor-memory allocation, descriptor prefetch) before pdl_wait(),
+// which returns once the previous kernel has completed and its memory is
+// visible, and calls pdl_trigger() right after so that the next kernel's
+// launch overlaps its own work.  Without the launch attribute both are no-ops.
+// Setting DQ_PDL=0 in the environment launches without the attribute.
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, unsigned cluster_x, Args&&... args) {
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Device-side error words written by kernels whose bounded waits expire
 // (one per translation unit); read_device_error combines them.

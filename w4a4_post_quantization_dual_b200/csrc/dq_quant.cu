@@ -83,6 +83,8 @@ quantize_act_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int64_t K
                     const float* __restrict__ c, uint8_t* __restrict__ codes,
                     uint8_t* __restrict__ scales, float* __restrict__ s_tok) {
   __shared__ float red[32];
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x, NT = blockDim.x;
   const int64_t S = K / G;
   for (int64_t t = blockIdx.x; t < Mpad; t += gridDim.x) {
@@ -182,6 +184,8 @@ quantize_act_rows_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int6
                          uint8_t* __restrict__ scales, float* __restrict__ s_tok) {
   constexpr int PIECES = G * (int)sizeof(XT) / 16;   // 16-byte loads per block
   __shared__ float red[2][R][16];
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int NWARP = (NT + 31) >> 5;
   const int64_t S = K / G;
@@ -484,17 +488,29 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
   const int S = (int)(K / G), S4 = S >> 2;
 
   // per-thread constants of the owned blocks s = tl + j * NTS
-  bool own[BPT], sfw[BPT];
+  bool own[BPT];
   uint32_t boff[BPT], coff[BPT], sfo[BPT];
-  float2 cv[BPT][H];  // column scales, in the rotated piece order
 #pragma unroll
   for (int j = 0; j < BPT; ++j) {
     const int s = tl + j * NTS;
     own[j] = s < S;
-    sfw[j] = own[j] && (s & 3) == 0;
     boff[j] = (uint32_t)rt * row_bytes + (uint32_t)s * (G * 2);
     coff[j] = (uint32_t)s * (G / 2);
     sfo[j] = ((uint32_t)(s >> 2) << 9) | (uint32_t)(s & 3);
+  }
+  if (tid < 48) rowmax[tid] = 0u;
+  if (tid == 0) {
+    for (int i = 0; i < NST; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(aq::smem_u32(&full[i])));
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  pdl_wait();     // inputs and outputs may belong to the previous kernel of the stream
+  pdl_trigger();
+  float2 cv[BPT][H];  // column scales of the owned blocks, in the rotated piece order
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    const int s = tl + j * NTS;
 #pragma unroll
     for (int p = 0; p < P; ++p) {
       const int q = (p + rot) & (P - 1);
@@ -507,13 +523,6 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
         cv[j][4 * p + 2 * h + 1] = make_float2(v.z, v.w);
       }
     }
-  }
-  if (tid < 48) rowmax[tid] = 0u;
-  if (tid == 0) {
-    for (int i = 0; i < NST; ++i)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(aq::smem_u32(&full[i])));
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
@@ -582,11 +591,9 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
             act_block_scale<F>(ab[j], st, d6, byte, inv, zero);
             act_block_codes<F, G>(xt[j], inv, zero, rot, crow + coff[j]);
           }
-          // the scale bytes of 4 consecutive blocks form one 32-bit word of
-          // the layout; gather them in the lane whose block index is a multiple of 4
-          const uint32_t b2 = byte | (__shfl_down_sync(0xffffffffu, byte, 1) << 8);
-          const uint32_t b4 = b2 | (__shfl_down_sync(0xffffffffu, b2, 2) << 16);
-          if (sfw[j]) *reinterpret_cast<uint32_t*>(sfrow + sfo[j]) = b4;
+          // one scale byte per block: the 4 bytes of a layout word come from
+          // 4 consecutive lanes of the same store instruction
+          if (own[j]) sfrow[sfo[j]] = (uint8_t)byte;
         }
       }
       rb = rb == 2 ? 0 : rb + 1;
@@ -604,9 +611,7 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
             act_block_scale<F>(ab, 0.0f, 0.0f, byte, inv, zero);
             act_block_codes<F, G>(xt, inv, zero, rot, crow + coff[j]);
           }
-          const uint32_t b2 = byte | (__shfl_down_sync(0xffffffffu, byte, 1) << 8);
-          const uint32_t b4 = b2 | (__shfl_down_sync(0xffffffffu, b2, 2) << 16);
-          if (sfw[j]) *reinterpret_cast<uint32_t*>(sfrow + sfo[j]) = b4;
+          if (own[j]) sfrow[sfo[j]] = (uint8_t)byte;
         }
       }
       __syncthreads();  // the stage is consumed
@@ -716,10 +721,11 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
         int64_t grid = (Mpad + RT - 1) / RT;
         if (grid > (int64_t)num_sms() * minb) grid = (int64_t)num_sms() * minb;
         if (!ensure_kernel_attrs((const void*)kern, (int)smem, false)) return (int)DQ_ERR_CUDA;
-        kern<<<(unsigned)grid, NTS * RT, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(X), M,
-                                                     Mpad, K, c, codes, scales, s_tok, NTS, RT,
-                                                     NST);
-        return cudaGetLastError() == cudaSuccess ? (int)DQ_OK : (int)DQ_ERR_CUDA;
+        const cudaError_t e =
+            launch_ex(kern, dim3((unsigned)grid), dim3(NTS * RT), smem, st, 1,
+                      reinterpret_cast<const __nv_bfloat16*>(X), M, Mpad, K, c, codes, scales,
+                      s_tok, NTS, RT, NST);
+        return e == cudaSuccess ? (int)DQ_OK : (int)DQ_ERR_CUDA;
       };
       int rc = -1;
       if constexpr (F == NVFP4) {
@@ -742,15 +748,21 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
     if (bpt == 1) {
       auto k = quantize_act_rows_kernel<F, G, XT, 1, R>;
       if (!ensure_kernel_attrs((const void*)k, 0, false)) return DQ_ERR_CUDA;
-      k<<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
+      if (launch_ex(k, dim3((unsigned)grid), dim3(NT), 0, st, 1, Xp, M, Mpad, K, c, codes, scales,
+                    s_tok) != cudaSuccess)
+        return DQ_ERR_CUDA;
     } else if (bpt == 2) {
       auto k = quantize_act_rows_kernel<F, G, XT, 2, R / 2>;
       if (!ensure_kernel_attrs((const void*)k, 0, false)) return DQ_ERR_CUDA;
-      k<<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
+      if (launch_ex(k, dim3((unsigned)grid), dim3(NT), 0, st, 1, Xp, M, Mpad, K, c, codes, scales,
+                    s_tok) != cudaSuccess)
+        return DQ_ERR_CUDA;
     } else if (bpt <= 4) {
       auto k = quantize_act_rows_kernel<F, G, XT, 4, 1>;
       if (!ensure_kernel_attrs((const void*)k, 0, false)) return DQ_ERR_CUDA;
-      k<<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok);
+      if (launch_ex(k, dim3((unsigned)grid), dim3(NT), 0, st, 1, Xp, M, Mpad, K, c, codes, scales,
+                    s_tok) != cudaSuccess)
+        return DQ_ERR_CUDA;
     } else {
       return DQ_ERR_UNSUPPORTED;
     }
@@ -758,14 +770,24 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
   }
   int64_t grid = (int64_t)num_sms() * (2048 / NT);
   if (grid > Mpad) grid = Mpad;
+  cudaError_t e;
   switch (bpt) {
-    case 1: quantize_act_kernel<F, G, XT, 1><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok); break;
-    case 2: quantize_act_kernel<F, G, XT, 2><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok); break;
+    case 1:
+      e = launch_ex(quantize_act_kernel<F, G, XT, 1>, dim3((unsigned)grid), dim3(NT), 0, st, 1, Xp,
+                    M, Mpad, K, c, codes, scales, s_tok);
+      break;
+    case 2:
+      e = launch_ex(quantize_act_kernel<F, G, XT, 2>, dim3((unsigned)grid), dim3(NT), 0, st, 1, Xp,
+                    M, Mpad, K, c, codes, scales, s_tok);
+      break;
     case 3:
-    case 4: quantize_act_kernel<F, G, XT, 4><<<(unsigned)grid, NT, 0, st>>>(Xp, M, Mpad, K, c, codes, scales, s_tok); break;
+    case 4:
+      e = launch_ex(quantize_act_kernel<F, G, XT, 4>, dim3((unsigned)grid), dim3(NT), 0, st, 1, Xp,
+                    M, Mpad, K, c, codes, scales, s_tok);
+      break;
     default: return DQ_ERR_UNSUPPORTED;
   }
-  return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
+  return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
 }
 
 int read_quant_error(int clear) {
