@@ -44,6 +44,23 @@ def test_gemm_small_parity(fmt, M, N, K):
     assert np.mean(Y16 == ref16) >= 0.99
 
 
+@pytest.mark.parametrize("fmt,M,N,K", [(O.NVFP4, 300, 9216, 512), (O.MXFP4, 200, 9216, 768),
+                                        (O.NVFP4, 512, 8960, 256)])
+def test_gemm_paired_tiles_parity(fmt, M, N, K):
+    """Shapes with enough 256 x 256 tiles for the paired-SM kernel, including
+    a ragged last tile whose second CTA lies entirely beyond M, and the
+    per-output-row factor in its epilogue."""
+    A, sA, st, B, sB, sW = operands(M, N, K, fmt, seed=M + K)
+    rr = np.exp(np.random.default_rng(1).uniform(-1, 1, N)).astype(np.float32)
+    ref = O.linear(A, sA, st, B, sB, sW, M, N, K, fmt, r_row=rr)
+    Y32 = gpu_linear(A, sA, st, B, sB, sW, M, N, K, fmt, torch.float32, r_row=rr)
+    assert rel_fro(Y32, ref) <= 1e-3
+    Y16 = gpu_linear(A, sA, st, B, sB, sW, M, N, K, fmt, torch.bfloat16, r_row=rr)
+    ref16 = bf16_round(ref)
+    assert rel_fro(Y16, ref16) <= 1e-3
+    assert np.mean(Y16 == ref16) >= 0.99
+
+
 def test_gemm_row_factor_epilogue():
     M, N, K = 64, 256, 512
     A, sA, st, B, sB, sW = operands(M, N, K, O.NVFP4, seed=3)

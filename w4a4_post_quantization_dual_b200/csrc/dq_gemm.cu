@@ -18,16 +18,17 @@
 //               accumulation in tensor memory; commits free the ring slots.
 //   warps 2..5  epilogue: tcgen05.ld the accumulator (each warp its 32-lane
 //               quadrant), release it to the MMA warp, scale, convert, store.
-//   warp 6      copies each stage's scale atoms into that stage's own slot of
-//               tensor memory (tcgen05.cp 32x128b.warpx4) and signals the MMA
-//               warp, so the copies for later stages run while the MMAs of
-//               the current stage execute (issued by the MMA thread itself,
-//               the copies serialise with the MMAs).
+//   warps 6..9  copy each stage's scale atoms into that stage's own slot of
+//               tensor memory (tcgen05.cp 32x128b.warpx4), a quarter each,
+//               and signal the MMA warp: a thread's copies run one after
+//               another at about an MMA's duration each, but the copies of
+//               different warps overlap each other and the MMAs.
 // Every mbarrier wait is bounded (globaltimer); on expiry the kernel records
 // DQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "dq_device.cuh"
 #include "dq_internal.h"
@@ -41,7 +42,13 @@ namespace gemm {
 constexpr int BM = 128;
 constexpr int BK = 256;             // four-bit elements per k-tile (128 bytes per row)
 constexpr int BKB = BK / 2;         // bytes per row per k-tile
-constexpr int NUM_THREADS = 224;
+constexpr int NUM_THREADS = 320;
+// Scale-factor copies: one tcgen05.cp occupies its issuing thread's queue for
+// roughly an MMA's time, while copies issued by different warps run
+// concurrently with each other and with the MMAs.  Four copier warps
+// (6..9) therefore share each stage's scale atoms round-robin.
+constexpr int COPIERS = 4;
+constexpr int FIRST_COPIER = 6;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -272,7 +279,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&sfready[s], 1);
+      mbar_init(&sfready[s], COPIERS);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
@@ -371,9 +378,12 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         mma_commit(acc_full);
       }
     }
-  } else if (warp == 6) {
-    // ------------------------------------------------------------ scale copier
+  } else if (warp >= FIRST_COPIER && warp < FIRST_COPIER + COPIERS) {
+    // ------------------------------------------------------------ scale copiers
+    // atom a of a stage (SFA atoms first, then the SFB groups) goes to copier
+    // a % COPIERS; each copier commits to the stage's sfready barrier
     if (lane == 0) {
+      const int me = warp - FIRST_COPIER;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -385,22 +395,22 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const uint32_t sfb_base = smem_u32(sSFB + stage * C::SFB_BYTES);
           const uint32_t sfa0 = C::SF_BASE + stage * C::SF_COLS;
           const uint32_t sfb0 = sfa0 + 4 * C::SF_ATOMS;
-#pragma unroll
-          for (int j = 0; j < C::SF_ATOMS; ++j)
-            tmem_cp_32x128b_x4(tmem + sfa0 + 4 * j, smem_desc(sfa_base + j * 512, 0, 128, LAYOUT_NONE));
-#pragma unroll
-          for (int g = 0; g < BN / 128; ++g)
-#pragma unroll
-            for (int j = 0; j < C::SF_ATOMS; ++j)
+          for (int a = me; a < C::SF_ATOMS * (1 + BN / 128); a += COPIERS) {
+            if (a < C::SF_ATOMS) {
+              tmem_cp_32x128b_x4(tmem + sfa0 + 4 * a, smem_desc(sfa_base + a * 512, 0, 128, LAYOUT_NONE));
+            } else {
+              const int g = (a - C::SF_ATOMS) / C::SF_ATOMS, j = (a - C::SF_ATOMS) % C::SF_ATOMS;
               tmem_cp_32x128b_x4(tmem + sfb0 + 4 * (BN / 128) * j + 4 * g,
                                  smem_desc(sfb_base + (g * C::SF_ATOMS + j) * 512, 0, 128,
                                            LAYOUT_NONE));
+            }
+          }
           mma_commit(&sfready[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;                 // tensor-memory lane quadrant of this warp
     const float sw = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
@@ -534,7 +544,7 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&sfready[s], 1);
+      mbar_init(&sfready[s], COPIERS);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -613,8 +623,9 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
       }
       if (ok) mma_commit(acc_full);
     }
-  } else if (warp == 6) {
+  } else if (warp >= FIRST_COPIER && warp < FIRST_COPIER + COPIERS) {
     if (lane == 0) {
+      const int me = warp - FIRST_COPIER;
       int stage = 0;
       uint32_t phase = 0;
       for (int kt = 0; kt < kt_per_slice; ++kt) {
@@ -624,16 +635,18 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t sfb_base = smem_u32(sSFB + stage * C::SFB_BYTES);
         const uint32_t sfa0 = C::SF_BASE + stage * C::SF_COLS;
         const uint32_t sfb0 = sfa0 + 4 * C::SF_ATOMS;
-#pragma unroll
-        for (int j = 0; j < C::SF_ATOMS; ++j) {
-          tmem_cp_32x128b_x4(tmem + sfa0 + 4 * j, smem_desc(sfa_base + j * 512, 0, 128, LAYOUT_NONE));
-          tmem_cp_32x128b_x4(tmem + sfb0 + 4 * j, smem_desc(sfb_base + j * 512, 0, 128, LAYOUT_NONE));
+        for (int a = me; a < 2 * C::SF_ATOMS; a += COPIERS) {
+          if (a < C::SF_ATOMS)
+            tmem_cp_32x128b_x4(tmem + sfa0 + 4 * a, smem_desc(sfa_base + a * 512, 0, 128, LAYOUT_NONE));
+          else
+            tmem_cp_32x128b_x4(tmem + sfb0 + 4 * (a - C::SF_ATOMS),
+                               smem_desc(sfb_base + (a - C::SF_ATOMS) * 512, 0, 128, LAYOUT_NONE));
         }
         mma_commit(&sfready[stage]);
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // drain this CTA's partial tile (rows that exist) straight into the
     // shared memory of the CTA that reduces each column slice: owner q keeps
     // slice [q * cols, (q + 1) * cols) of every rank, at part[rank][row][.]
@@ -699,6 +712,369 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
   if (warp == 1) {
     fence_after_sync();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Paired-SM variant for large problems: one 256 x 256 output tile per
+// cluster of two CTAs (one per SM), tcgen05.mma.cta_group::2.  Each CTA
+// loads its own 128 rows of A, its own 128 columns of B, the block scales
+// of its A rows and all 256 B scale rows; the even CTA ("leader") issues the
+// scale copies and the MMAs for both, which read A and the scale copies from
+// each CTA's own shared memory, B from both, and accumulate 128 x 256 in each
+// CTA's tensor memory.  Per 256 x 256 tile the pair reads 512 operand rows
+// from L2 instead of the 768 that two 128 x 256 tiles need.
+//   warp 0      TMA producer (both CTAs; completions counted on the leader's
+//               barrier, the cta_group::2 form of the tensor copy, no multicast)
+//   warp 1      tensor-memory allocation (both); MMA issuer (leader)
+//   warps 2..5  epilogue (both), each CTA its own 128 rows
+//   warps 6..9  scale copiers (leader): tcgen05.cp.cta_group::2, each a
+//               quarter of every stage's atoms
+// ---------------------------------------------------------------------------
+namespace pair {
+constexpr int BN = 256;                             // output columns per tile
+template <int FMT>
+struct Cfg2 {
+  static constexpr int G = (FMT == NVFP4) ? 16 : 32;
+  static constexpr int SF_ATOMS = (BK / G) / 4;     // 512-byte atoms per 128 rows per k-tile
+  static constexpr int A_BYTES = BM * BKB;          // own 128 rows
+  static constexpr int B_BYTES = 128 * BKB;         // own 128 columns
+  static constexpr int SFA_BYTES = SF_ATOMS * 512;
+  static constexpr int SFB_BYTES = 2 * SF_ATOMS * 512;  // all 256 scale rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = (227 * 1024 - 1024 - 256) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static constexpr int SF_COLS = 4 * SF_ATOMS * 3;  // SFA (one group) + SFB (two groups)
+  static constexpr int SF_BASE = BN;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int K_STEPS = BK / 64;
+  static_assert(SF_BASE + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
+  static_assert(4 * STAGES * 8 + 32 <= 256, "barrier area");
+  static_assert(STAGES >= 3, "pipeline depth");
+};
+
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// Tensor copy into this CTA's shared memory whose completion is counted on
+// the pair leader's barrier (cluster address `bar`).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar,
+                                                 int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_cp_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+template <int FMT>
+__device__ __forceinline__ void mma_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate, uint32_t tsfa,
+                                         uint32_t tsfb) {
+  if constexpr (FMT == NVFP4) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+        : "memory");
+  }
+}
+// Arrive on the barrier at the same offset in both CTAs of the pair once the
+// leader's earlier tcgen05 operations have completed.
+__device__ __forceinline__ void commit_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+      ::"r"(smem_u32(bar)), "h"((uint16_t)0x3)
+      : "memory");
+}
+// Arrive on the leader's own barrier once its earlier tcgen05 operations completed.
+__device__ __forceinline__ void commit_leader(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+__device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (barriers that receive arrivals
+// from the other CTA of the pair).
+__device__ __noinline__ bool wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+      *abort_flag = 1;
+      atomicExch(&g_dq_device_error, DQ_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+// Instruction descriptor: E2M1 A and B, K-major, M = 256 (the pair), N = 256.
+__host__ __device__ constexpr uint32_t idesc_pair(bool e8m0_scales) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((e8m0_scales ? 1u : 0u) << 23) |
+         ((uint32_t)(256 >> 4) << 24);
+}
+}  // namespace pair
+
+template <int FMT, int YT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmSFA,
+                      const __grid_constant__ CUtensorMap tmSFB, const float* __restrict__ s_tok,
+                      const float* __restrict__ s_w, const float* __restrict__ r_row,
+                      void* __restrict__ Y, int M, int N, int K) {
+  using C = pair::Cfg2<FMT>;
+  constexpr int BN = pair::BN;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* sA = smem;
+  unsigned char* sB = sA + C::STAGES * C::A_BYTES;
+  unsigned char* sSFA = sB + C::STAGES * C::B_BYTES;
+  unsigned char* sSFB = sSFA + C::STAGES * C::SFA_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + C::STAGES * C::SFB_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* sfready = empty + C::STAGES;
+  uint64_t* acc_full = sfready + C::STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();            // 0: leader, 1: peer
+  const bool leader = rank == 0;
+  const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  const int tiles_m = (M + 255) / 256, tiles_n = N / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int KT = K / BK;
+  const int S4 = (K / C::G) / 4;                   // scale atoms along K per 128-row block
+  constexpr uint32_t TX = 2u * C::STAGE_BYTES;     // both CTAs' bytes per stage
+
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmSFA);
+    prefetch_tmap(&tmSFB);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sfready[s], COPIERS);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);                       // 4 epilogue warps in each CTA
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_base_slot)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  cluster_barrier();   // both CTAs' barriers are initialised before any remote use
+  fence_after_sync();
+  const uint32_t tmem = *tmem_base_slot;
+  pdl_wait();     // operands and output may belong to the previous kernel of the stream
+  pdl_trigger();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
+        const int tm = tile % tiles_m, tn = tile / tiles_m;
+        const int m_own = tm * 256 + (int)rank * 128, n_own = tn * BN + (int)rank * 128;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          const uint32_t bar = pair::mapa(smem_u32(&full[stage]), 0);
+          if (leader) mbar_expect_tx(&full[stage], TX);
+          pair::tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kt * BKB, m_own);
+          pair::tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kt * BKB, n_own);
+          // scale atoms as rows of 256 bytes: atom a of row block rb is rows 2a, 2a + 1
+          pair::tma_load_2d_pair(sSFA + stage * C::SFA_BYTES, &tmSFA, bar, 0,
+                                 2 * ((m_own / 128) * S4 + kt * C::SF_ATOMS));
+#pragma unroll
+          for (int g = 0; g < 2; ++g)
+            pair::tma_load_2d_pair(sSFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512, &tmSFB, bar,
+                                   0, 2 * ((tn * 2 + g) * S4 + kt * C::SF_ATOMS));
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      const uint32_t idesc0 = pair::idesc_pair(FMT != NVFP4);
+      for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs, ++it) {
+        if (!pair::wait_cluster(acc_empty, (it & 1) ^ 1, abort_flag)) break;
+        fence_after_sync();
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag) ||
+              !mbar_wait(&sfready[stage], phase, abort_flag)) { ok = false; break; }
+          fence_after_sync();
+          const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
+          const uint32_t sfa0 = C::SF_BASE + stage * C::SF_COLS;
+          const uint32_t sfb0 = sfa0 + 4 * C::SF_ATOMS;
+#pragma unroll
+          for (int kk = 0; kk < C::K_STEPS; ++kk) {
+            const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, LAYOUT_SW128);
+            const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, LAYOUT_SW128);
+            uint32_t sf_id, sfa_col, sfb_col;
+            if constexpr (FMT == NVFP4) {
+              sf_id = 0;
+              sfa_col = sfa0 + 4 * kk;
+              sfb_col = sfb0 + 8 * kk;
+            } else {
+              sf_id = 2 * (kk & 1);
+              sfa_col = sfa0 + 4 * (kk >> 1);
+              sfb_col = sfb0 + 8 * (kk >> 1);
+            }
+            const uint32_t idesc = idesc0 | (sf_id << 29) | (sf_id << 4);
+            pair::mma_pair<FMT>(tmem, ad, bd, idesc, (kt > 0 || kk > 0) ? 1u : 0u,
+                                (tmem + sfa_col) | (sf_id << 30), (tmem + sfb_col) | (sf_id << 30));
+          }
+          pair::commit_both(&empty[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        pair::commit_both(acc_full);
+      }
+    }
+  } else if (warp >= FIRST_COPIER && warp < FIRST_COPIER + COPIERS) {
+    // ------------------------------------------------------------ scale copiers (leader)
+    if (leader && lane == 0) {
+      const int me = warp - FIRST_COPIER;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          fence_after_sync();
+          const uint32_t sfa_base = smem_u32(sSFA + stage * C::SFA_BYTES);
+          const uint32_t sfb_base = smem_u32(sSFB + stage * C::SFB_BYTES);
+          const uint32_t sfa0 = C::SF_BASE + stage * C::SF_COLS;
+          const uint32_t sfb0 = sfa0 + 4 * C::SF_ATOMS;
+          for (int a = me; a < 3 * C::SF_ATOMS; a += COPIERS) {
+            if (a < C::SF_ATOMS) {
+              pair::tmem_cp_pair(tmem + sfa0 + 4 * a, smem_desc(sfa_base + a * 512, 0, 128, LAYOUT_NONE));
+            } else {
+              const int g = (a - C::SF_ATOMS) / C::SF_ATOMS, j = (a - C::SF_ATOMS) % C::SF_ATOMS;
+              pair::tmem_cp_pair(tmem + sfb0 + 8 * j + 4 * g,
+                                 smem_desc(sfb_base + (g * C::SF_ATOMS + j) * 512, 0, 128,
+                                           LAYOUT_NONE));
+            }
+          }
+          pair::commit_leader(&sfready[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ------------------------------------------------------------ epilogue (both)
+    const int quad = warp & 3;
+    const float sw = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
+    const uint32_t acc_empty_leader = pair::mapa(smem_u32(acc_empty), 0);
+    int it = 0;
+    for (int tile = pair_id; tile < num_tiles; tile += num_pairs, ++it) {
+      const int tm = tile % tiles_m, tn = tile / tiles_m;
+      const int row = tm * 256 + (int)rank * 128 + quad * 32 + lane;
+      const int n0 = tn * BN;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(acc_full, it & 1, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      fence_after_sync();
+      float rs = sw;
+      if (FMT == NVFP4 && s_tok && row < M) rs = __fmul_rn(s_tok[row], sw);
+      // drain the 128 x 256 accumulator slice of this warp into registers,
+      // release it to the leader's MMA warp, then scale, convert and store
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          float f0 = __fmul_rn(__uint_as_float(v[k]), rs);
+          float f1 = __fmul_rn(__uint_as_float(v[k + 1]), rs);
+          if (r_row) {
+            f0 = __fmul_rn(f0, __ldg(r_row + n0 + c0 + k));
+            f1 = __fmul_rn(f1, __ldg(r_row + n0 + c0 + k + 1));
+          }
+          if constexpr (YT == 1) {
+            __nv_bfloat162 p2 = __floats2bfloat162_rn(f0, f1);
+            pk[(c0 + k) / 2] = *reinterpret_cast<uint32_t*>(&p2);
+          } else {
+            v[k] = __float_as_uint(f0);
+            v[k + 1] = __float_as_uint(f1);
+          }
+        }
+        if constexpr (YT != 1) {   // fp32 output: store this 32-column chunk now
+          if (row < M) {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(Y) + (size_t)row * N + n0 + c0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                   __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+          }
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) pair::arrive_remote(acc_empty_leader);
+      if constexpr (YT == 1) {
+        if (row < M) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(Y) + (size_t)row * N + n0);
+#pragma unroll
+          for (int q = 0; q < BN / 8; ++q)
+            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+    }
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  cluster_barrier();   // the leader's last MMAs into this CTA's tensor memory are done
+  if (warp == 1) {
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"((uint32_t)C::TMEM_COLS)
                  : "memory");
   }
@@ -1083,6 +1459,69 @@ static int launch_splitk(const uint8_t* A, const uint8_t* sA, const float* s_tok
   return DQ_OK;
 }
 
+// Paired-SM launch: 2 CTAs per cluster, persistent over 256 x 256 tiles.
+template <int FMT, int YT>
+static int pair_max_clusters() {
+  static int cache[16];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return 0;
+  if (cache[dev]) return cache[dev] > 0 ? cache[dev] : 0;
+  using C = pair::Cfg2<FMT>;
+  auto kern = w4a4_gemm_pair_kernel<FMT, YT>;
+  int n = 0;
+  if (ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void*)kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+  }
+  cache[dev] = n > 0 ? n : -1;
+  return n > 0 ? n : 0;
+}
+
+template <int FMT, int YT>
+static int launch_pair(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
+                       const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
+                       int64_t M, int64_t N, int64_t K, int max_pairs, cudaStream_t st) {
+  using C = pair::Cfg2<FMT>;
+  const int64_t S4 = (K / C::G) / 4;
+  const int64_t sfa_rows = ((M + 127) / 128) * S4 * 2;  // scale atoms as 256-byte rows
+  const int64_t sfb_rows = (N / 128) * S4 * 2;
+  CUtensorMap ta, tb, tsa, tsb;
+  if (!make_map(&ta, A, M, K / 2, BM) || !make_map(&tb, B, N, K / 2, 128) ||
+      !make_map(&tsa, sA, sfa_rows, 256, 2 * C::SF_ATOMS, 256) ||
+      !make_map(&tsb, sB, sfb_rows, 256, 2 * C::SF_ATOMS, 256))
+    return DQ_ERR_CUDA;
+  auto kern = w4a4_gemm_pair_kernel<FMT, YT>;
+  if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
+  const int64_t tiles = ((M + 255) / 256) * (N / pair::BN);
+  const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
+  const cudaError_t e = launch_ex(kern, dim3(2 * pairs), dim3(NUM_THREADS), C::SMEM_BYTES, st, 2,
+                                  ta, tb, tsa, tsb, s_tok, s_w, r_row, Y, (int)M, (int)N, (int)K);
+  return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
+}
+
+// DQ_GEMM_PAIR: 0 never uses the paired-SM kernel, 2 prefers it whenever N
+// is a multiple of 256, anything else (default) lets the tile policy decide.
+static int pair_mode() {
+  static const int mode = [] {
+    const char* e = getenv("DQ_GEMM_PAIR");
+    return (e && e[0] == '0') ? 0 : ((e && e[0] == '2') ? 2 : 1);
+  }();
+  return mode;
+}
+
 // How many clusters of S split-K CTAs the device runs at once (each CTA
 // takes one SM's shared memory; a cluster must fit inside one GPC).
 template <int FMT, int YT>
@@ -1122,8 +1561,21 @@ static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, con
                     const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int64_t M,
                     int64_t N, int64_t K, cudaStream_t st) {
   const int64_t tm = (M + BM - 1) / BM, sms = num_sms();
+  if (N % 256 == 0 && pair_mode() == 2) {
+    const int max_pairs = pair_max_clusters<FMT, YT>();
+    if (max_pairs > 0)
+      return launch_pair<FMT, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, max_pairs, st);
+  }
   if (N % 256 == 0 && tm * (N / 256) >= sms)
     return launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
+  if (N % 256 == 0 && pair_mode() != 0) {
+    // too few 128 x 256 tiles to fill the SMs: paired-SM 256 x 256 tiles
+    // once they occupy at least half of the SM pairs
+    const int max_pairs = pair_max_clusters<FMT, YT>();
+    const int64_t tiles2 = ((M + 255) / 256) * (N / 256);
+    if (max_pairs > 0 && 2 * tiles2 >= max_pairs)
+      return launch_pair<FMT, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, max_pairs, st);
+  }
   const int64_t t128 = tm * (N / 128);
   const int KT = (int)(K / BK);
   // largest split whose clusters (one per output tile) all run in one wave
