@@ -17,12 +17,14 @@
 //                     reduction in fp64 -> per-CTA sums in cluster-visible
 //                     shared memory -> every CTA reads all C partial sums
 //                     over DSMEM in rank order (identical c in every CTA).
-// Each CTA stages its rows of the tile in shared memory once (clusters of up
-// to 16 CTAs keep the share <= 96 KB) and reads them from there in every
-// pass; tiles too tall for that stream their rows through the read-only
+// Each CTA stages its rows of the tile in shared memory once, converted to
+// fp32 (clusters of up to 16 CTAs keep the share <= 96 KB), and reads them
+// from there in every pass; tiles too tall for that stream their rows through the read-only
 // global path (L1 / L2 hits after the first round).  HBM sees W about once.
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "dq_device.cuh"
 #include "dq_internal.h"
@@ -88,11 +90,14 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
 }
+// A double of CTA `rank`'s shared memory.  No memory clobber: the loads of
+// all CTAs are issued back to back before they are summed; the cluster
+// barrier before them orders them after the peers' writes.
 __device__ __forceinline__ double ld_dsmem_f64(const double* local, uint32_t rank) {
   uint32_t a = (uint32_t)__cvta_generic_to_shared(local), ra;
   double v;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
-  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(ra) : "memory");
+  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(ra));
   return v;
 }
 
@@ -265,18 +270,17 @@ __device__ __forceinline__ void grid8_packed(const float2* z, float2* q) {
       q[k].y = rintf(fminf(fmaxf(z[k].y, -8.0f), 7.0f));
     }
   } else {
-    uint32_t codes;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(codes)
-        : "f"(z[0].x), "f"(z[0].y), "f"(z[1].x), "f"(z[1].y), "f"(z[2].x), "f"(z[2].y),
-          "f"(z[3].x), "f"(z[3].y));
+    // nearest E2M1 value of each argument (RNE, saturating): the pair's code
+    // byte goes straight back to an f16x2 of its values (exact), then to fp32
 #pragma unroll
-    for (int k = 0; k < 4; ++k) q[k] = __half22float2(e2m1x2_to_half2((codes >> (8 * k)) & 0xFFu));
+    for (int k = 0; k < 4; ++k) {
+      uint32_t h;
+      asm("{\n\t.reg .b8 t;\n\t"
+          "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+          "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+          : "=r"(h) : "f"(z[k].x), "f"(z[k].y));
+      q[k] = __half22float2(*reinterpret_cast<__half2*>(&h));
+    }
   }
 }
 
@@ -311,8 +315,10 @@ __device__ __forceinline__ void unpack8_global(const WT* __restrict__ p, float2*
   }
 }
 
-template <int F, int G, typename WT, bool WSMEM, bool TRACE>
-__global__ void __launch_bounds__(SolverShape<G>::NT)
+// STG: 0 rows stream through the read-only global path, 1 rows staged in
+// shared memory as WT, 2 rows staged as fp32 (no unpacking in the passes).
+template <int F, int G, typename WT, int STG, bool TRACE>
+__global__ void __launch_bounds__(SolverShape<G>::NT, 2048 / SolverShape<G>::NT / 2)
 solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int T,
                  float* __restrict__ r_out, float* __restrict__ c_io, float* __restrict__ sT_out,
                  SolverWs* ws) {
@@ -323,7 +329,9 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
   float* a_s = r_s + (size_t)steps * S::RPS;
   float* rtab = a_s + (size_t)steps * S::RPS;       // NVFP4: r and alpha of every scale byte
   float* atab = rtab + 128;
-  WT* wch = reinterpret_cast<WT*>(atab + 128);      // staged rows (WSMEM)
+  constexpr bool WSMEM = STG != 0;
+  using ST = typename std::conditional<STG == 2, float, WT>::type;  // staged element type
+  ST* wch = reinterpret_cast<ST*>(atab + 128);      // staged rows
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int oct = lane % S::OPB, rslot = warp * S::RPW + lane / S::OPB;
@@ -346,10 +354,25 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
   if (rank == 0 && b == 0 && tid == 0) *sT_out = sT;
   const float inv_sT = __frcp_rn(sT);
 
-  if constexpr (WSMEM) {
-    // stage rows [row0, row0 + rows_cta) x columns [b*G, b*G+G) (zeros past m)
-    constexpr int V = 16 / sizeof(WT);                // elements per 16-byte piece
-    constexpr int PPR = G / V;                        // pieces per row
+  if constexpr (STG == 2) {
+    // stage rows [row0, row0 + rows_cta) x columns [b*G, b*G+G) (zeros past
+    // m) as fp32, so the passes below read values without unpacking
+    constexpr int PPR = G / 8;                        // 8-element pieces per row
+    for (int p = tid; p < rows_cta * PPR; p += S::NT) {
+      const int lr = p / PPR, pc = p % PPR;
+      const int64_t i = row0 + lr;
+      float2 v[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                     make_float2(0.f, 0.f)};
+      if (i < m) unpack8_global<WT>(W + i * n + b * G + pc * 8, v);
+      float4* dst = reinterpret_cast<float4*>(wch + (size_t)lr * G + pc * 8);
+      dst[0] = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+      dst[1] = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
+    }
+    __syncthreads();
+  } else if constexpr (STG == 1) {
+    // stage the rows in their own type (16-byte pieces, zeros past m)
+    constexpr int V = 16 / sizeof(WT);
+    constexpr int PPR = G / V;
     for (int p = tid; p < rows_cta * PPR; p += S::NT) {
       const int lr = p / PPR, pc = p % PPR;
       const int64_t i = row0 + lr;
@@ -359,10 +382,22 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
     }
     __syncthreads();
   }
+  // this thread's row-steps s cover rows row0 + s*RPS + rslot; those below m
+  // are s < s_end.  Per-thread bases and constant strides for the hot loops.
+  const int64_t first_row = row0 + rslot;
+  const int s_end = first_row >= m ? 0
+                    : (int)((m - first_row + S::RPS - 1) / S::RPS) < steps
+                          ? (int)((m - first_row + S::RPS - 1) / S::RPS)
+                          : steps;
+  const ST* xsm = WSMEM ? wch + (size_t)rslot * G + oct * 8 : nullptr;
+  const WT* xgl = WSMEM ? nullptr : W + first_row * n + col0;
+  constexpr int XSM_STEP = S::RPS * G;
+  const int64_t xgl_step = (int64_t)S::RPS * n;
+  float* rsl = r_s + rslot;
+  float* asl = a_s + rslot;
   auto load_x = [&](int s, float2* x) {
-    const int lr = s * S::RPS + rslot;
-    if constexpr (WSMEM) unpack8<WT>(wch + (size_t)lr * G + oct * 8, x);
-    else unpack8_global<WT>(W + (row0 + lr) * n + col0, x);
+    if constexpr (WSMEM) unpack8<ST>(xsm + s * XSM_STEP, x);
+    else unpack8_global<WT>(xgl + s * xgl_step, x);
   };
 
   float2 cc[4], beta[4];
@@ -375,9 +410,8 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
   // r0: format-native absmax scale of W diag(c0)^-1 per row-block (IEEE
   // arithmetic: the same fp32 decisions as the oracle's initialisation)
   for (int s = 0; s < steps; ++s) {
-    const int64_t i = row0 + (int64_t)s * S::RPS + rslot;
     float a = 0.0f;
-    if (i < m) {
+    if (s < s_end) {
       float2 x[4];
       load_x(s, x);
 #pragma unroll
@@ -390,8 +424,8 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
     for (int o = 1; o < S::OPB; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     if (oct == 0) {
       float r0 = rtn_block_scale<F>(a, sT);
-      r_s[s * S::RPS + rslot] = r0;
-      a_s[s * S::RPS + rslot] = __frcp_rn(r0);
+      rsl[s * S::RPS] = r0;
+      asl[s * S::RPS] = __frcp_rn(r0);
     }
   }
   __syncwarp();
@@ -401,11 +435,10 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
     float e_acc = 0.0f;
     if (t < T || TRACE) {
       for (int s = 0; s < steps; ++s) {
-        const int lr = s * S::RPS + rslot;
-        const int64_t i = row0 + (int64_t)s * S::RPS + rslot;
+        const bool valid = s < s_end;
         float2 num2 = make_float2(0.f, 0.f), den2 = num2, err2 = num2;
-        const float rr = r_s[lr], alpha = a_s[lr];
-        if (i < m) {
+        const float rr = rsl[s * S::RPS], alpha = asl[s * S::RPS];
+        if (valid) {
           float2 x[4], z[4], q[4];
           load_x(s, x);
           const float2 a2 = make_float2(alpha, alpha);
@@ -431,12 +464,12 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
           if constexpr (TRACE) err += __shfl_xor_sync(0xffffffffu, err, o);
         }
         if (TRACE && oct == 0) e_acc += err;
-        if (t < T && oct == 0 && i < m) {
+        if (t < T && oct == 0 && valid) {
           float rn, an;
           if (den > 0.0f) RowProj<F>::apply(__fdividef(num, den), inv_sT, rtab, atab, sT, rn, an);
           else RowProj<F>::apply(1.0f, inv_sT, rtab, atab, sT, rn, an);
-          r_s[lr] = rn;
-          a_s[lr] = an;
+          rsl[s * S::RPS] = rn;
+          asl[s * S::RPS] = an;
         }
       }
     }
@@ -452,11 +485,9 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
     float2 acc[8];
 #pragma unroll
     for (int v = 0; v < 8; ++v) acc[v] = make_float2(0.f, 0.f);
-    for (int s = 0; s < steps; ++s) {
-      const int lr = s * S::RPS + rslot;
-      const int64_t i = row0 + (int64_t)s * S::RPS + rslot;
-      if (i < m) {
-        const float rr = r_s[lr], alpha = a_s[lr];
+    for (int s = 0; s < s_end; ++s) {
+      {
+        const float rr = rsl[s * S::RPS], alpha = asl[s * S::RPS];
         float2 x[4], z[4], q[4];
         load_x(s, x);
         const float2 a2 = make_float2(alpha, alpha), r2 = make_float2(rr, rr);
@@ -485,10 +516,21 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
     cluster_sync_all();
     if (tid < G) {
       const int j = tid, o = j >> 3, k = j & 7;
-      double sn = 0.0, sd = 0.0;
-      for (uint32_t q = 0; q < C; ++q) {
-        sn += ld_dsmem_f64(&sm.cpart[par][o * 16 + 2 * k], q);
-        sd += ld_dsmem_f64(&sm.cpart[par][o * 16 + 2 * k + 1], q);
+      double sn = 0.0, sd = 0.0;   // rank order; four CTAs' partials in flight at a time
+      for (int q0 = 0; q0 < (int)C; q0 += 4) {
+        double pn[4], pd[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (q0 + u < (int)C) {
+            pn[u] = ld_dsmem_f64(&sm.cpart[par][o * 16 + 2 * k], (uint32_t)(q0 + u));
+            pd[u] = ld_dsmem_f64(&sm.cpart[par][o * 16 + 2 * k + 1], (uint32_t)(q0 + u));
+          }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (q0 + u < (int)C) {
+            sn += pn[u];
+            sd += pd[u];
+          }
       }
       float cn = (sd > 0.0) ? proj_beta<F>((float)(sn / sd)) : proj_beta<F>(1.0f);
       sm.c_s[j] = cn;
@@ -503,10 +545,8 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
   }
 
   // outputs
-  for (int s = 0; s < steps; ++s) {
-    const int64_t i = row0 + (int64_t)s * S::RPS + rslot;
-    if (oct == 0 && i < m) r_out[i * nb + b] = r_s[s * S::RPS + rslot];
-  }
+  for (int s = 0; s < s_end; ++s)
+    if (oct == 0) r_out[(first_row + (int64_t)s * S::RPS) * nb + b] = rsl[s * S::RPS];
   if (rank == 0 && tid < G && T > 0) c_io[b * G + tid] = sm.c_s[tid];
   cluster_sync_all();  // no CTA leaves while a peer may still read its cpart
 }
@@ -519,34 +559,37 @@ __global__ void solve_finalize_kernel(const SolverWs* ws, int T, double* mse_tra
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int G, typename WT>
-static size_t solver_smem_bytes(int steps, bool wsmem) {
+template <int G>
+static size_t solver_smem_bytes(int steps, size_t staged_elem_bytes) {
   const size_t rows = (size_t)steps * SolverShape<G>::RPS;
   return sizeof(SolverSmem<G>) + 2 * sizeof(float) * rows + 2 * 128 * sizeof(float) +
-         (wsmem ? rows * G * sizeof(WT) : 0);
+         rows * G * staged_elem_bytes;
 }
 
 // Launch geometry: the tile's rows are split over C CTAs of one cluster,
 // `steps` row-steps of RPS rows per CTA.  Prefer staging the CTA's rows in
-// shared memory (<= 96 KB of rows, clusters of up to 16 CTAs); otherwise
-// stream them through the read-only global path with clusters of 8.
+// shared memory as fp32, then in the weight's own type (<= 96 KB of rows,
+// clusters of up to 16 CTAs); otherwise stream them through the read-only
+// global path with clusters of 8.  stg: 2 fp32, 1 own type, 0 global.
 template <int G, typename WT>
-static void solver_geometry(int64_t m, int& steps, int& C, bool& wsmem) {
+static void solver_geometry(int64_t m, int& steps, int& C, int& stg) {
   using S = SolverShape<G>;
-  const size_t row_bytes = (size_t)G * sizeof(WT);
-  for (int cmax : {8, 16}) {
-    int st = (int)((m + (int64_t)S::RPS * cmax - 1) / ((int64_t)S::RPS * cmax));
-    if (st < 1) st = 1;
-    if ((size_t)st * S::RPS * row_bytes <= 96 * 1024) {
-      steps = st;
-      C = (int)((m + (int64_t)S::RPS * st - 1) / ((int64_t)S::RPS * st));
-      wsmem = true;
-      return;
+  for (int s_try : {2, 1}) {
+    const size_t row_bytes = (size_t)G * (s_try == 2 ? sizeof(float) : sizeof(WT));
+    for (int cmax : {8, 16}) {
+      int st = (int)((m + (int64_t)S::RPS * cmax - 1) / ((int64_t)S::RPS * cmax));
+      if (st < 1) st = 1;
+      if ((size_t)st * S::RPS * row_bytes <= 96 * 1024) {
+        steps = st;
+        C = (int)((m + (int64_t)S::RPS * st - 1) / ((int64_t)S::RPS * st));
+        stg = s_try;
+        return;
+      }
     }
   }
   steps = (int)((m + (int64_t)S::RPS * 8 - 1) / ((int64_t)S::RPS * 8));
   C = (int)((m + (int64_t)S::RPS * steps - 1) / ((int64_t)S::RPS * steps));
-  wsmem = false;
+  stg = 0;
 }
 
 template <typename K>
@@ -559,10 +602,11 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, float* r, 
                          float* sT, double* trace, SolverWs* ws, cudaStream_t st) {
   using S = SolverShape<G>;
   const WT* W = reinterpret_cast<const WT*>(Wv);
-  int steps, C;
-  bool wsmem;
-  solver_geometry<G, WT>(m, steps, C, wsmem);
-  const size_t sm_init = sizeof(SolverSmem<G>), sm_main = solver_smem_bytes<G, WT>(steps, wsmem);
+  int steps, C, stg;
+  solver_geometry<G, WT>(m, steps, C, stg);
+  const size_t sm_init = sizeof(SolverSmem<G>),
+               sm_main = solver_smem_bytes<G>(
+                   steps, stg == 2 ? sizeof(float) : (stg == 1 ? sizeof(WT) : 0));
   if (sm_main > 227 * 1024) return DQ_ERR_UNSUPPORTED;
 
   cudaLaunchAttribute attr[1];
@@ -590,10 +634,12 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, float* r, 
     if (!allow_big_cluster(km, sm_main)) return DQ_ERR_CUDA;                               \
     e = cudaLaunchKernelEx(&cfg, km, W, m, n, steps, T, r, c, sT, ws);                      \
   }
-  if (wsmem) {
-    if (trace) DQ_MAIN(true, true) else DQ_MAIN(true, false)
+  if (stg == 2) {
+    if (trace) DQ_MAIN(2, true) else DQ_MAIN(2, false)
+  } else if (stg == 1) {
+    if (trace) DQ_MAIN(1, true) else DQ_MAIN(1, false)
   } else {
-    if (trace) DQ_MAIN(false, true) else DQ_MAIN(false, false)
+    if (trace) DQ_MAIN(0, true) else DQ_MAIN(0, false)
   }
 #undef DQ_MAIN
   if (e != cudaSuccess) return DQ_ERR_CUDA;
