@@ -729,8 +729,10 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
       };
       int rc = -1;
       if constexpr (F == NVFP4) {
-        if (S <= 512) rc = ring(quantize_act_ring_kernel<F, G, 1, 512, 2>, 1, 512, 2);
-        else if (S <= 1024) rc = ring(quantize_act_ring_kernel<F, G, 2, 512, 1>, 2, 512, 1);
+        // two blocks per thread halve the per-row overhead per element once
+        // a row has enough blocks to keep 128+ threads busy
+        if (S >= 256 && S <= 1024) rc = ring(quantize_act_ring_kernel<F, G, 2, 512, 1>, 2, 512, 1);
+        else if (S <= 512) rc = ring(quantize_act_ring_kernel<F, G, 1, 512, 2>, 1, 512, 2);
       } else {
         if (S <= 384) rc = ring(quantize_act_ring_kernel<F, G, 1, 384, 2>, 1, 384, 2);
         else if (S <= 512) rc = ring(quantize_act_ring_kernel<F, G, 1, 512, 1>, 1, 512, 1);
