@@ -419,6 +419,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int tm = tile % tiles_m, tn = tile / tiles_m;
       const int row = tm * BM + quad * 32 + lane;
       const int n0 = tn * BN;
+      // this row's scale is loaded before the accumulator wait, off the
+      // critical path of the hand-off back to the MMA warp
+      float rs = sw;
+      if (FMT == NVFP4 && s_tok && row < M) rs = __fmul_rn(s_tok[row], sw);
       // one lane waits, the warp follows (the tensor-memory loads below are
       // warp-collective and must never run in a partial warp)
       int ok = 1;
@@ -426,8 +430,6 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       fence_after_sync();
-      float rs = sw;
-      if (FMT == NVFP4 && s_tok && row < M) rs = __fmul_rn(s_tok[row], sw);
       if constexpr (YT == 1) {
         if (r_row)
           epilogue_bf16<BN, true>(tmem, quad, lane, row, M, N, n0, rs, r_row, Y, acc_empty);
@@ -512,7 +514,8 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const uint8_t* __restrict__ sfA,
                         const uint8_t* __restrict__ sfB, const float* __restrict__ s_tok,
                         const float* __restrict__ s_w, const float* __restrict__ r_row,
-                        void* __restrict__ Y, int M, int N, int K, int kt_per_slice) {
+                        void* __restrict__ Y, int M, int N, int K, int kt_per_slice,
+                        int a_rows) {
   constexpr int BN = SK_BN;
   using C = Cfg<FMT, BN, SK_PART_BYTES>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -529,6 +532,8 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
   uint64_t* acc_full = sfready + C::STAGES;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+  __shared__ float s_rs[BM];       // per-row output scale
+  __shared__ float s_rr[SK_BN];    // per-output-column factor of this tile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -570,7 +575,9 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
       uint32_t phase = 0;
       for (int kt = 0; kt < kt_per_slice; ++kt) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
-        mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+        // A tiles carry only the a_rows rows that exist (rounded up to 16):
+        // the MMA's other rows feed accumulator rows that are never stored
+        mbar_expect_tx(&full[stage], C::STAGE_BYTES - (BM - a_rows) * BKB);
         tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], (kt0 + kt) * BKB, m0);
         tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], (kt0 + kt) * BKB, n0);
         bulk_load(sSFA + stage * C::SFA_BYTES,
@@ -623,8 +630,11 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
       }
       if (ok) mma_commit(acc_full);
     }
-  } else if (warp >= FIRST_COPIER && warp < FIRST_COPIER + COPIERS) {
-    if (lane == 0) {
+  } else {
+    // warps 2..5 and the copier warps 6..9 drain the partial tile after the
+    // mainloop, each pair of warps one TMEM lane quadrant, half the columns each
+    const bool copier = warp >= FIRST_COPIER;
+    if (copier && lane == 0) {
       const int me = warp - FIRST_COPIER;
       int stage = 0;
       uint32_t phase = 0;
@@ -646,12 +656,22 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
-  } else if (warp >= 2 && warp <= 5) {
+    __syncwarp();
+    const int quad = warp & 3;
+    if (!copier) {
+      // per-row scale and the tile's output-row factors, staged before the
+      // accumulator wait so the reduction below reads shared memory only
+      const int rr = quad * 32 + lane;
+      float rs = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
+      if (FMT == NVFP4 && s_tok && m0 + rr < M) rs = __fmul_rn(s_tok[m0 + rr], rs);
+      s_rs[rr] = rs;
+      s_rr[rr] = r_row ? __ldg(r_row + n0 + rr) : 1.0f;
+    }
     // drain this CTA's partial tile (rows that exist) straight into the
     // shared memory of the CTA that reduces each column slice: owner q keeps
     // slice [q * cols, (q + 1) * cols) of every rank, at part[rank][row][.]
-    const int quad = warp & 3;
     const int cols = BN / (int)S;
+    const int c_lo = copier ? BN / 2 : 0;
     int ok = 1;
     if (lane == 0) ok = mbar_wait(acc_full, 0, abort_flag) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -660,14 +680,14 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
       const int row = quad * 32 + lane;
       const uint32_t mine = smem_u32(part + ((size_t)rank * BM + row) * cols);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c0, v);
 #pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-          const int c = c0 + k, q = c / cols;
-          st_dsmem_f32x4(mine + (uint32_t)(c - q * cols) * 4, (uint32_t)q, v[k], v[k + 1], v[k + 2],
-                         v[k + 3]);
+        for (int kk = 0; kk < 32; kk += 4) {
+          const int c = c0 + kk, q = c / cols;
+          st_dsmem_f32x4(mine + (uint32_t)(c - q * cols) * 4, (uint32_t)q, v[kk], v[kk + 1],
+                         v[kk + 2], v[kk + 3]);
         }
       }
     }
@@ -681,7 +701,6 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
     const int cols = BN / (int)S, c4 = cols / 4, c_begin = (int)rank * cols;
     const int rows = (M - m0) < BM ? (M - m0) : BM;
     const int total = rows * c4;
-    const float sw = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
     for (int idx = threadIdx.x; idx < total; idx += NUM_THREADS) {
       const int r = idx / c4, cc = (idx % c4) * 4, c = c_begin + cc;
       float4 acc = *reinterpret_cast<const float4*>(part + (size_t)r * cols + cc);
@@ -689,13 +708,12 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
         const float4 p = *reinterpret_cast<const float4*>(part + ((size_t)q * BM + r) * cols + cc);
         acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
       }
-      float rs = sw;
-      if (FMT == NVFP4 && s_tok) rs = __fmul_rn(s_tok[m0 + r], sw);
+      const float rs = s_rs[r];
       float f[4] = {__fmul_rn(acc.x, rs), __fmul_rn(acc.y, rs), __fmul_rn(acc.z, rs),
                     __fmul_rn(acc.w, rs)};
       if (r_row) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) f[k] = __fmul_rn(f[k], __ldg(r_row + n0 + c + k));
+        for (int q = 0; q < 4; ++q) f[q] = __fmul_rn(f[q], s_rr[c + q]);
       }
       const size_t o = (size_t)(m0 + r) * N + n0 + c;
       if constexpr (YT == 1) {
@@ -1015,13 +1033,13 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       const int tm = tile % tiles_m, tn = tile / tiles_m;
       const int row = tm * 256 + (int)rank * 128 + quad * 32 + lane;
       const int n0 = tn * BN;
+      float rs = sw;   // loaded before the accumulator wait
+      if (FMT == NVFP4 && s_tok && row < M) rs = __fmul_rn(s_tok[row], sw);
       int ok = 1;
       if (lane == 0) ok = mbar_wait(acc_full, it & 1, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       fence_after_sync();
-      float rs = sw;
-      if (FMT == NVFP4 && s_tok && row < M) rs = __fmul_rn(s_tok[row], sw);
       // drain the 128 x 256 accumulator slice of this warp into registers,
       // release it to the leader's MMA warp, then scale, convert and store
       uint32_t pk[BN / 2];
@@ -1447,14 +1465,15 @@ static int launch_splitk(const uint8_t* A, const uint8_t* sA, const float* s_tok
                          const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                          int64_t M, int64_t N, int64_t K, int S, cudaStream_t st) {
   using C = Cfg<FMT, SK_BN, SK_PART_BYTES>;
+  const int a_rows = M < BM ? (int)((M + 15) / 16 * 16) : BM;
   CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K / 2, BM) || !make_map(&tb, B, N, K / 2, SK_BN)) return DQ_ERR_CUDA;
+  if (!make_map(&ta, A, M, K / 2, a_rows) || !make_map(&tb, B, N, K / 2, SK_BN)) return DQ_ERR_CUDA;
   auto kern = w4a4_gemm_splitk_kernel<FMT, YT>;
   if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
   const int kt_per_slice = (int)(K / BK) / S;
   if (launch_ex(kern, dim3(S, (unsigned)(N / SK_BN), (unsigned)((M + BM - 1) / BM)),
                 dim3(NUM_THREADS), C::SMEM_BYTES, st, (unsigned)S, ta, tb, sA, sB, s_tok, s_w,
-                r_row, Y, (int)M, (int)N, (int)K, kt_per_slice) != cudaSuccess)
+                r_row, Y, (int)M, (int)N, (int)K, kt_per_slice, a_rows) != cudaSuccess)
     return DQ_ERR_CUDA;
   return DQ_OK;
 }
