@@ -183,6 +183,12 @@ DQ_API int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, con
  * block-scaled tensor-core form on sm_100a).
  * Sizes: M >= 1, N % 128 == 0, K % 256 == 0; A, B, sA, sB 16-byte aligned.
  * FP32 accumulation in tensor memory.
+ * Ordering: stream-ordered.  The inference kernels use programmatic
+ * dependent launch and read the weight operand (B, sB) before waiting for
+ * the kernel launched just before them in the stream; B and sB must
+ * therefore not be written by such a kernel when it triggers its
+ * dependents early (dq_quantize_weight's packer, memory copies and ordinary
+ * kernels do not).  A, sA, s_tok and Y are accessed only after that wait.
  * ---------------------------------------------------------------------- */
 DQ_API int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                    const uint8_t* sB, const float* s_w, const float* r_row, void* Y,

@@ -297,31 +297,48 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_base_slot;
-  pdl_wait();     // operands and output may belong to the previous kernel of the stream
+  // Programmatic dependent launch: the weight operand (B and its scales) is
+  // never written by the kernel launched just before a GEMM (the activation
+  // quantiser), so the producer fetches the first stages' weights before the
+  // dependency wait; the activations, the per-token scales and the output
+  // are touched only after it (producer and epilogue roles).
   pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      auto load_b = [&](int stage, int n0, int kt) {
+        tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kt * BKB, n0);
+#pragma unroll
+        for (int g = 0; g < BN / 128; ++g)
+          bulk_load(sSFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512,
+                    sfB + ((size_t)(n0 / 128 + g) * S4 + (size_t)kt * C::SF_ATOMS) * 512,
+                    C::SF_ATOMS * 512, &full[stage]);
+      };
+      // weights of the first stages ahead of the dependency wait
+      const int pre = (blockIdx.x < num_tiles) ? (KT < C::STAGES ? KT : C::STAGES) : 0;
+      for (int kt = 0; kt < pre; ++kt) {
+        mbar_expect_tx(&full[kt], C::STAGE_BYTES);
+        load_b(kt, (blockIdx.x / tiles_m) * BN, kt);
+      }
+      pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      bool first = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, first = false) {
         const int tm = tile % tiles_m, tn = tile / tiles_m;
         const int m0 = tm * BM, n0 = tn * BN;
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+          if (!(first && kt < pre)) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+            mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+            load_b(stage, n0, kt);
+          }
           tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kt * BKB, m0);
-          tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kt * BKB, n0);
           bulk_load(sSFA + stage * C::SFA_BYTES,
                     sfA + ((size_t)(m0 / 128) * S4 + (size_t)kt * C::SF_ATOMS) * 512,
                     C::SFA_BYTES, &full[stage]);
-#pragma unroll
-          for (int g = 0; g < BN / 128; ++g)
-            bulk_load(sSFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512,
-                      sfB + ((size_t)(n0 / 128 + g) * S4 + (size_t)kt * C::SF_ATOMS) * 512,
-                      C::SF_ATOMS * 512, &full[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -413,6 +430,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;                 // tensor-memory lane quadrant of this warp
+    pdl_wait();
     const float sw = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
@@ -566,26 +584,37 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_base_slot;
-  pdl_wait();     // operands and output may belong to the previous kernel of the stream
-  pdl_trigger();
+  pdl_trigger();   // weights are fetched before the dependency wait (see the 1-CTA kernel)
 
   if (warp == 0) {
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int kt = 0; kt < kt_per_slice; ++kt) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
-        // A tiles carry only the a_rows rows that exist (rounded up to 16):
-        // the MMA's other rows feed accumulator rows that are never stored
-        mbar_expect_tx(&full[stage], C::STAGE_BYTES - (BM - a_rows) * BKB);
-        tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], (kt0 + kt) * BKB, m0);
+      // A tiles carry only the a_rows rows that exist (rounded up to 16): the
+      // MMA's other rows feed accumulator rows that are never stored
+      const uint32_t tx = C::STAGE_BYTES - (BM - a_rows) * BKB;
+      auto load_b = [&](int stage, int kt) {
         tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], (kt0 + kt) * BKB, n0);
-        bulk_load(sSFA + stage * C::SFA_BYTES,
-                  sfA + ((size_t)(m0 / 128) * S4 + (size_t)(kt0 + kt) * C::SF_ATOMS) * 512,
-                  C::SFA_BYTES, &full[stage]);
         bulk_load(sSFB + stage * C::SFB_BYTES,
                   sfB + ((size_t)(n0 / 128) * S4 + (size_t)(kt0 + kt) * C::SF_ATOMS) * 512,
                   C::SFB_BYTES, &full[stage]);
+      };
+      const int pre = kt_per_slice < C::STAGES ? kt_per_slice : C::STAGES;
+      for (int kt = 0; kt < pre; ++kt) {   // weights ahead of the dependency wait
+        mbar_expect_tx(&full[kt], tx);
+        load_b(kt, kt);
+      }
+      pdl_wait();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = 0; kt < kt_per_slice; ++kt) {
+        if (kt >= pre) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+          mbar_expect_tx(&full[stage], tx);
+          load_b(stage, kt);
+        }
+        tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], (kt0 + kt) * BKB, m0);
+        bulk_load(sSFA + stage * C::SFA_BYTES,
+                  sfA + ((size_t)(m0 / 128) * S4 + (size_t)(kt0 + kt) * C::SF_ATOMS) * 512,
+                  C::SFA_BYTES, &full[stage]);
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
       for (int s = 0; s < C::STAGES; ++s) {  // drain: every issued stage lands before exit
@@ -661,6 +690,9 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
     if (!copier) {
       // per-row scale and the tile's output-row factors, staged before the
       // accumulator wait so the reduction below reads shared memory only
+      // (these warps pass the dependency wait before the output is written
+      // by anyone: every thread writes it only after the cluster barrier)
+      pdl_wait();
       const int rr = quad * 32 + lane;
       float rs = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
       if (FMT == NVFP4 && s_tok && m0 + rr < M) rs = __fmul_rn(s_tok[m0 + rr], rs);
@@ -920,31 +952,44 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   cluster_barrier();   // both CTAs' barriers are initialised before any remote use
   fence_after_sync();
   const uint32_t tmem = *tmem_base_slot;
-  pdl_wait();     // operands and output may belong to the previous kernel of the stream
-  pdl_trigger();
+  pdl_trigger();   // weights are fetched before the dependency wait (see the 1-CTA kernel)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      auto load_b = [&](int stage, int tn, int kt) {
+        const uint32_t bar = pair::mapa(smem_u32(&full[stage]), 0);
+        pair::tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kt * BKB, tn * BN + (int)rank * 128);
+#pragma unroll
+        for (int g = 0; g < 2; ++g)
+          pair::tma_load_2d_pair(sSFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512, &tmSFB, bar,
+                                 0, 2 * ((tn * 2 + g) * S4 + kt * C::SF_ATOMS));
+      };
+      // weights of the first stages ahead of the dependency wait
+      const int pre = (pair_id < num_tiles) ? (KT < C::STAGES ? KT : C::STAGES) : 0;
+      for (int kt = 0; kt < pre; ++kt) {
+        if (leader) mbar_expect_tx(&full[kt], TX);
+        load_b(kt, pair_id / tiles_m, kt);
+      }
+      pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
+      bool first = true;
+      for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs, first = false) {
         const int tm = tile % tiles_m, tn = tile / tiles_m;
-        const int m_own = tm * 256 + (int)rank * 128, n_own = tn * BN + (int)rank * 128;
+        const int m_own = tm * 256 + (int)rank * 128;
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
           const uint32_t bar = pair::mapa(smem_u32(&full[stage]), 0);
-          if (leader) mbar_expect_tx(&full[stage], TX);
+          if (!(first && kt < pre)) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+            if (leader) mbar_expect_tx(&full[stage], TX);
+            load_b(stage, tn, kt);
+          }
           pair::tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kt * BKB, m_own);
-          pair::tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kt * BKB, n_own);
           // scale atoms as rows of 256 bytes: atom a of row block rb is rows 2a, 2a + 1
           pair::tma_load_2d_pair(sSFA + stage * C::SFA_BYTES, &tmSFA, bar, 0,
                                  2 * ((m_own / 128) * S4 + kt * C::SF_ATOMS));
-#pragma unroll
-          for (int g = 0; g < 2; ++g)
-            pair::tma_load_2d_pair(sSFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512, &tmSFB, bar,
-                                   0, 2 * ((tn * 2 + g) * S4 + kt * C::SF_ATOMS));
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -1026,6 +1071,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue (both)
     const int quad = warp & 3;
+    pdl_wait();
     const float sw = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
     const uint32_t acc_empty_leader = pair::mapa(smem_u32(acc_empty), 0);
     int it = 0;
