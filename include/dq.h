@@ -157,6 +157,10 @@ DQ_API int dq_quantize_weight(const void* W, dq_dtype wt, int64_t m, int64_t n, 
  * block scale = bf16(amax_blk / 7).  Codes: grid(x~ * fl(1/scale)), round
  * to nearest even, saturating; an all-zero block gives zero codes.
  * Bit-exact with the oracle.
+ * Ordering: stream-ordered; launched with programmatic dependent launch,
+ * the kernel reads c before waiting for the kernel launched just before it,
+ * so c must not be written by such a kernel when it triggers its
+ * dependents early (the solver, memory copies and ordinary kernels do not).
  * ---------------------------------------------------------------------- */
 DQ_API int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, const float* c,
                     dq_format f, int group, uint8_t* codes, void* scales, float* s_tok,

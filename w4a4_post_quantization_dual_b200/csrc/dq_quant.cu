@@ -184,7 +184,6 @@ quantize_act_rows_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int6
                          uint8_t* __restrict__ scales, float* __restrict__ s_tok) {
   constexpr int PIECES = G * (int)sizeof(XT) / 16;   // 16-byte loads per block
   __shared__ float red[2][R][16];
-  pdl_wait();
   pdl_trigger();
   const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int NWARP = (NT + 31) >> 5;
@@ -200,6 +199,7 @@ quantize_act_rows_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int6
       cv[j][k] = v.x; cv[j][k + 1] = v.y; cv[j][k + 2] = v.z; cv[j][k + 3] = v.w;
     }
   }
+  pdl_wait();   // c was read ahead of the dependency wait, X and the outputs after it
   // element k of a block held as raw 16-byte pieces
   auto elem = [&](const uint4 (&raw)[PIECES], int k) -> float {
     if constexpr (sizeof(XT) == 2) {
@@ -505,9 +505,11 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  pdl_wait();     // inputs and outputs may belong to the previous kernel of the stream
   pdl_trigger();
-  float2 cv[BPT][H];  // column scales of the owned blocks, in the rotated piece order
+  // column scales of the owned blocks, in the rotated piece order: c comes
+  // from the solver, never from the kernel launched just before this one, so
+  // it is read ahead of the dependency wait (X and the outputs after it)
+  float2 cv[BPT][H];
 #pragma unroll
   for (int j = 0; j < BPT; ++j) {
     const int s = tl + j * NTS;
@@ -524,6 +526,7 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
       }
     }
   }
+  pdl_wait();
   __syncthreads();
 
   const int64_t step = (int64_t)gridDim.x * RT;  // rows between consecutive groups of a CTA
