@@ -194,7 +194,7 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = (227 * 1024 - 1024 - 256 - RESERVE) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + RESERVE;
-  static_assert(3 * STAGES * 8 + 32 <= 256, "barrier area");
+  static_assert(4 * STAGES * 8 + 32 <= 256, "barrier area");
   // tensor-memory columns: accumulator, then one scale slot per stage
   // (SFA: 4 columns per atom; SFB: 4 columns per atom and 128-row group)
   static constexpr int SF_COLS = 4 * SF_ATOMS * (1 + BN / 128);
@@ -260,7 +260,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + C::STAGES * C::SFB_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* sfready = empty + C::STAGES;
-  uint64_t* acc_full = sfready + C::STAGES;
+  uint64_t* sffull = sfready + C::STAGES;   // scale atoms of the stage landed
+  uint64_t* acc_full = sffull + C::STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
@@ -280,6 +281,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sfready[s], COPIERS);
+      mbar_init(&sffull[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
@@ -307,18 +309,23 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // the scale atoms of a stage complete on sffull (issued first, so the
+      // copier warps move them into tensor memory while the A / B tiles are
+      // still landing), the code tiles on full
+      constexpr uint32_t TX_AB = C::A_BYTES + C::B_BYTES, TX_SF = C::SFA_BYTES + C::SFB_BYTES;
       auto load_b = [&](int stage, int n0, int kt) {
-        tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kt * BKB, n0);
 #pragma unroll
         for (int g = 0; g < BN / 128; ++g)
           bulk_load(sSFB + stage * C::SFB_BYTES + g * C::SF_ATOMS * 512,
                     sfB + ((size_t)(n0 / 128 + g) * S4 + (size_t)kt * C::SF_ATOMS) * 512,
-                    C::SF_ATOMS * 512, &full[stage]);
+                    C::SF_ATOMS * 512, &sffull[stage]);
+        tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kt * BKB, n0);
       };
       // weights of the first stages ahead of the dependency wait
       const int pre = (blockIdx.x < num_tiles) ? (KT < C::STAGES ? KT : C::STAGES) : 0;
       for (int kt = 0; kt < pre; ++kt) {
-        mbar_expect_tx(&full[kt], C::STAGE_BYTES);
+        mbar_expect_tx(&sffull[kt], TX_SF);
+        mbar_expect_tx(&full[kt], TX_AB);
         load_b(kt, (blockIdx.x / tiles_m) * BN, kt);
       }
       pdl_wait();
@@ -332,13 +339,14 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         for (int kt = 0; kt < KT; ++kt) {
           if (!(first && kt < pre)) {
             if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-            mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+            mbar_expect_tx(&sffull[stage], TX_SF);
+            mbar_expect_tx(&full[stage], TX_AB);
             load_b(stage, n0, kt);
           }
-          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kt * BKB, m0);
           bulk_load(sSFA + stage * C::SFA_BYTES,
                     sfA + ((size_t)(m0 / 128) * S4 + (size_t)kt * C::SF_ATOMS) * 512,
-                    C::SFA_BYTES, &full[stage]);
+                    C::SFA_BYTES, &sffull[stage]);
+          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kt * BKB, m0);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -406,7 +414,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&sffull[stage], phase, abort_flag)) { ok = false; break; }
           fence_after_sync();
           const uint32_t sfa_base = smem_u32(sSFA + stage * C::SFA_BYTES);
           const uint32_t sfb_base = smem_u32(sSFB + stage * C::SFB_BYTES);
