@@ -61,6 +61,9 @@ def lib():
                                      ctypes.c_float, _f32p]),
             "oracle_solve": (None, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     _i64p, _i64, _f32p, _f32p, _f32p, _f64p, _f64p]),
+            "oracle_solve_ex": (None, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, _f32p, _f32p, _i64p, _i64,
+                                       _f32p, _f32p, _f32p, _f64p, _f64p]),
             "oracle_error": (ctypes.c_double, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int,
                                                _f32p, _f32p]),
             "oracle_error_fixed_q": (ctypes.c_double, [_f32p, _u8p, _i64, _i64, ctypes.c_int,
@@ -200,6 +203,39 @@ def solve(W, fmt, G, T, tiles=None):
         tp, nt = _p(tarr, _i64p), len(tarr)
     lib().oracle_solve(_p(W, _f32p), m, n, fmt, G, T, tp, nt, _p(r, _f32p), _p(c, _f32p),
                        _p(sT, _f32p), _p(err, _f64p), _p(w2, _f64p))
+    trace = err / w2[0] if w2[0] > 0 else err
+    return {"r": r, "c": c, "s_T": float(sT[0]), "trace": trace, "err": err, "w2": float(w2[0])}
+
+
+ALPHA_ONLY, BETA_ONLY, KEEP_S = 1, 2, 4
+
+
+def solve_ex(W, fmt, G, T, flags=0, r0=None, c0=None, s_T=None, tiles=None):
+    """Algorithm 1 with an ablation mode (ALPHA_ONLY / BETA_ONLY, Table 4)
+    and optional initial scales r0 (m, n/G) / c0 (n,), projected onto the
+    admissible sets; with KEEP_S the NVFP4 tensor scale s_T is given rather
+    than computed.  Same return value as solve()."""
+    W = _f32(W)
+    m, n = W.shape
+    nb = n // G
+    r = np.empty((m, nb), np.float32)
+    c = np.empty(n, np.float32)
+    sT = np.array([s_T if s_T is not None else 0.0], np.float32)
+    if (flags & KEEP_S) and s_T is None:
+        raise ValueError("KEEP_S needs s_T")
+    err = np.zeros(T + 1, np.float64)
+    w2 = np.zeros(1, np.float64)
+    if tiles is None:
+        tp, nt = None, 0
+    else:
+        tarr = np.ascontiguousarray(tiles, dtype=np.int64)
+        tp, nt = _p(tarr, _i64p), len(tarr)
+    r0p = _p(_f32(np.asarray(r0).reshape(m, nb)), _f32p) if r0 is not None else None
+    c0p = _p(_f32(np.asarray(c0).reshape(n)), _f32p) if c0 is not None else None
+    keep = (r0p, c0p)  # noqa: F841 (keep the arrays alive through the call)
+    lib().oracle_solve_ex(_p(W, _f32p), m, n, fmt, G, T, flags, r0p, c0p, tp, nt,
+                          _p(r, _f32p), _p(c, _f32p), _p(sT, _f32p), _p(err, _f64p),
+                          _p(w2, _f64p))
     trace = err / w2[0] if w2[0] > 0 else err
     return {"r": r, "c": c, "s_T": float(sT[0]), "trace": trace, "err": err, "w2": float(w2[0])}
 

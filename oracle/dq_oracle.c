@@ -351,6 +351,14 @@ static double tile_error(const float* W, int64_t m, int64_t n, int fmt, int G, i
   return e;
 }
 
+/* Ablation flags (Table 4, scale ablation): ALPHA_ONLY keeps the column
+ * scales fixed and runs only the row half-steps; BETA_ONLY keeps the
+ * row-block scales fixed and runs only the column half-steps. */
+#define ORACLE_ALPHA_ONLY 1
+#define ORACLE_BETA_ONLY 2
+/* Warm start with a given NVFP4 tensor scale: *s_T is read, not computed. */
+#define ORACLE_KEEP_S 4
+
 /* ------------------------------------------------------------------ */
 /* Algorithm 1 on one m x G tile (columns b*G .. b*G+G-1).             */
 /* Per round (Section 4.3, cycle (i)-(iv); Appendix A.2):              */
@@ -362,16 +370,18 @@ static double tile_error(const float* W, int64_t m, int64_t n, int fmt, int G, i
 /* Assumption 1 and the convention that follows it).                   */
 /* err_trace[t] (t = 0..T, may be NULL) accumulates the tile's squared */
 /* error at the scales after round t (t = 0: initialisation).          */
+/* flags skip the row (BETA_ONLY) or column (ALPHA_ONLY) half-step.    */
 /* ------------------------------------------------------------------ */
-static void solve_tile(const float* W, int64_t m, int64_t n, int fmt, int G, int T, int64_t b,
-                       float s_T, float* r, float* c, double* err_trace) {
+static void solve_tile_flags(const float* W, int64_t m, int64_t n, int fmt, int G, int T,
+                             int64_t b, float s_T, float* r, float* c, double* err_trace,
+                             int flags) {
   int64_t nb = n / G;
   double* num = (double*)malloc(sizeof(double) * (size_t)G);
   double* den = (double*)malloc(sizeof(double) * (size_t)G);
   if (err_trace) err_trace[0] += tile_error(W, m, n, fmt, G, b, r, c);
   for (int t = 1; t <= T; ++t) {
     /* row half-step */
-    for (int64_t i = 0; i < m; ++i) {
+    for (int64_t i = 0; i < m && !(flags & ORACLE_BETA_ONLY); ++i) {
       float alpha = inv32(r[i * nb + b]);
       double sn = 0.0, sd = 0.0;
       for (int j = 0; j < G; ++j) {
@@ -386,7 +396,7 @@ static void solve_tile(const float* W, int64_t m, int64_t n, int fmt, int G, int
     }
     /* re-quantise, column half-step */
     for (int j = 0; j < G; ++j) { num[j] = 0.0; den[j] = 0.0; }
-    for (int64_t i = 0; i < m; ++i) {
+    for (int64_t i = 0; i < m && !(flags & ORACLE_ALPHA_ONLY); ++i) {
       float rr = r[i * nb + b];
       float alpha = inv32(rr);
       for (int j = 0; j < G; ++j) {
@@ -398,12 +408,17 @@ static void solve_tile(const float* W, int64_t m, int64_t n, int fmt, int G, int
         den[j] += S * S;
       }
     }
-    for (int j = 0; j < G; ++j)
+    for (int j = 0; j < G && !(flags & ORACLE_ALPHA_ONLY); ++j)
       c[b * G + j] = (den[j] > 0.0) ? proj_beta(fmt, num[j] / den[j]) : proj_beta(fmt, 1.0);
     if (err_trace) err_trace[t] += tile_error(W, m, n, fmt, G, b, r, c);
   }
   free(num);
   free(den);
+}
+
+static void solve_tile(const float* W, int64_t m, int64_t n, int fmt, int G, int T, int64_t b,
+                       float s_T, float* r, float* c, double* err_trace) {
+  solve_tile_flags(W, m, n, fmt, G, T, b, s_T, r, c, err_trace, 0);
 }
 
 /* Full solve of the listed tiles (all tiles when tiles == NULL).
@@ -433,6 +448,52 @@ void oracle_solve(const float* W, int64_t m, int64_t n, int fmt, int G, int T,
   for (int64_t k = 0; k < cnt; ++k) {
     int64_t b = tiles ? tiles[k] : k;
     solve_tile(W, m, n, fmt, G, T, b, sT, r, c, err_trace);
+  }
+}
+
+/* Algorithm 1 with an ablation mode and an optional warm start.
+ * flags: 0 both scales (as oracle_solve), ORACLE_ALPHA_ONLY (Table 4
+ * "alpha-only": beta fixed, at 1 unless c0 is given), ORACLE_BETA_ONLY
+ * (Table 4 "beta-only": alpha fixed at its initial value, the format-native
+ * RTN scale of W diag(c)^-1 unless r0 is given).
+ * c0 (n, nullable): initial column scales, projected onto F_beta (Section
+ * 4.3 projection); replaces the l1 initialisation.  The NVFP4 tensor scale
+ * is then taken with these c, unless ORACLE_KEEP_S is set: then *s_T is
+ * an input (NVFP4) and kept, so that a solve resumed from an earlier
+ * result (r, c, s_T) continues it exactly.  r0 (m x n/G, nullable): initial
+ * row-block scales, projected onto F_alpha; replaces the RTN
+ * initialisation. */
+void oracle_solve_ex(const float* W, int64_t m, int64_t n, int fmt, int G, int T, int flags,
+                     const float* r0, const float* c0, const int64_t* tiles, int64_t ntiles,
+                     float* r, float* c, float* s_T, double* err_trace, double* w2) {
+  int64_t nb = n / G;
+  if (c0) {
+    for (int64_t j = 0; j < n; ++j) c[j] = proj_beta(fmt, (double)c0[j]);
+  } else if (flags & ORACLE_ALPHA_ONLY) {
+    for (int64_t j = 0; j < n; ++j) c[j] = proj_beta(fmt, 1.0);
+  } else {
+    oracle_init_c(W, m, n, fmt, G, c);
+  }
+  float sT = 1.0f;
+  if (fmt == F_NVFP4) sT = (flags & ORACLE_KEEP_S) ? *s_T : oracle_tensor_scale(W, m, n, c);
+  *s_T = sT;
+  int64_t cnt = tiles ? ntiles : nb;
+  if (err_trace) for (int t = 0; t <= T; ++t) err_trace[t] = 0.0;
+  double ww = 0.0;
+  for (int64_t k = 0; k < cnt; ++k) {
+    int64_t b = tiles ? tiles[k] : k;
+    for (int64_t i = 0; i < m; ++i)
+      for (int j = 0; j < G; ++j) { double v = W[i * n + b * G + j]; ww += v * v; }
+  }
+  if (w2) *w2 = ww;
+  if (r0) {
+    for (int64_t i = 0; i < m * nb; ++i) r[i] = proj_alpha(fmt, (double)r0[i], sT);
+  } else {
+    for (int64_t b = 0; b < nb; ++b) init_r_tile(W, m, n, fmt, G, b, c, sT, r);
+  }
+  for (int64_t k = 0; k < cnt; ++k) {
+    int64_t b = tiles ? tiles[k] : k;
+    solve_tile_flags(W, m, n, fmt, G, T, b, sT, r, c, err_trace, flags);
   }
 }
 
