@@ -354,6 +354,17 @@ def run_ours(args, rank, world, local_rank):
             kt[(M, j)] = (t_act, t_gemm)
             del Bc
         del Xc
+    # ---- solver ablation modes (Table 4 arms) on the largest weight: both
+    # scales, alpha-only, beta-only; each mode is one dq_solve_scales_ex call
+    jb = max(range(len(Wd)), key=lambda j: Wd[j].numel())
+    Wb, bb = Wd[jb], Wbuf[jb]
+    modes = {"both": 0, "alpha_only": dq.DQ_SOLVE_ALPHA_ONLY, "beta_only": dq.DQ_SOLVE_BETA_ONLY}
+    mode_ms = {}
+    for name, flags in modes.items():
+        mode_ms[name] = 1e-3 * per_launch_us(lambda i: dq.dq_solve_scales_ex(
+            Wb, fmt, T, bb["r"], bb["c"], bb["sT"], flags=flags, workspace=ws, group=G), 3)
+    # restore the step's scales of that weight (the last mode overwrote them)
+    dq.dq_solve_scales(Wb, fmt, T, bb["r"], bb["c"], bb["sT"], None, ws, group=G)
     torch.cuda.synchronize()
     if dq.dq_device_error(clear=True) != 0:
         raise RuntimeError("device error word set during the per-kernel timing")
@@ -460,6 +471,14 @@ def run_ours(args, rank, world, local_rank):
         "per_M_us": per_m,
         "per_kernel_timing": "after the timed steps: launches back to back between two events, "
                              "each on its own copy of the inputs (copies > 2x L2)",
+        "solver_modes": {
+            "weight": list(Wb.shape), "T": T, "ms_per_call": mode_ms,
+            "achieved_tops": {k: (12.0 if k == "both" else 6.0) * Wb.numel() * T
+                              / (v * 1e-3) / 1e12 for k, v in mode_ms.items()},
+            "frac_alu": {k: (12.0 if k == "both" else 6.0) * Wb.numel() * T
+                         / (v * 1e-3) / 1e12 / alu_peak for k, v in mode_ms.items()},
+            "note": "Table 4 arms through dq_solve_scales_ex; algorithmic fp32 ops per "
+                    "element per round: 12 (both half-steps), 6 (one half-step)"},
         "solver": {"gbs_effective": solver_gbs, "frac_hbm": solver_gbs / hbm,
                    "ms_per_weight_set": solve_ms / args.steps,
                    "definition": "T * bytes(W bf16) / solver time (tile stays on chip)"},

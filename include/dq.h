@@ -120,6 +120,49 @@ DQ_API int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_
                     void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * dq_solve_scales_ex -- dq_solve_scales with an ablation mode and a warm
+ * start.  dq_solve_scales(...) is dq_solve_scales_ex with flags 0 and no
+ * r0 / c0.
+ *
+ * flags (dq_solve_flags, OR-ed; ALPHA_ONLY and BETA_ONLY exclude each other):
+ *  DQ_SOLVE_ALPHA_ONLY  the "alpha-only" arm of the scale ablation
+ *           (Table 4): beta stays fixed -- at 1 (c = 1), or at the
+ *           projection of c0 when given -- and each round is the row
+ *           half-step only (Eq. 10 / Eq. 11).  With T = 0 and no c0 this is
+ *           the single-scale RTN quantiser (Appendix F baseline).
+ *  DQ_SOLVE_BETA_ONLY   the "beta-only" arm: alpha stays at its initial
+ *           value (RTN of W diag(c0)^-1, or the projection of r0 when
+ *           given) and each round is the column half-step only (Eq. 14 /
+ *           Eq. 15).
+ *  DQ_SOLVE_KEEP_TENSOR_SCALE  NVFP4: *s_tensor is an INPUT (device fp32,
+ *           positive, finite) and is used as the per-tensor scale instead
+ *           of amax(W diag(c0)^-1)/2688; it is not written.  Resuming from
+ *           an earlier result (r, c, s_tensor) with this flag continues
+ *           that solve exactly: T1 rounds then T2 resumed rounds give the
+ *           scales and trace tail of T1 + T2 rounds.  Ignored (s_tensor
+ *           receives 1.0) for the other formats.
+ *  r0       nullable, device, m x (n/G) fp32, positive and finite: initial
+ *           row-block scales (the initialisation (alpha_0, beta_0) of
+ *           Section 5.3 given by the caller), each projected onto F_alpha
+ *           (nearest admissible value; NVFP4 with the tensor scale in use).
+ *           May alias r (in-place resume).
+ *  c0       nullable, device, n fp32, positive and finite: initial column
+ *           scales, each projected onto F_beta; replaces the l1
+ *           initialisation.  May alias c.
+ * The other arguments and the error behaviour are those of dq_solve_scales;
+ * unknown flag bits or both ablation flags return DQ_ERR_ARG.
+ * ---------------------------------------------------------------------- */
+typedef enum {
+  DQ_SOLVE_ALPHA_ONLY = 1,
+  DQ_SOLVE_BETA_ONLY = 2,
+  DQ_SOLVE_KEEP_TENSOR_SCALE = 4
+} dq_solve_flags;
+DQ_API int dq_solve_scales_ex(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f,
+                              int group, int T, unsigned flags, const float* r0, const float* c0,
+                              float* r, float* c, float* s_tensor, double* mse_trace,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * dq_quantize_weight -- the stored low-precision weight of Algorithm 1's
  * result, What = Q(Diag(alpha) W Diag(beta)), packed for the GEMM
  * (Section 4.4 artefacts; Appendix I, packed offline).

@@ -78,3 +78,22 @@ def rel_fro(a, b):
     b = np.asarray(b, np.float64)
     den = np.linalg.norm(b)
     return float(np.linalg.norm(a - b) / (den if den > 0 else 1.0))
+
+
+def gpu_solve_ex(W, fmt, G, T, flags=0, r0=None, c0=None, s_T=None, wdtype=torch.bfloat16):
+    """dq_solve_scales_ex on seeded host inputs; r0 / c0 / s_T (host) are
+    copied into the output buffers, which the call reads in place."""
+    m, n = W.shape
+    Wd = to_dev(W.astype(np.float32), wdtype)
+    r = (to_dev(np.asarray(r0, np.float32).reshape(m, n // G)) if r0 is not None else
+         torch.full((m, n // G), -1.0, dtype=torch.float32, device=DEV))
+    c = (to_dev(np.asarray(c0, np.float32).reshape(n)) if c0 is not None else
+         torch.full((n,), -1.0, dtype=torch.float32, device=DEV))
+    sT = to_dev(np.array([s_T if s_T is not None else 0.0], np.float32))
+    tr = torch.full((T + 1,), -1.0, dtype=torch.float64, device=DEV)
+    ws = torch.full((dq.solve_workspace_size(T),), 0x5A, dtype=torch.uint8, device=DEV)
+    dq.dq_solve_scales_ex(Wd, fmt, T, r, c, sT, flags=flags,
+                          r0=r if r0 is not None else None, c0=c if c0 is not None else None,
+                          mse_trace=tr, workspace=ws, group=G)
+    torch.cuda.synchronize()
+    return r.cpu().numpy(), c.cpu().numpy(), float(sT.cpu()[0]), tr.cpu().numpy()

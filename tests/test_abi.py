@@ -59,6 +59,14 @@ def test_invalid_arguments_rejected_without_launch(L):
     assert L.dq_solve_scales(fake, 1, 64, 40, 3, 16, 5, fake, fake, fake, None, ws, 4096, None) == 1
     # workspace too small
     assert L.dq_solve_scales(fake, 1, 64, 64, 3, 16, 5, fake, fake, fake, None, ws, 8, None) == 5
+    # ablation flags: both arms at once, or an unknown bit; misaligned r0
+    for flags in (3, 8, 1 | 16):
+        assert L.dq_solve_scales_ex(fake, 1, 64, 64, 3, 16, 5, flags, None, None, fake, fake,
+                                    fake, None, ws, 4096, None) == 1
+    assert L.dq_solve_scales_ex(fake, 1, 64, 64, 3, 16, 5, 0, ctypes.c_void_p(0x1002), None,
+                                fake, fake, fake, None, ws, 4096, None) == 1
+    assert L.dq_solve_scales_ex(fake, 1, 64, 64, 3, 16, 5, 4, None, None, fake, fake, fake, None,
+                                ws, 8, None) == 5
     # bad group for the format
     assert L.dq_quantize_weight(fake, 1, 64, 64, 2, 16, fake, fake, fake, fake, fake, None) == 1
     # NVFP4 weight packing needs the tensor scale pointer

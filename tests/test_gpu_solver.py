@@ -3,7 +3,10 @@
 Tolerance (fp accumulation order differs: fp32 per thread + fp64 across
 threads on the GPU, fp64 sequential in the oracle): final normalised MSE
 within 1e-4 relative, >= 99.9 % identical codes, the MSE trace within 1e-4
-relative per round, the NVFP4 tensor scale identical.  Full-size layers are
+relative per round, the NVFP4 tensor scale identical.  The scales
+themselves are also compared bit for bit: the kernel recomputes any update
+that lies within its fp32 error bound of a projection boundary from exact
+fp64 sums, so its decisions are those of exact arithmetic, as the oracle's.  Full-size layers are
 checked on sampled column-block tiles (tiles are independent problems)."""
 import numpy as np
 import pytest
@@ -31,6 +34,9 @@ def _compare(W, fmt, G, T, tiles, r, c, sT, trace=None):
     same = float(np.mean(q_g == q_o))
     assert same >= 0.999, same
     assert sT == res["s_T"]
+    # every scale decision is the exact one (updates near a projection
+    # boundary are recomputed from exact fp64 sums): the oracle's scales
+    assert np.array_equal(r_g, r_o) and np.array_equal(c_g, c_o)
     if trace is not None and len(tiles) == W.shape[1] // G:
         np.testing.assert_allclose(trace, res["trace"], rtol=1e-4, atol=0)
     return same, float(np.mean(r_g == r_o)), float(np.mean(c_g == c_o))
@@ -75,9 +81,9 @@ def test_solver_full_size_sampled_tiles(workload, index, fmt, G):
     nb = W.shape[1] // G
     tiles = [0, nb // 3, nb - 1]
     _compare(W, fmt, G, T, tiles, r, c, sT)
-    # initial column scales over every column agree with the oracle's
+    # initial column scales over every column are the oracle's
     c0_g = gpu_solve(W, fmt, G, 0, trace=False)[1]
-    assert np.mean(c0_g == O.init_c(W, fmt, G)) >= 0.999
+    assert np.array_equal(c0_g, O.init_c(W, fmt, G))
     assert np.all(np.isfinite(tr)) and tr[-1] <= tr[0]
 
 
@@ -102,5 +108,5 @@ def test_solver_t0_is_initialisation():
     for fmt, G in [(O.NVFP4, 16), (O.MXFP4, 32), (O.INT4, 64)]:
         r, c, sT, tr = gpu_solve(W, fmt, G, 0)
         res = O.solve(W, fmt, G, 0)
-        assert np.mean(r == res["r"]) >= 0.999 and np.mean(c == res["c"]) >= 0.999
+        assert np.array_equal(r, res["r"]) and np.array_equal(c, res["c"])
         np.testing.assert_allclose(tr, res["trace"], rtol=1e-4)

@@ -90,7 +90,7 @@ const char* dq_status_string(int s) {
   return "unknown dq status";
 }
 
-int dq_version(void) { return 100; }
+int dq_version(void) { return 200; }
 
 int dq_native_group(dq_format f) {
   switch (f) {
@@ -112,18 +112,29 @@ size_t dq_scales_bytes(int64_t rows, int64_t k, dq_format f, int group) {
 
 size_t dq_solve_workspace_size(int T) { return T < 0 ? 0 : dq::solve_workspace_bytes(T); }
 
-int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f, int group,
-                    int T, float* r, float* c, float* s_tensor, double* mse_trace,
-                    void* workspace, size_t ws_bytes, void* stream) {
+int dq_solve_scales_ex(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f, int group,
+                       int T, unsigned flags, const float* r0, const float* c0, float* r,
+                       float* c, float* s_tensor, double* mse_trace, void* workspace,
+                       size_t ws_bytes, void* stream) {
   const int G = resolve_group(f, group);
+  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE;
   if (!W || !r || !c || !s_tensor || m <= 0 || n <= 0 || T < 0 || !valid_dtype(wt) ||
       !valid_group(f, G) || n % G || !aligned(W, 16) || !aligned(r, 4) || !aligned(c, 4) ||
+      !aligned(r0, 4) || !aligned(c0, 4) || (flags & ~known) ||
+      ((flags & DQ_SOLVE_ALPHA_ONLY) && (flags & DQ_SOLVE_BETA_ONLY)) ||
       m > (int64_t)1 << 30 || n > (int64_t)1 << 30)
     return DQ_ERR_ARG;
   if (!workspace || ws_bytes < dq::solve_workspace_bytes(T) || !aligned(workspace, 16))
     return DQ_ERR_WORKSPACE;
-  return dq::solve_scales(W, wt, m, n, f, G, T, r, c, s_tensor, mse_trace, workspace,
-                          (cudaStream_t)stream);
+  return dq::solve_scales(W, wt, m, n, f, G, T, flags, r0, c0, r, c, s_tensor, mse_trace,
+                          workspace, (cudaStream_t)stream);
+}
+
+int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f, int group,
+                    int T, float* r, float* c, float* s_tensor, double* mse_trace,
+                    void* workspace, size_t ws_bytes, void* stream) {
+  return dq_solve_scales_ex(W, wt, m, n, f, group, T, 0u, nullptr, nullptr, r, c, s_tensor,
+                            mse_trace, workspace, ws_bytes, stream);
 }
 
 int dq_quantize_weight(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f, int group,

@@ -11,8 +11,9 @@
 namespace dq {
 
 size_t solve_workspace_bytes(int T);
-int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int T, float* r,
-                 float* c, float* sT, double* trace, void* ws, cudaStream_t st);
+int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int T,
+                 unsigned flags, const float* r0, const float* c0, float* r, float* c, float* sT,
+                 double* trace, void* ws, cudaStream_t st);
 int quantize_act(const void* X, int xt, int64_t M, int64_t K, const float* c, int f, int G,
                  uint8_t* codes, void* scales, float* s_tok, cudaStream_t st);
 int quantize_weight(const void* W, int wt, int64_t m, int64_t n, int f, int G, const float* r,

@@ -48,6 +48,16 @@ struct SolverWs {
   double err[1];
 };
 
+// Ablation mode and warm start (DualQuant, Table 4 scale ablation; the
+// initialisation (alpha_0, beta_0) of Section 5.3 given by the caller).
+// Flag values are those of dq_solve_flags in include/dq.h.
+struct SolveOpts {
+  unsigned flags;
+  const float* r0;   // nullable, m x (n/G)
+  const float* c0;   // nullable, n
+};
+constexpr unsigned SOLVE_ALPHA_ONLY = 1u, SOLVE_BETA_ONLY = 2u, SOLVE_KEEP_S = 4u;
+
 template <typename WT>
 __device__ __forceinline__ void load8(const WT* __restrict__ W, int64_t off, float* x);
 template <>
@@ -134,6 +144,68 @@ __device__ __forceinline__ void cta_octet_reduce(const float* acc, float* scr, d
   __syncthreads();
 }
 
+// Same reduction for V fp64 partials per thread; scr (the float scratch of
+// SolverSmem) is reused as OPB * V * (RPS + 1) doubles, V <= 8.
+template <int G, int V>
+__device__ __forceinline__ void cta_octet_reduce_f64(const double* acc, double* scr,
+                                                     double* part, double* out) {
+  using S = SolverShape<G>;
+  constexpr int NV = S::OPB * V;
+  constexpr int P = S::NT / NV;
+  constexpr int SPP = S::RPS / P;
+  static_assert(V <= 8 && S::NT % NV == 0 && S::RPS % P == 0, "reduction shape");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int oct = lane % S::OPB, rslot = warp * S::RPW + lane / S::OPB;
+#pragma unroll
+  for (int v = 0; v < V; ++v) scr[(oct * V + v) * (S::RPS + 1) + rslot] = acc[v];
+  __syncthreads();
+  {
+    const int gv = tid % NV, p = tid / NV;
+    double s = 0.0;
+    const double* src = scr + gv * (S::RPS + 1) + p * SPP;
+    for (int i = 0; i < SPP; ++i) s += src[i];
+    part[gv * P + p] = s;
+  }
+  __syncthreads();
+  if (tid < NV) {
+    double s = 0.0;
+    for (int p = 0; p < P; ++p) s += part[tid * P + p];
+    out[tid] = s;
+  }
+  __syncthreads();
+}
+
+// Closeness of an fp32 scale update to a rounding boundary of its
+// projection.  The fast passes sum positive terms in fp32 (row: a tree of
+// depth at most 9 per row-block; column: a chain of at most `steps` terms
+// per thread, then fp64), so num and den are each within (depth) * 2^-24
+// relative of their exact values and the quotient within 2 * depth + 4 fp32
+// ulps.  An update whose distance to a boundary is inside that window is
+// recomputed from exact fp64 sums, so that every projected scale is the one
+// the exact quotient selects.  win = half-width of the window in ulps.
+__device__ __forceinline__ bool near_half(uint32_t bits, int drop, uint32_t win) {
+  const uint32_t mask = (1u << drop) - 1u, half = 1u << (drop - 1);
+  return ((bits - half + win) & mask) <= 2u * win;   // |low bits - half| <= win
+}
+template <int F>
+__device__ __forceinline__ bool near_tie_beta(float u, uint32_t win) {
+  if constexpr (F == NVFP4) {
+    // UE4M3: 3 mantissa bits above 2^-6; below it (subnormal steps of 2^-9,
+    // a rare range) every update takes the exact path
+    return u < 0.015625f || near_half(__float_as_uint(u), 20, win);
+  } else if constexpr (F == MXFP4 || F == MXINT4) {
+    return near_half(__float_as_uint(u), 23, win);      // E8M0: midpoint 1.5 * 2^k
+  } else {
+    return near_half(__float_as_uint(u), 16, win);      // bf16
+  }
+}
+template <int F>
+__device__ __forceinline__ bool near_tie_alpha(float u, float inv_sT, uint32_t win) {
+  if constexpr (F == NVFP4) return near_tie_beta<F>(u * inv_sT, win + 2);  // + fl(1/s_T)
+  else return near_tie_beta<F>(u, win);
+}
+constexpr uint32_t ROW_TIE_WIN = 24;   // 2 * 9 + 4, rounded up
+
 template <int G>
 struct SolverSmem {
   using S = SolverShape<G>;
@@ -141,19 +213,21 @@ struct SolverSmem {
   double part[S::NT];                       // NV * P == NT
   double cpart[2][2 * G];                   // cluster-visible, double-buffered
   float c_s[G], b_s[G];
-  double l1[G];
+  float b_old[G];                           // beta before the column update
+  double l1[G];                             // init: column l1; main: exact-pass totals
 };
 
 // ---------------------------------------------------------------------------
 // Initialisation kernel: c0 (Section 5.3, read as the inverse column scale
 // proportional to the column l1 norm, normalised to mean 1 per tile and
-// projected onto F_beta), the NVFP4 per-tensor amax of W diag(c0)^-1, and
-// ||W||_F^2 for the trace normalisation.
+// projected onto F_beta; or the projection of the caller's c0, or of 1 for
+// alpha-only), the NVFP4 per-tensor amax of W diag(c0)^-1 (unless the
+// caller's tensor scale is kept), and ||W||_F^2 for the trace.
 // ---------------------------------------------------------------------------
 template <int F, int G, typename WT>
 __global__ void __launch_bounds__(SolverShape<G>::NT)
-solve_init_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, float* __restrict__ c,
-                  SolverWs* ws) {
+solve_init_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, float* c,
+                  SolverWs* ws, SolveOpts o) {
   using S = SolverShape<G>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SolverSmem<G>& sm = *reinterpret_cast<SolverSmem<G>*>(smem_raw);
@@ -163,10 +237,16 @@ solve_init_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, flo
   const int64_t b = blockIdx.y;
   const int64_t col0 = b * G + oct * 8;
   const int64_t row0 = (int64_t)rank * steps * S::RPS;
+  // the caller's c0 is read before the cluster barrier below, after which
+  // rank 0 writes c (c0 may alias c)
+  const bool given_c = o.c0 != nullptr || (o.flags & SOLVE_ALPHA_ONLY);
+  const float c0v = (o.c0 != nullptr && tid < G) ? o.c0[b * G + tid] : 1.0f;
 
-  float acc[8];
+  // column l1 norms in fp64 (exact for bf16 weights: the same sums as a
+  // sequential fp64 loop), so c0's projection decisions are the exact ones
+  double acc[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+  for (int k = 0; k < 8; ++k) acc[k] = 0.0;
   float w2 = 0.0f;
   for (int s = 0; s < steps; ++s) {
     int64_t i = row0 + (int64_t)s * S::RPS + rslot;
@@ -175,7 +255,7 @@ solve_init_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, flo
       load8<WT>(W, i * n + col0, x);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        acc[k] += fabsf(x[k]);
+        acc[k] += (double)fabsf(x[k]);
         w2 = fmaf(x[k], x[k], w2);
       }
     }
@@ -185,7 +265,8 @@ solve_init_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, flo
   for (int o = 16; o; o >>= 1) w2 += __shfl_xor_sync(0xffffffffu, w2, o);
   if (lane == 0) atomicAdd(&ws->w2, (double)w2);
 
-  cta_octet_reduce<G, 8>(acc, sm.scr, sm.part, sm.cpart[0]);  // cpart[0][j] = CTA l1 of col j
+  cta_octet_reduce_f64<G, 8>(acc, reinterpret_cast<double*>(sm.scr), sm.part,
+                             sm.cpart[0]);  // cpart[0][j] = CTA l1 of col j
   cluster_sync_all();
   if (tid < G) {
     double s = 0.0;
@@ -198,13 +279,15 @@ solve_init_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, flo
     for (int j = 0; j < G; ++j) mean += sm.l1[j];
     mean /= (double)G;
     double v = sm.l1[tid];
-    float cj = (mean > 0.0 && v > 0.0) ? proj_beta<F>((float)(v / mean)) : proj_beta<F>(1.0f);
+    float cj = given_c                  ? proj_beta<F>(c0v)
+               : (mean > 0.0 && v > 0.0) ? proj_beta<F>((float)(v / mean))
+                                         : proj_beta<F>(1.0f);
     sm.c_s[tid] = cj;
     sm.b_s[tid] = __frcp_rn(cj);
     if (rank == 0) c[b * G + tid] = cj;
   }
   __syncthreads();
-  if constexpr (F == NVFP4) {
+  if (F == NVFP4 && !(o.flags & SOLVE_KEEP_S)) {
     float beta[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) beta[k] = sm.b_s[oct * 8 + k];
@@ -284,6 +367,21 @@ __device__ __forceinline__ void grid8_packed(const float2* z, float2* q) {
   }
 }
 
+// Grid value of one pair of arguments (as grid8_packed).
+template <int F>
+__device__ __forceinline__ float2 grid2_packed(float2 z) {
+  if constexpr (is_int_grid(F)) {
+    return make_float2(rintf(fminf(fmaxf(z.x, -8.0f), 7.0f)), rintf(fminf(fmaxf(z.y, -8.0f), 7.0f)));
+  } else {
+    uint32_t h;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(h) : "f"(z.x), "f"(z.y));
+    return __half22float2(*reinterpret_cast<__half2*>(&h));
+  }
+}
+
 template <typename WT>
 __device__ __forceinline__ void unpack8(const WT* p, float2* x);
 template <>
@@ -315,13 +413,24 @@ __device__ __forceinline__ void unpack8_global(const WT* __restrict__ p, float2*
   }
 }
 
+// Columns 2k, 2k+1 of an 8-column piece, as fp32.
+template <typename T>
+__device__ __forceinline__ float2 load_pair(const T* p, int k) {
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(p + 2 * k);
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  } else {
+    return *reinterpret_cast<const float2*>(p + 2 * k);
+  }
+}
+
 // STG: 0 rows stream through the read-only global path, 1 rows staged in
 // shared memory as WT, 2 rows staged as fp32 (no unpacking in the passes).
 template <int F, int G, typename WT, int STG, bool TRACE>
 __global__ void __launch_bounds__(SolverShape<G>::NT, 2048 / SolverShape<G>::NT / 2)
 solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int T,
-                 float* __restrict__ r_out, float* __restrict__ c_io, float* __restrict__ sT_out,
-                 SolverWs* ws) {
+                 float* r_out, float* __restrict__ c_io, float* sT_io, SolverWs* ws,
+                 SolveOpts o) {
   using S = SolverShape<G>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SolverSmem<G>& sm = *reinterpret_cast<SolverSmem<G>*>(smem_raw);
@@ -341,17 +450,23 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
   const int64_t row0 = (int64_t)rank * steps * S::RPS;
   const int rows_cta = steps * S::RPS;
 
+  const bool alpha_only = o.flags & SOLVE_ALPHA_ONLY, beta_only = o.flags & SOLVE_BETA_ONLY;
+  const bool keep_s = F == NVFP4 && (o.flags & SOLVE_KEEP_S);
   float sT = 1.0f;
   if constexpr (F == NVFP4) {
-    float amax = __uint_as_float(*(volatile uint32_t*)&ws->amax_bits);
-    sT = (amax > 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+    if (keep_s) {
+      sT = *sT_io;
+    } else {
+      float amax = __uint_as_float(*(volatile uint32_t*)&ws->amax_bits);
+      sT = (amax > 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+    }
     if (tid < 128) {
       float rv = __fmul_rn(sT, ue4m3_value(tid ? (uint32_t)tid : 1u));
       rtab[tid] = rv;
       atab[tid] = __frcp_rn(rv);
     }
   }
-  if (rank == 0 && b == 0 && tid == 0) *sT_out = sT;
+  if (rank == 0 && b == 0 && tid == 0 && !keep_s) *sT_io = sT;
   const float inv_sT = __frcp_rn(sT);
 
   if constexpr (STG == 2) {
@@ -406,9 +521,25 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
     cc[k] = make_float2(c_io[col0 + 2 * k], c_io[col0 + 2 * k + 1]);
     beta[k] = make_float2(__frcp_rn(cc[k].x), __frcp_rn(cc[k].y));
   }
+  if (tid < G) {   // the current beta also in shared memory (exact column pass)
+    sm.c_s[tid] = c_io[b * G + tid];
+    sm.b_s[tid] = __frcp_rn(sm.c_s[tid]);
+  }
 
-  // r0: format-native absmax scale of W diag(c0)^-1 per row-block (IEEE
-  // arithmetic: the same fp32 decisions as the oracle's initialisation)
+  // r0: the caller's scales projected onto F_alpha (rows past m take the
+  // projection of 1), or else the format-native absmax scale of
+  // W diag(c0)^-1 per row-block (IEEE arithmetic: the same fp32 decisions
+  // as the oracle's initialisation).  Each r0 entry is read by the thread
+  // that writes the same entry of r at the end (r0 may alias r).
+  if (o.r0 != nullptr) {
+    if (oct == 0)
+      for (int s = 0; s < steps; ++s) {
+        const float u = s < s_end ? o.r0[(first_row + (int64_t)s * S::RPS) * nb + b] : 1.0f;
+        const float rv = proj_alpha<F>(u, sT);
+        rsl[s * S::RPS] = rv;
+        asl[s * S::RPS] = __frcp_rn(rv);
+      }
+  } else
   for (int s = 0; s < steps; ++s) {
     float a = 0.0f;
     if (s < s_end) {
@@ -430,10 +561,14 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
   }
   __syncwarp();
 
+  int xb = 0;  // exchange buffer of the next column exchange
+  // column window: 2 * steps + 4 ulps, + 4 for S = r q rounded to fp32
+  const uint32_t col_win = 2u * (uint32_t)steps + 8u;
   for (int t = 0; t <= T; ++t) {
     // ---- row half-step (t < T) / error at the current scales ----
     float e_acc = 0.0f;
-    if (t < T || TRACE) {
+    bool any_tie = false;
+    if ((t < T && !beta_only) || TRACE) {
       for (int s = 0; s < steps; ++s) {
         const bool valid = s < s_end;
         float2 num2 = make_float2(0.f, 0.f), den2 = num2, err2 = num2;
@@ -464,12 +599,56 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
           if constexpr (TRACE) err += __shfl_xor_sync(0xffffffffu, err, o);
         }
         if (TRACE && oct == 0) e_acc += err;
-        if (t < T && oct == 0 && valid) {
-          float rn, an;
-          if (den > 0.0f) RowProj<F>::apply(__fdividef(num, den), inv_sT, rtab, atab, sT, rn, an);
-          else RowProj<F>::apply(1.0f, inv_sT, rtab, atab, sT, rn, an);
-          rsl[s * S::RPS] = rn;
-          asl[s * S::RPS] = an;
+        if (t < T && !beta_only) {
+          const float u = den > 0.0f ? __fdividef(num, den) : 1.0f;
+          // all lanes of a row-block hold the same sums, hence the same flag
+          const bool tie = den > 0.0f && near_tie_alpha<F>(u, inv_sT, ROW_TIE_WIN);  // den = 0 past m
+          any_tie |= tie;
+          if (oct == 0 && valid) {
+            float rn, an;
+            RowProj<F>::apply(u, inv_sT, rtab, atab, sT, rn, an);
+            // exact update pending: r holds -alpha (the alpha it needs)
+            rsl[s * S::RPS] = tie ? -alpha : rn;
+            asl[s * S::RPS] = an;
+          }
+        }
+      }
+      // rare: row-blocks whose update lies near a projection boundary get it
+      // from exact sums -- <W_i, R_i> and ||R_i||^2 in fp64 (x * R is exact
+      // in fp64, R = q * c exact in fp32), the quotient rounded once to fp32
+      if (t < T && !beta_only && __any_sync(0xffffffffu, any_tie)) {
+        __syncwarp();
+        for (int s = 0; s < steps; ++s) {
+          const bool need = rsl[s * S::RPS] < 0.0f;   // the same word for the whole row-block
+          if (!__any_sync(0xffffffffu, need)) continue;
+          double dn = 0.0, dd = 0.0;
+          if (need) {   // one column pair at a time (few live registers)
+            const float alpha = -rsl[s * S::RPS];
+            const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              float2 xp;
+              if constexpr (WSMEM) xp = load_pair<ST>(xsm + s * XSM_STEP, k);
+              else xp = load_pair<WT>(xgl + s * xgl_step, k);
+              const float2 q = grid2_packed<F>(__fmul2_rn(__fmul2_rn(xp, beta[k]), a2));
+              const float2 R = __fmul2_rn(q, cc[k]);
+              dn = fma((double)xp.x, (double)R.x, dn);
+              dn = fma((double)xp.y, (double)R.y, dn);
+              dd = fma((double)R.x, (double)R.x, dd);
+              dd = fma((double)R.y, (double)R.y, dd);
+            }
+          }
+#pragma unroll
+          for (int o = 1; o < S::OPB; o <<= 1) {
+            dn += __shfl_xor_sync(0xffffffffu, dn, o);
+            dd += __shfl_xor_sync(0xffffffffu, dd, o);
+          }
+          __syncwarp();
+          if (need && oct == 0) {
+            const float rn = proj_alpha<F>((float)(dn / dd), sT);
+            rsl[s * S::RPS] = rn;
+            asl[s * S::RPS] = __frcp_rn(rn);
+          }
         }
       }
     }
@@ -480,6 +659,7 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
     }
     if (t == T) break;
     __syncwarp();
+    if (alpha_only) continue;
 
     // ---- column half-step: re-quantise with the new r, update c ----
     float2 acc[8];
@@ -511,19 +691,24 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
       accv[4 * k + 2] = acc[2 * k].y;       // num of column 2k+1
       accv[4 * k + 3] = acc[2 * k + 1].y;   // den of column 2k+1
     }
-    const int par = t & 1;
-    cta_octet_reduce<G, 16>(accv, sm.scr, sm.part, sm.cpart[par]);
+    // the exchange buffer alternates with every exchange: a CTA writes
+    // buffer xb only after all peers passed the barrier that follows their
+    // last reads of it
+    cta_octet_reduce<G, 16>(accv, sm.scr, sm.part, sm.cpart[xb]);
     cluster_sync_all();
-    if (tid < G) {
-      const int j = tid, o = j >> 3, k = j & 7;
-      double sn = 0.0, sd = 0.0;   // rank order; four CTAs' partials in flight at a time
+    // column j's total (num, den) over the cluster, summed in rank order;
+    // four CTAs' partials in flight at a time
+    auto cluster_sum = [&](int j, double& sn, double& sd) {
+      const int o = j >> 3, k = j & 7;
+      sn = 0.0;
+      sd = 0.0;
       for (int q0 = 0; q0 < (int)C; q0 += 4) {
         double pn[4], pd[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
           if (q0 + u < (int)C) {
-            pn[u] = ld_dsmem_f64(&sm.cpart[par][o * 16 + 2 * k], (uint32_t)(q0 + u));
-            pd[u] = ld_dsmem_f64(&sm.cpart[par][o * 16 + 2 * k + 1], (uint32_t)(q0 + u));
+            pn[u] = ld_dsmem_f64(&sm.cpart[xb][o * 16 + 2 * k], (uint32_t)(q0 + u));
+            pd[u] = ld_dsmem_f64(&sm.cpart[xb][o * 16 + 2 * k + 1], (uint32_t)(q0 + u));
           }
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -532,11 +717,66 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
             sd += pd[u];
           }
       }
-      float cn = (sd > 0.0) ? proj_beta<F>((float)(sn / sd)) : proj_beta<F>(1.0f);
-      sm.c_s[j] = cn;
-      sm.b_s[j] = __frcp_rn(cn);
+    };
+    // projected update, written at once; a column near a projection
+    // boundary is redone below from exact sums
+    bool ctie = false;
+    if (tid < G) {
+      double sn, sd;
+      cluster_sum(tid, sn, sd);
+      const float cu = (sd > 0.0) ? (float)(sn / sd) : 1.0f;
+      ctie = sd > 0.0 && near_tie_beta<F>(cu, col_win);
+      const float cn = proj_beta<F>(cu);
+      sm.b_old[tid] = sm.b_s[tid];
+      sm.c_s[tid] = cn;
+      sm.b_s[tid] = __frcp_rn(cn);
     }
-    __syncthreads();
+    xb ^= 1;
+    // every CTA of the cluster sums the same partials in the same order, so
+    // the flag is cluster-uniform and the exact pass below (with its cluster
+    // barrier) runs in all of them or in none
+    if (__syncthreads_or(ctie)) {
+      // rare: exact fp64 column sums of the tile
+      // -- per thread <S_j, W_j> and ||S_j||^2 for one column pair of its
+      // octet at a time, S = r q formed in fp64 (exact) and S * S rounded
+      // once as in a plain fp64 loop, reduced over the CTA in fp64 into the
+      // exchange layout of the fast pass (the old beta from shared memory,
+      // the pair loaded on its own: no register array is indexed by kp)
+#pragma unroll 1
+      for (int kp = 0; kp < 4; ++kp) {
+        double a4[4] = {0.0, 0.0, 0.0, 0.0};
+        const float2 bp = make_float2(sm.b_old[oct * 8 + 2 * kp], sm.b_old[oct * 8 + 2 * kp + 1]);
+        for (int s = 0; s < s_end; ++s) {
+          const float rr = rsl[s * S::RPS], alpha = asl[s * S::RPS];
+          float2 xp;
+          if constexpr (WSMEM) xp = load_pair<ST>(xsm + s * XSM_STEP, kp);
+          else xp = load_pair<WT>(xgl + s * xgl_step, kp);
+          const float2 q = grid2_packed<F>(__fmul2_rn(__fmul2_rn(xp, bp), make_float2(alpha, alpha)));
+          const double s0 = (double)rr * (double)q.x, s1 = (double)rr * (double)q.y;
+          a4[0] = __dadd_rn(a4[0], __dmul_rn(s0, (double)xp.x));
+          a4[1] = __dadd_rn(a4[1], __dmul_rn(s0, s0));
+          a4[2] = __dadd_rn(a4[2], __dmul_rn(s1, (double)xp.y));
+          a4[3] = __dadd_rn(a4[3], __dmul_rn(s1, s1));
+        }
+        cta_octet_reduce_f64<G, 4>(a4, reinterpret_cast<double*>(sm.scr), sm.part, sm.l1);
+        if (tid < S::OPB * 4) sm.cpart[xb][(tid >> 2) * 16 + 4 * kp + (tid & 3)] = sm.l1[tid];
+        __syncthreads();
+      }
+      cluster_sync_all();
+      if (ctie) {   // rank order, one CTA at a time (rare path)
+        const int o = tid >> 3, k = tid & 7;
+        double sn = 0.0, sd = 0.0;
+        for (uint32_t q = 0; q < C; ++q) {
+          sn += ld_dsmem_f64(&sm.cpart[xb][o * 16 + 2 * k], q);
+          sd += ld_dsmem_f64(&sm.cpart[xb][o * 16 + 2 * k + 1], q);
+        }
+        const float cn = proj_beta<F>((float)(sn / sd));
+        sm.c_s[tid] = cn;
+        sm.b_s[tid] = __frcp_rn(cn);
+      }
+      xb ^= 1;
+      __syncthreads();
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       cc[k] = make_float2(sm.c_s[oct * 8 + 2 * k], sm.c_s[oct * 8 + 2 * k + 1]);
@@ -547,7 +787,7 @@ solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int 
   // outputs
   for (int s = 0; s < s_end; ++s)
     if (oct == 0) r_out[(first_row + (int64_t)s * S::RPS) * nb + b] = rsl[s * S::RPS];
-  if (rank == 0 && tid < G && T > 0) c_io[b * G + tid] = sm.c_s[tid];
+  if (rank == 0 && tid < G && T > 0 && !alpha_only) c_io[b * G + tid] = sm.c_s[tid];
   cluster_sync_all();  // no CTA leaves while a peer may still read its cpart
 }
 
@@ -598,8 +838,9 @@ static bool allow_big_cluster(K kern, size_t smem) {
 }
 
 template <int F, int G, typename WT>
-static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, float* r, float* c,
-                         float* sT, double* trace, SolverWs* ws, cudaStream_t st) {
+static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, const SolveOpts& o,
+                         float* r, float* c, float* sT, double* trace, SolverWs* ws,
+                         cudaStream_t st) {
   using S = SolverShape<G>;
   const WT* W = reinterpret_cast<const WT*>(Wv);
   int steps, C, stg;
@@ -624,7 +865,7 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, float* r, 
   auto kinit = solve_init_kernel<F, G, WT>;
   if (!allow_big_cluster(kinit, sm_init)) return DQ_ERR_CUDA;
   cfg.dynamicSmemBytes = sm_init;
-  if (cudaLaunchKernelEx(&cfg, kinit, W, m, n, steps, c, ws) != cudaSuccess) return DQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kinit, W, m, n, steps, c, ws, o) != cudaSuccess) return DQ_ERR_CUDA;
 
   cfg.dynamicSmemBytes = sm_main;
   cudaError_t e;
@@ -632,7 +873,7 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, float* r, 
   {                                                                                         \
     auto km = solve_bcd_kernel<F, G, WT, WS, TR>;                                          \
     if (!allow_big_cluster(km, sm_main)) return DQ_ERR_CUDA;                               \
-    e = cudaLaunchKernelEx(&cfg, km, W, m, n, steps, T, r, c, sT, ws);                      \
+    e = cudaLaunchKernelEx(&cfg, km, W, m, n, steps, T, r, c, sT, ws, o);                   \
   }
   if (stg == 2) {
     if (trace) DQ_MAIN(2, true) else DQ_MAIN(2, false)
@@ -651,16 +892,17 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, float* r, 
 }
 
 template <typename WT>
-static int dispatch_solver(const void* W, int64_t m, int64_t n, int f, int G, int T, float* r,
-                           float* c, float* sT, double* trace, SolverWs* ws, cudaStream_t st) {
+static int dispatch_solver(const void* W, int64_t m, int64_t n, int f, int G, int T,
+                           const SolveOpts& o, float* r, float* c, float* sT, double* trace,
+                           SolverWs* ws, cudaStream_t st) {
   switch (f) {
-    case NVFP4: return launch_solver<NVFP4, 16, WT>(W, m, n, T, r, c, sT, trace, ws, st);
-    case MXFP4: return launch_solver<MXFP4, 32, WT>(W, m, n, T, r, c, sT, trace, ws, st);
-    case MXINT4: return launch_solver<MXINT4, 32, WT>(W, m, n, T, r, c, sT, trace, ws, st);
+    case NVFP4: return launch_solver<NVFP4, 16, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
+    case MXFP4: return launch_solver<MXFP4, 32, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
+    case MXINT4: return launch_solver<MXINT4, 32, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
     case INT4:
-      if (G == 32) return launch_solver<INT4, 32, WT>(W, m, n, T, r, c, sT, trace, ws, st);
-      if (G == 64) return launch_solver<INT4, 64, WT>(W, m, n, T, r, c, sT, trace, ws, st);
-      return launch_solver<INT4, 128, WT>(W, m, n, T, r, c, sT, trace, ws, st);
+      if (G == 32) return launch_solver<INT4, 32, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
+      if (G == 64) return launch_solver<INT4, 64, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
+      return launch_solver<INT4, 128, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
   }
   return DQ_ERR_ARG;
 }
@@ -670,13 +912,15 @@ size_t solve_workspace_bytes(int T) {
   return (b + 255) & ~(size_t)255;
 }
 
-int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int T, float* r,
-                 float* c, float* sT, double* trace, void* ws, cudaStream_t st) {
+int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int T,
+                 unsigned flags, const float* r0, const float* c0, float* r, float* c, float* sT,
+                 double* trace, void* ws, cudaStream_t st) {
   if (cudaMemsetAsync(ws, 0, solve_workspace_bytes(T), st) != cudaSuccess) return DQ_ERR_CUDA;
   SolverWs* w = reinterpret_cast<SolverWs*>(ws);
+  const SolveOpts o{flags, r0, c0};
   if (wt == 1)
-    return dispatch_solver<__nv_bfloat16>(W, m, n, f, G, T, r, c, sT, trace, w, st);
-  return dispatch_solver<float>(W, m, n, f, G, T, r, c, sT, trace, w, st);
+    return dispatch_solver<__nv_bfloat16>(W, m, n, f, G, T, o, r, c, sT, trace, w, st);
+  return dispatch_solver<float>(W, m, n, f, G, T, o, r, c, sT, trace, w, st);
 }
 
 }  // namespace dq

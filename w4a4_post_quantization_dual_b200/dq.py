@@ -30,6 +30,8 @@ SIGNATURES = {
     "dq_solve_workspace_size": (_sz, [_int]),
     "dq_solve_scales": (_int, [_vp, _int, _i64, _i64, _int, _int, _int, _vp, _vp, _vp, _vp, _vp,
                                _sz, _vp]),
+    "dq_solve_scales_ex": (_int, [_vp, _int, _i64, _i64, _int, _int, _int, ctypes.c_uint, _vp,
+                                  _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "dq_quantize_weight": (_int, [_vp, _int, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp,
                                   _vp]),
     "dq_quantize_act": (_int, [_vp, _int, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp, _vp]),
@@ -114,6 +116,25 @@ def dq_solve_scales(W, fmt, T, r, c, s_tensor, mse_trace=None, workspace=None, g
                                  _ptr(s_tensor), _ptr(mse_trace), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)),
            "dq_solve_scales")
+
+
+DQ_SOLVE_ALPHA_ONLY, DQ_SOLVE_BETA_ONLY, DQ_SOLVE_KEEP_TENSOR_SCALE = 1, 2, 4
+
+
+def dq_solve_scales_ex(W, fmt, T, r, c, s_tensor, flags=0, r0=None, c0=None, mse_trace=None,
+                       workspace=None, group=0, stream=None):
+    """Algorithm 1 with an ablation mode (DQ_SOLVE_ALPHA_ONLY / _BETA_ONLY),
+    optional initial scales r0 / c0 and DQ_SOLVE_KEEP_TENSOR_SCALE (s_tensor
+    read as input) -- see include/dq.h."""
+    m, n = W.shape
+    if workspace is None:
+        raise DQError("workspace required (solve_workspace_size(T) bytes)")
+    _check(lib().dq_solve_scales_ex(_ptr(W), _dtype(W), m, n, _fmt(fmt), group, T, flags,
+                                    _ptr(r0), _ptr(c0), _ptr(r), _ptr(c), _ptr(s_tensor),
+                                    _ptr(mse_trace), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(),
+                                    _stream(stream)),
+           "dq_solve_scales_ex")
 
 
 def dq_solve_scales_noalloc(W, fmt, T, r, c, s_tensor, mse_trace=None, group=0, stream=None):
