@@ -365,6 +365,16 @@ def run_ours(args, rank, world, local_rank):
             Wb, fmt, T, bb["r"], bb["c"], bb["sT"], flags=flags, workspace=ws, group=G), 3)
     # restore the step's scales of that weight (the last mode overwrote them)
     dq.dq_solve_scales(Wb, fmt, T, bb["r"], bb["c"], bb["sT"], None, ws, group=G)
+    # activation SQNR of the prefill activations with each weight's column
+    # scales (beta) and without them (Appendix E, Table 6)
+    act_sqnr = {}
+    for W, b in zip(Wd, Wbuf):
+        key = f"N{W.shape[0]}"
+        act_sqnr[key] = {"with_beta_db": dq.act_sqnr_db(Xd[prefill_M], fmt, b["c"], group=G)}
+    no_beta = dq.act_sqnr_db(Xd[prefill_M], fmt, None, group=G)
+    for v in act_sqnr.values():
+        v["without_beta_db"] = no_beta
+        v["delta_db"] = v["with_beta_db"] - no_beta
     torch.cuda.synchronize()
     if dq.dq_device_error(clear=True) != 0:
         raise RuntimeError("device error word set during the per-kernel timing")
@@ -479,6 +489,11 @@ def run_ours(args, rank, world, local_rank):
                          / (v * 1e-3) / 1e12 / alu_peak for k, v in mode_ms.items()},
             "note": "Table 4 arms through dq_solve_scales_ex; algorithmic fp32 ops per "
                     "element per round: 12 (both half-steps), 6 (one half-step)"},
+        "act_sqnr": {"per_weight": act_sqnr, "rows": prefill_M,
+                     "note": "SQNR of the dequantised activations mapped back by 1/c vs X, "
+                             "measured on the device (dq_act_quant_error); synthetic "
+                             "activations and weights, so the sign of the delta is not the "
+                             "paper's model result"},
         "solver": {"gbs_effective": solver_gbs, "frac_hbm": solver_gbs / hbm,
                    "ms_per_weight_set": solve_ms / args.steps,
                    "definition": "T * bytes(W bf16) / solver time (tile stays on chip)"},

@@ -242,6 +242,27 @@ DQ_API int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_to
                    dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream);
 
 /* ------------------------------------------------------------------------
+ * dq_act_quant_error -- quantisation error of the activation path, for the
+ * activation SQNR with and without the column scales (Appendix E, Table 6:
+ * the quantised weights held fixed, only the presence of the beta
+ * pre-scaling varies).
+ *
+ *  X        M x K (dtype xt), the activations before rescaling.
+ *  c        K fp32 column scales that dq_quantize_act used (NULL = none,
+ *           i.e. the path without beta).
+ *  codes, scales, s_tok  as written by dq_quantize_act(X, c, f, group).
+ *  sums     out, device, 2 doubles (the call zeroes them first):
+ *           sums[0] = sum x^2, sums[1] = sum (x - x^)^2, where
+ *           x^_ij = (q_ij * s_blk (* s_tok_i for NVFP4)) / c_j in fp64.
+ *           SQNR (dB) = 10 log10(sums[0] / sums[1]).
+ * K % 8 == 0.  Stream-ordered; the fp64 sums are accumulated with atomics
+ * (summation order unspecified).  Not part of the inference path.
+ * ---------------------------------------------------------------------- */
+DQ_API int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, const float* c,
+                              dq_format f, int group, const uint8_t* codes, const void* scales,
+                              const float* s_tok, double* sums, void* stream);
+
+/* ------------------------------------------------------------------------
  * dq_solve_scales_noalloc -- dq_solve_scales for callers that cannot
  * allocate device memory (the paper has no counterpart: this is a library
  * convenience).  Some callers have no way to provide the workspace: a

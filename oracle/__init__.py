@@ -361,6 +361,32 @@ def linear(A, sA, s_tok, B, sB, s_W, M, N, K, fmt, r_row=None):
     return Y
 
 
+def act_error_sums(X, c, fmt, G):
+    """Quantisation error of the activation path (Appendix E, Table 6): X is
+    rescaled by c (None: without beta, c = 1), quantised by quantize_act,
+    dequantised and mapped back by 1/c, all in fp64.  Returns
+    (sum x^2, sum (x - x^)^2) over all elements."""
+    X = _f32(X)
+    M, K = X.shape
+    cc = np.ones(K, np.float32) if c is None else _f32(c)
+    cod, sc, st = quantize_act(X, cc, fmt, G)
+    if fmt == INT4:
+        q = elem_value_table(fmt)[unpack_codes(cod, K)]
+        s = np.vectorize(bf16_value)(sc.astype(np.int64))
+        xt = q * np.repeat(s, G, axis=1)
+    else:
+        xt = dequant(cod, sc, M, K, fmt, G, st if fmt == NVFP4 else None)
+    xh = xt / cc.astype(np.float64)[None, :]
+    x = X.astype(np.float64)
+    return float(np.sum(x * x)), float(np.sum((x - xh) ** 2))
+
+
+def act_sqnr_db(X, c, fmt, G):
+    """10 log10(sum x^2 / sum (x - x^)^2) of act_error_sums."""
+    sx, se = act_error_sums(X, c, fmt, G)
+    return 10.0 * np.log10(sx / se) if se > 0 else np.inf
+
+
 def dequant_rows(packed, sf, row_idx, K, fmt, G=None):
     """Dequantised rows `row_idx` (fp64, len(row_idx) x K) of an operand whose
     codes are (R, K/2) bytes and whose scales are in the GEMM layout."""

@@ -160,6 +160,18 @@ int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, const floa
   return dq::quantize_act(X, xt, M, K, c, f, G, codes, scales, s_tok, (cudaStream_t)stream);
 }
 
+int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, const float* c,
+                       dq_format f, int group, const uint8_t* codes, const void* scales,
+                       const float* s_tok, double* sums, void* stream) {
+  const int G = resolve_group(f, group);
+  if (!X || !codes || !scales || !sums || M <= 0 || K <= 0 || !valid_dtype(xt) ||
+      !valid_group(f, G) || K % G || K % 8 || !aligned(X, 16) || !aligned(codes, 4) ||
+      !aligned(scales, 2) || !aligned(sums, 8) || !aligned(c, 4) || (f == DQ_NVFP4 && !s_tok))
+    return DQ_ERR_ARG;
+  return dq::act_quant_error(X, xt, M, K, c, f, G, codes, scales, s_tok, sums,
+                             (cudaStream_t)stream);
+}
+
 int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                    const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                    dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream) {

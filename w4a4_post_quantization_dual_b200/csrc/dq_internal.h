@@ -16,6 +16,9 @@ int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int 
                  double* trace, void* ws, cudaStream_t st);
 int quantize_act(const void* X, int xt, int64_t M, int64_t K, const float* c, int f, int G,
                  uint8_t* codes, void* scales, float* s_tok, cudaStream_t st);
+int act_quant_error(const void* X, int xt, int64_t M, int64_t K, const float* c, int f, int G,
+                    const uint8_t* codes, const void* scales, const float* s_tok, double* sums,
+                    cudaStream_t st);
 int quantize_weight(const void* W, int wt, int64_t m, int64_t n, int f, int G, const float* r,
                     const float* c, const float* sT, uint8_t* codes, void* scales,
                     cudaStream_t st);

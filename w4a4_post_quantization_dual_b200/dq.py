@@ -6,6 +6,7 @@ kernels of libdq.so.  There is no CPU or PyTorch fallback: if the library is
 missing or no GPU is present the call raises.
 """
 import ctypes
+import math
 import os
 
 import torch
@@ -39,6 +40,8 @@ SIGNATURES = {
                               _int, _vp]),
     "dq_solve_scales_noalloc": (_int, [_vp, _int, _i64, _i64, _int, _int, _int, _vp, _vp, _vp,
                                        _vp, _vp]),
+    "dq_act_quant_error": (_int, [_vp, _int, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp, _vp,
+                                  _vp]),
     "dq_device_error": (_int, [_int]),
     "dq_version": (_int, []),
 }
@@ -170,6 +173,15 @@ def dq_w4a4_linear(A, sA, s_tok, B, sB, s_w, Y, fmt, r_row=None, stream=None):
            "dq_w4a4_linear")
 
 
+def dq_act_quant_error(X, fmt, c, codes, scales, s_tok, sums, group=0, stream=None):
+    """sums[0] = sum x^2, sums[1] = sum (x - x^)^2 of the activation path (include/dq.h)."""
+    M, K = X.shape
+    _check(lib().dq_act_quant_error(_ptr(X), _dtype(X), M, K, _ptr(c), _fmt(fmt), group,
+                                    _ptr(codes), _ptr(scales), _ptr(s_tok), _ptr(sums),
+                                    _stream(stream)),
+           "dq_act_quant_error")
+
+
 def dq_device_error(clear=True):
     return lib().dq_device_error(1 if clear else 0)
 
@@ -202,6 +214,23 @@ def quantize_linear(W, fmt, T, group=0, mse_trace=False):
     scales = torch.empty(scales_bytes(m, n, fmt, G), dtype=torch.uint8, device=dev)
     dq_quantize_weight(W, fmt, r, c, sT, codes, scales, group=G)
     return QuantizedLinear(codes, scales, c, sT, fmt, G, (m, n)), r, tr
+
+
+def act_sqnr_db(X, fmt, c=None, group=0):
+    """Activation SQNR (dB) of the W4A4 activation path on device activations X:
+    rescale by c (None: without beta), quantise, and compare the dequantised
+    activations mapped back by 1/c with X (Appendix E, Table 6)."""
+    M, K = X.shape
+    dev = X.device
+    G = group or native_group(fmt)
+    A = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    sA = torch.empty(scales_bytes(M, K, fmt, G), dtype=torch.uint8, device=dev)
+    st = torch.empty(M, dtype=torch.float32, device=dev) if _fmt(fmt) == DQ_NVFP4 else None
+    sums = torch.empty(2, dtype=torch.float64, device=dev)
+    dq_quantize_act(X, fmt, c, A, sA, st, group=G)
+    dq_act_quant_error(X, fmt, c, A, sA, st, sums, group=G)
+    s = sums.cpu()
+    return 10.0 * math.log10(float(s[0]) / float(s[1])) if float(s[1]) > 0 else math.inf
 
 
 def linear(X, q: QuantizedLinear, out_dtype=torch.bfloat16, r_row=None):
