@@ -435,6 +435,13 @@ def run_ours(args, rank, world, local_rank):
     gemm_tf = 2.0 * prefill_M * Wd[j0].shape[0] * K0 / (t_gemm * 1e-6) / 1e12
     a_bytes = prefill_M * K0 * (2 + 0.5 + 1.0 / 16) + prefill_M * 4
     act_gbs = a_bytes / (t_act * 1e-6) / 1e9
+    # decode GEMM (M = 1, the largest weight): weight-bandwidth bound; bytes =
+    # codes N*K/2 + scales N*K/16 + A M*K/2 + A scales + Y 2*M*N
+    Md = min(Xd)
+    t_dec = kt[(Md, j0)][1]
+    Nd = Wd[j0].shape[0]
+    dec_bytes = Nd * K0 / 2 + Nd * K0 / 16 + Md * K0 / 2 + Md * K0 / 16 + 4 * Md + 2 * Md * Nd
+    dec_gbs = dec_bytes / (t_dec * 1e-6) / 1e9
     # whole-job throughput: every rank runs the same per-GPU workload (weak
     # scaling); the time is the slowest rank's
     value = world * lin_flops * args.steps / (lin_ms * 1e-3) / 1e12
@@ -478,6 +485,11 @@ def run_ours(args, rank, world, local_rank):
                          "traffic": measured_traffic("act_nvfp4_4096x4096",
                                                      ["dq_quant.cu", "dq_device.cuh"]),
                          "shape": f"M={prefill_M} x K=4096"},
+        "roofline_decode": {"kernel": "w4a4_gemm_splitk_kernel", "bound": "hbm",
+                            "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
+                            "frac": dec_gbs / hbm, "us_per_launch": t_dec,
+                            "algorithmic_bytes": dec_bytes,
+                            "shape": f"M={Md} x N={Nd} x K={K0}"},
         "per_M_us": per_m,
         "per_kernel_timing": "after the timed steps: launches back to back between two events, "
                              "each on its own copy of the inputs (copies > 2x L2)",
