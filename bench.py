@@ -365,6 +365,30 @@ def run_ours(args, rank, world, local_rank):
             Wb, fmt, T, bb["r"], bb["c"], bb["sT"], flags=flags, workspace=ws, group=G), 3)
     # restore the step's scales of that weight (the last mode overwrote them)
     dq.dq_solve_scales(Wb, fmt, T, bb["r"], bb["c"], bb["sT"], None, ws, group=G)
+    # batched solver entry on the seven projections of one Llama-3.1-8B layer
+    # (q, k, v, o, gate, up, down; random bf16 weights, same format and T):
+    # separate calls vs one dq_solve_scales_batched call
+    lshapes = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (14336, 4096),
+               (14336, 4096), (4096, 14336)]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    LW = [(torch.randn(m_, n_, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+          for m_, n_ in lshapes]
+    Lr = [torch.empty((m_, n_ // G), device=dev) for m_, n_ in lshapes]
+    Lc = [torch.empty(n_, device=dev) for _, n_ in lshapes]
+    Ls = [torch.empty(1, device=dev) for _ in lshapes]
+    Lws = torch.empty(dq.solve_batched_workspace_size(len(LW), T), dtype=torch.uint8, device=dev)
+
+    def layer_separate(_):
+        for W_, r_, c_, s_ in zip(LW, Lr, Lc, Ls):
+            dq.dq_solve_scales(W_, fmt, T, r_, c_, s_, None, ws, group=G)
+
+    def layer_batched(_):
+        dq.dq_solve_scales_batched(LW, fmt, T, Lr, Lc, Ls, None, Lws, group=G)
+
+    batched_ms = {"separate": 1e-3 * per_launch_us(layer_separate, 1),
+                  "batched": 1e-3 * per_launch_us(layer_batched, 1)}
+    del LW, Lr, Lc, Ls, Lws
     # activation SQNR of the prefill activations with each weight's column
     # scales (beta) and without them (Appendix E, Table 6)
     act_sqnr = {}
@@ -501,6 +525,10 @@ def run_ours(args, rank, world, local_rank):
                          / (v * 1e-3) / 1e12 / alu_peak for k, v in mode_ms.items()},
             "note": "Table 4 arms through dq_solve_scales_ex; algorithmic fp32 ops per "
                     "element per round: 12 (both half-steps), 6 (one half-step)"},
+        "solver_batched": {"ms_per_layer": batched_ms, "T": T,
+                           "weights": "q, k, v, o 4096/1024 x 4096; gate, up 14336 x 4096; "
+                                      "down 4096 x 14336 (one Llama-3.1-8B layer)",
+                           "launches": {"separate": 14, "batched": 6}},
         "act_sqnr": {"per_weight": act_sqnr, "rows": prefill_M,
                      "note": "SQNR of the dequantised activations mapped back by 1/c vs X, "
                              "measured on the device (dq_act_quant_error); synthetic "

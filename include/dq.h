@@ -242,6 +242,33 @@ DQ_API int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_to
                    dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream);
 
 /* ------------------------------------------------------------------------
+ * dq_solve_scales_batched -- dq_solve_scales on nw weights of one format and
+ * dtype in few launches: weights with the same row count m share one
+ * initialisation and one BCD launch (up to 16 weights per launch), so a
+ * model's many projections fill the GPU together instead of one after the
+ * other.  Every tile is still an independent problem (Algorithm 1 per m x G
+ * tile), so each weight's r, c, s_tensor are exactly those of a separate
+ * dq_solve_scales call; traces agree up to the order of fp64 atomic adds.
+ *
+ *  nw       number of weights (> 0).
+ *  W, m, n  HOST arrays of nw entries: device pointer to weight i (m[i] x
+ *           n[i], dtype wt, 16-byte aligned) and its sizes.
+ *  r, c, s_tensor  HOST arrays of nw device pointers (the outputs of
+ *           dq_solve_scales for weight i).
+ *  mse_trace nullable HOST array of nw nullable device pointers (T+1
+ *           doubles each).
+ *  flags    as dq_solve_scales_ex (warm starts are single-weight only).
+ *  workspace dq_solve_batched_workspace_size(nw, T) bytes, 16-byte aligned.
+ * Errors as dq_solve_scales; nothing is enqueued when an argument is invalid.
+ * ---------------------------------------------------------------------- */
+DQ_API size_t dq_solve_batched_workspace_size(int nw, int T);
+DQ_API int dq_solve_scales_batched(int nw, const void* const* W, dq_dtype wt, const int64_t* m,
+                                   const int64_t* n, dq_format f, int group, int T,
+                                   unsigned flags, float* const* r, float* const* c,
+                                   float* const* s_tensor, double* const* mse_trace,
+                                   void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * dq_act_quant_error -- quantisation error of the activation path, for the
  * activation SQNR with and without the column scales (Appendix E, Table 6:
  * the quantised weights held fixed, only the presence of the beta

@@ -67,6 +67,19 @@ def test_invalid_arguments_rejected_without_launch(L):
                                 fake, fake, fake, None, ws, 4096, None) == 1
     assert L.dq_solve_scales_ex(fake, 1, 64, 64, 3, 16, 5, 4, None, None, fake, fake, fake, None,
                                 ws, 8, None) == 5
+    # batched solver: empty batch, n % G, unknown flag, workspace too small
+    arr = lambda *v: (ctypes.c_void_p * len(v))(*v)
+    i64 = lambda *v: (ctypes.c_int64 * len(v))(*v)
+    two = arr(0x1000, 0x2000)
+    assert L.dq_solve_batched_workspace_size(2, 5) == 2 * L.dq_solve_workspace_size(5)
+    assert L.dq_solve_scales_batched(0, two, 1, i64(64, 64), i64(64, 64), 3, 16, 5, 0, two, two,
+                                     two, None, ws, 4096, None) == 1
+    assert L.dq_solve_scales_batched(2, two, 1, i64(64, 64), i64(64, 40), 3, 16, 5, 0, two, two,
+                                     two, None, ws, 4096, None) == 1
+    assert L.dq_solve_scales_batched(2, two, 1, i64(64, 64), i64(64, 64), 3, 16, 5, 8, two, two,
+                                     two, None, ws, 4096, None) == 1
+    assert L.dq_solve_scales_batched(2, two, 1, i64(64, 64), i64(64, 64), 3, 16, 5, 0, two, two,
+                                     two, None, ws, 100, None) == 5
     # bad group for the format
     assert L.dq_quantize_weight(fake, 1, 64, 64, 2, 16, fake, fake, fake, fake, fake, None) == 1
     # NVFP4 weight packing needs the tensor scale pointer

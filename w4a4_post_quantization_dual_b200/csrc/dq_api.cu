@@ -130,6 +130,33 @@ int dq_solve_scales_ex(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_form
                           workspace, (cudaStream_t)stream);
 }
 
+size_t dq_solve_batched_workspace_size(int nw, int T) {
+  return (T < 0 || nw <= 0) ? 0 : (size_t)nw * dq::solve_workspace_bytes(T);
+}
+
+int dq_solve_scales_batched(int nw, const void* const* W, dq_dtype wt, const int64_t* m,
+                            const int64_t* n, dq_format f, int group, int T, unsigned flags,
+                            float* const* r, float* const* c, float* const* s_tensor,
+                            double* const* mse_trace, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  const int G = resolve_group(f, group);
+  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE;
+  if (nw <= 0 || !W || !m || !n || !r || !c || !s_tensor || T < 0 || !valid_dtype(wt) ||
+      !valid_group(f, G) || (flags & ~known) ||
+      ((flags & DQ_SOLVE_ALPHA_ONLY) && (flags & DQ_SOLVE_BETA_ONLY)))
+    return DQ_ERR_ARG;
+  for (int i = 0; i < nw; ++i) {
+    if (!W[i] || !r[i] || !c[i] || !s_tensor[i] || m[i] <= 0 || n[i] <= 0 || n[i] % G ||
+        !aligned(W[i], 16) || !aligned(r[i], 4) || !aligned(c[i], 4) ||
+        m[i] > (int64_t)1 << 30 || n[i] > (int64_t)1 << 30)
+      return DQ_ERR_ARG;
+  }
+  if (!workspace || ws_bytes < dq_solve_batched_workspace_size(nw, T) || !aligned(workspace, 16))
+    return DQ_ERR_WORKSPACE;
+  return dq::solve_scales_batched(nw, W, wt, m, n, f, G, T, flags, r, c, s_tensor, mse_trace,
+                                  workspace, (cudaStream_t)stream);
+}
+
 int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f, int group,
                     int T, float* r, float* c, float* s_tensor, double* mse_trace,
                     void* workspace, size_t ws_bytes, void* stream) {

@@ -16,6 +16,10 @@ int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int 
                  double* trace, void* ws, cudaStream_t st);
 int quantize_act(const void* X, int xt, int64_t M, int64_t K, const float* c, int f, int G,
                  uint8_t* codes, void* scales, float* s_tok, cudaStream_t st);
+int solve_scales_batched(int nw, const void* const* W, int wt, const int64_t* m,
+                         const int64_t* n, int f, int G, int T, unsigned flags, float* const* r,
+                         float* const* c, float* const* sT, double* const* trace, void* ws,
+                         cudaStream_t st);
 int act_quant_error(const void* X, int xt, int64_t M, int64_t K, const float* c, int f, int G,
                     const uint8_t* codes, const void* scales, const float* s_tok, double* sums,
                     cudaStream_t st);

@@ -25,6 +25,7 @@
 #include <stdint.h>
 
 #include <type_traits>
+#include <vector>
 
 #include "dq_device.cuh"
 #include "dq_internal.h"
@@ -57,6 +58,21 @@ struct SolveOpts {
   const float* c0;   // nullable, n
 };
 constexpr unsigned SOLVE_ALPHA_ONLY = 1u, SOLVE_BETA_ONLY = 2u, SOLVE_KEEP_S = 4u;
+
+// The weights of one launch (all with the same row count m): launch z-index
+// i solves weight i.  Passed by value (kernel parameter space).
+constexpr int SOLVE_BATCH_MAX = 16;
+struct SolveItem {
+  const void* W;      // m x n
+  float* r;           // m x n/G
+  float* c;           // n
+  float* sT;          // 1
+  SolverWs* ws;       // this weight's workspace
+  int64_t n;
+};
+struct SolveBatch {
+  SolveItem item[SOLVE_BATCH_MAX];
+};
 
 template <typename WT>
 __device__ __forceinline__ void load8(const WT* __restrict__ W, int64_t off, float* x);
@@ -226,9 +242,13 @@ struct SolverSmem {
 // ---------------------------------------------------------------------------
 template <int F, int G, typename WT>
 __global__ void __launch_bounds__(SolverShape<G>::NT)
-solve_init_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, float* c,
-                  SolverWs* ws, SolveOpts o) {
+solve_init_kernel(SolveBatch bt, int64_t m, int steps, SolveOpts o) {
   using S = SolverShape<G>;
+  const int64_t n = bt.item[blockIdx.z].n;
+  if ((int64_t)blockIdx.y >= n / G) return;   // whole clusters (they span x only)
+  const WT* __restrict__ W = reinterpret_cast<const WT*>(bt.item[blockIdx.z].W);
+  float* c = bt.item[blockIdx.z].c;
+  SolverWs* ws = bt.item[blockIdx.z].ws;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SolverSmem<G>& sm = *reinterpret_cast<SolverSmem<G>*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -428,10 +448,15 @@ __device__ __forceinline__ float2 load_pair(const T* p, int k) {
 // shared memory as WT, 2 rows staged as fp32 (no unpacking in the passes).
 template <int F, int G, typename WT, int STG, bool TRACE>
 __global__ void __launch_bounds__(SolverShape<G>::NT, 2048 / SolverShape<G>::NT / 2)
-solve_bcd_kernel(const WT* __restrict__ W, int64_t m, int64_t n, int steps, int T,
-                 float* r_out, float* __restrict__ c_io, float* sT_io, SolverWs* ws,
-                 SolveOpts o) {
+solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   using S = SolverShape<G>;
+  const int64_t n = bt.item[blockIdx.z].n;
+  if ((int64_t)blockIdx.y >= n / G) return;   // whole clusters (they span x only)
+  const WT* __restrict__ W = reinterpret_cast<const WT*>(bt.item[blockIdx.z].W);
+  float* r_out = bt.item[blockIdx.z].r;
+  float* __restrict__ c_io = bt.item[blockIdx.z].c;
+  float* sT_io = bt.item[blockIdx.z].sT;
+  SolverWs* ws = bt.item[blockIdx.z].ws;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SolverSmem<G>& sm = *reinterpret_cast<SolverSmem<G>*>(smem_raw);
   float* r_s = reinterpret_cast<float*>(smem_raw + sizeof(SolverSmem<G>));
@@ -844,18 +869,25 @@ static bool allow_big_cluster(K kern, size_t smem) {
   return ensure_kernel_attrs((const void*)kern, (int)smem, true);
 }
 
+// One launch pair (initialisation + BCD) for `count` weights of row count m;
+// traces[i] may be null.
 template <int F, int G, typename WT>
-static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, const SolveOpts& o,
-                         float* r, float* c, float* sT, double* trace, SolverWs* ws,
-                         cudaStream_t st) {
+static int launch_solver(const SolveBatch& bt, int count, int64_t m, int T, const SolveOpts& o,
+                         double* const* traces, cudaStream_t st) {
   using S = SolverShape<G>;
-  const WT* W = reinterpret_cast<const WT*>(Wv);
   int steps, C, stg;
   solver_geometry<G, WT>(m, steps, C, stg);
   const size_t sm_init = sizeof(SolverSmem<G>),
                sm_main = solver_smem_bytes<G>(
                    steps, stg == 2 ? sizeof(float) : (stg == 1 ? sizeof(WT) : 0));
   if (sm_main > 227 * 1024) return DQ_ERR_UNSUPPORTED;
+  int64_t tiles = 0;
+  bool any_trace = false;
+  for (int i = 0; i < count; ++i) {
+    tiles = bt.item[i].n / G > tiles ? bt.item[i].n / G : tiles;
+    any_trace = any_trace || (traces && traces[i]);
+  }
+  if (tiles > 65535) return DQ_ERR_UNSUPPORTED;
 
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -863,7 +895,7 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, const Solv
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(C, (unsigned)(n / G), 1);
+  cfg.gridDim = dim3(C, (unsigned)tiles, (unsigned)count);
   cfg.blockDim = dim3(S::NT, 1, 1);
   cfg.stream = st;
   cfg.attrs = attr;
@@ -872,7 +904,7 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, const Solv
   auto kinit = solve_init_kernel<F, G, WT>;
   if (!allow_big_cluster(kinit, sm_init)) return DQ_ERR_CUDA;
   cfg.dynamicSmemBytes = sm_init;
-  if (cudaLaunchKernelEx(&cfg, kinit, W, m, n, steps, c, ws, o) != cudaSuccess) return DQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kinit, bt, m, steps, o) != cudaSuccess) return DQ_ERR_CUDA;
 
   cfg.dynamicSmemBytes = sm_main;
   cudaError_t e;
@@ -880,36 +912,36 @@ static int launch_solver(const void* Wv, int64_t m, int64_t n, int T, const Solv
   {                                                                                         \
     auto km = solve_bcd_kernel<F, G, WT, WS, TR>;                                          \
     if (!allow_big_cluster(km, sm_main)) return DQ_ERR_CUDA;                               \
-    e = cudaLaunchKernelEx(&cfg, km, W, m, n, steps, T, r, c, sT, ws, o);                   \
+    e = cudaLaunchKernelEx(&cfg, km, bt, m, steps, T, o);                                   \
   }
   if (stg == 2) {
-    if (trace) DQ_MAIN(2, true) else DQ_MAIN(2, false)
+    if (any_trace) DQ_MAIN(2, true) else DQ_MAIN(2, false)
   } else if (stg == 1) {
-    if (trace) DQ_MAIN(1, true) else DQ_MAIN(1, false)
+    if (any_trace) DQ_MAIN(1, true) else DQ_MAIN(1, false)
   } else {
-    if (trace) DQ_MAIN(0, true) else DQ_MAIN(0, false)
+    if (any_trace) DQ_MAIN(0, true) else DQ_MAIN(0, false)
   }
 #undef DQ_MAIN
   if (e != cudaSuccess) return DQ_ERR_CUDA;
-  if (trace) {
-    solve_finalize_kernel<<<(T + 1 + 127) / 128, 128, 0, st>>>(ws, T, trace);
+  for (int i = 0; i < count && any_trace; ++i) {
+    if (!traces[i]) continue;
+    solve_finalize_kernel<<<(T + 1 + 127) / 128, 128, 0, st>>>(bt.item[i].ws, T, traces[i]);
     if (cudaGetLastError() != cudaSuccess) return DQ_ERR_CUDA;
   }
   return DQ_OK;
 }
 
 template <typename WT>
-static int dispatch_solver(const void* W, int64_t m, int64_t n, int f, int G, int T,
-                           const SolveOpts& o, float* r, float* c, float* sT, double* trace,
-                           SolverWs* ws, cudaStream_t st) {
+static int dispatch_solver(int f, int G, const SolveBatch& bt, int count, int64_t m, int T,
+                           const SolveOpts& o, double* const* traces, cudaStream_t st) {
   switch (f) {
-    case NVFP4: return launch_solver<NVFP4, 16, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
-    case MXFP4: return launch_solver<MXFP4, 32, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
-    case MXINT4: return launch_solver<MXINT4, 32, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
+    case NVFP4: return launch_solver<NVFP4, 16, WT>(bt, count, m, T, o, traces, st);
+    case MXFP4: return launch_solver<MXFP4, 32, WT>(bt, count, m, T, o, traces, st);
+    case MXINT4: return launch_solver<MXINT4, 32, WT>(bt, count, m, T, o, traces, st);
     case INT4:
-      if (G == 32) return launch_solver<INT4, 32, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
-      if (G == 64) return launch_solver<INT4, 64, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
-      return launch_solver<INT4, 128, WT>(W, m, n, T, o, r, c, sT, trace, ws, st);
+      if (G == 32) return launch_solver<INT4, 32, WT>(bt, count, m, T, o, traces, st);
+      if (G == 64) return launch_solver<INT4, 64, WT>(bt, count, m, T, o, traces, st);
+      return launch_solver<INT4, 128, WT>(bt, count, m, T, o, traces, st);
   }
   return DQ_ERR_ARG;
 }
@@ -923,11 +955,43 @@ int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int 
                  unsigned flags, const float* r0, const float* c0, float* r, float* c, float* sT,
                  double* trace, void* ws, cudaStream_t st) {
   if (cudaMemsetAsync(ws, 0, solve_workspace_bytes(T), st) != cudaSuccess) return DQ_ERR_CUDA;
-  SolverWs* w = reinterpret_cast<SolverWs*>(ws);
+  SolveBatch bt = {};
+  bt.item[0] = SolveItem{W, r, c, sT, reinterpret_cast<SolverWs*>(ws), n};
   const SolveOpts o{flags, r0, c0};
-  if (wt == 1)
-    return dispatch_solver<__nv_bfloat16>(W, m, n, f, G, T, o, r, c, sT, trace, w, st);
-  return dispatch_solver<float>(W, m, n, f, G, T, o, r, c, sT, trace, w, st);
+  double* traces[1] = {trace};
+  if (wt == 1) return dispatch_solver<__nv_bfloat16>(f, G, bt, 1, m, T, o, traces, st);
+  return dispatch_solver<float>(f, G, bt, 1, m, T, o, traces, st);
+}
+
+// Weights are grouped by row count (one geometry per launch), in order of
+// first appearance, up to SOLVE_BATCH_MAX per launch; a row count with more
+// weights than that is picked up again by the later, not yet done weights.
+int solve_scales_batched(int nw, const void* const* W, int wt, const int64_t* m,
+                         const int64_t* n, int f, int G, int T, unsigned flags, float* const* r,
+                         float* const* c, float* const* sT, double* const* trace, void* ws,
+                         cudaStream_t st) {
+  const size_t per = solve_workspace_bytes(T);
+  if (cudaMemsetAsync(ws, 0, per * (size_t)nw, st) != cudaSuccess) return DQ_ERR_CUDA;
+  const SolveOpts o{flags, nullptr, nullptr};
+  std::vector<char> done((size_t)nw, 0);
+  for (int i = 0; i < nw; ++i) {
+    if (done[i]) continue;
+    SolveBatch bt = {};
+    double* traces[SOLVE_BATCH_MAX] = {};
+    int count = 0;
+    for (int j = i; j < nw && count < SOLVE_BATCH_MAX; ++j) {
+      if (done[j] || m[j] != m[i]) continue;
+      bt.item[count] = SolveItem{W[j], r[j], c[j], sT[j],
+                                 reinterpret_cast<SolverWs*>((char*)ws + per * (size_t)j), n[j]};
+      traces[count] = trace ? trace[j] : nullptr;
+      done[j] = 1;
+      ++count;
+    }
+    const int rc = wt == 1 ? dispatch_solver<__nv_bfloat16>(f, G, bt, count, m[i], T, o, traces, st)
+                           : dispatch_solver<float>(f, G, bt, count, m[i], T, o, traces, st);
+    if (rc != DQ_OK) return rc;
+  }
+  return DQ_OK;
 }
 
 }  // namespace dq

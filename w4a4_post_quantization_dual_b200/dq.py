@@ -40,6 +40,9 @@ SIGNATURES = {
                               _int, _vp]),
     "dq_solve_scales_noalloc": (_int, [_vp, _int, _i64, _i64, _int, _int, _int, _vp, _vp, _vp,
                                        _vp, _vp]),
+    "dq_solve_batched_workspace_size": (_sz, [_int, _int]),
+    "dq_solve_scales_batched": (_int, [_int, _vp, _int, _vp, _vp, _int, _int, _int, ctypes.c_uint,
+                                       _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "dq_act_quant_error": (_int, [_vp, _int, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp, _vp,
                                   _vp]),
     "dq_device_error": (_int, [_int]),
@@ -138,6 +141,29 @@ def dq_solve_scales_ex(W, fmt, T, r, c, s_tensor, flags=0, r0=None, c0=None, mse
                                     workspace.numel() * workspace.element_size(),
                                     _stream(stream)),
            "dq_solve_scales_ex")
+
+
+def solve_batched_workspace_size(nw, T):
+    return lib().dq_solve_batched_workspace_size(nw, T)
+
+
+def dq_solve_scales_batched(Ws, fmt, T, rs, cs, sTs, traces=None, workspace=None, flags=0,
+                            group=0, stream=None):
+    """dq_solve_scales on a list of weights (same dtype) in few launches."""
+    nw = len(Ws)
+    if workspace is None:
+        raise DQError("workspace required (solve_batched_workspace_size(nw, T) bytes)")
+    if len({W.dtype for W in Ws}) != 1:
+        raise DQError("all weights of a batch share one dtype")
+    arr = lambda ts: (ctypes.c_void_p * nw)(*[_ptr(t) for t in ts])
+    m = (ctypes.c_int64 * nw)(*[W.shape[0] for W in Ws])
+    n = (ctypes.c_int64 * nw)(*[W.shape[1] for W in Ws])
+    tr = arr(traces) if traces is not None else None
+    _check(lib().dq_solve_scales_batched(nw, arr(Ws), _dtype(Ws[0]), m, n, _fmt(fmt), group, T,
+                                         flags, arr(rs), arr(cs), arr(sTs), tr, _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(stream)),
+           "dq_solve_scales_batched")
 
 
 def dq_solve_scales_noalloc(W, fmt, T, r, c, s_tensor, mse_trace=None, group=0, stream=None):
