@@ -89,7 +89,9 @@ DQ_API size_t dq_scales_bytes(int64_t rows, int64_t k, dq_format f, int group);
  * coordinate descent, Section 4.3; closed-form updates Eqs. 10 and 14,
  * Appendix B), run independently on every m x G column-block tile of W.
  *
- *  W        m x n, dtype wt (DQ_BF16 or DQ_F32).  n % G == 0.
+ *  W        m x n, dtype wt (DQ_BF16 or DQ_F32).  n % G == 0; n / G <= 65535
+ *           (one launch grid), else DQ_ERR_UNSUPPORTED before anything is
+ *           enqueued.
  *  f, group format and block size G (see dq_format).
  *  T        number of BCD rounds (>= 0).  Each round: quantise, update and
  *           project the row-block scales r, re-quantise, update and project

@@ -80,6 +80,12 @@ def test_invalid_arguments_rejected_without_launch(L):
                                      two, None, ws, 4096, None) == 1
     assert L.dq_solve_scales_batched(2, two, 1, i64(64, 64), i64(64, 64), 3, 16, 5, 0, two, two,
                                      two, None, ws, 100, None) == 5
+    # more column blocks than one launch grid holds: refused before anything is enqueued
+    wide = 16 * 65536
+    assert L.dq_solve_scales(fake, 1, 64, wide, 3, 16, 5, fake, fake, fake, None, ws, 4096,
+                             None) == 2
+    assert L.dq_solve_scales_batched(2, two, 1, i64(64, 64), i64(64, wide), 3, 16, 5, 0, two, two,
+                                     two, None, ws, 4096, None) == 2
     # bad group for the format
     assert L.dq_quantize_weight(fake, 1, 64, 64, 2, 16, fake, fake, fake, fake, fake, None) == 1
     # NVFP4 weight packing needs the tensor scale pointer

@@ -931,6 +931,31 @@ static int launch_solver(const SolveBatch& bt, int count, int64_t m, int T, cons
   return DQ_OK;
 }
 
+// Whether a launch of this shape is possible (grid and shared-memory
+// limits), checked before anything is enqueued.
+template <int G, typename WT>
+static int solver_supported(int64_t m, int64_t n) {
+  int steps, C, stg;
+  solver_geometry<G, WT>(m, steps, C, stg);
+  const size_t sm_main =
+      solver_smem_bytes<G>(steps, stg == 2 ? sizeof(float) : (stg == 1 ? sizeof(WT) : 0));
+  return (sm_main > 227 * 1024 || n / G > 65535) ? DQ_ERR_UNSUPPORTED : DQ_OK;
+}
+
+template <typename WT>
+static int check_solver(int f, int G, int64_t m, int64_t n) {
+  switch (f) {
+    case NVFP4: return solver_supported<16, WT>(m, n);
+    case MXFP4:
+    case MXINT4: return solver_supported<32, WT>(m, n);
+    case INT4:
+      if (G == 32) return solver_supported<32, WT>(m, n);
+      if (G == 64) return solver_supported<64, WT>(m, n);
+      return solver_supported<128, WT>(m, n);
+  }
+  return DQ_ERR_ARG;
+}
+
 template <typename WT>
 static int dispatch_solver(int f, int G, const SolveBatch& bt, int count, int64_t m, int T,
                            const SolveOpts& o, double* const* traces, cudaStream_t st) {
@@ -954,6 +979,8 @@ size_t solve_workspace_bytes(int T) {
 int solve_scales(const void* W, int wt, int64_t m, int64_t n, int f, int G, int T,
                  unsigned flags, const float* r0, const float* c0, float* r, float* c, float* sT,
                  double* trace, void* ws, cudaStream_t st) {
+  const int ok = wt == 1 ? check_solver<__nv_bfloat16>(f, G, m, n) : check_solver<float>(f, G, m, n);
+  if (ok != DQ_OK) return ok;
   if (cudaMemsetAsync(ws, 0, solve_workspace_bytes(T), st) != cudaSuccess) return DQ_ERR_CUDA;
   SolveBatch bt = {};
   bt.item[0] = SolveItem{W, r, c, sT, reinterpret_cast<SolverWs*>(ws), n};
@@ -970,6 +997,11 @@ int solve_scales_batched(int nw, const void* const* W, int wt, const int64_t* m,
                          const int64_t* n, int f, int G, int T, unsigned flags, float* const* r,
                          float* const* c, float* const* sT, double* const* trace, void* ws,
                          cudaStream_t st) {
+  for (int i = 0; i < nw; ++i) {   // every launch possible before any is enqueued
+    const int ok = wt == 1 ? check_solver<__nv_bfloat16>(f, G, m[i], n[i])
+                           : check_solver<float>(f, G, m[i], n[i]);
+    if (ok != DQ_OK) return ok;
+  }
   const size_t per = solve_workspace_bytes(T);
   if (cudaMemsetAsync(ws, 0, per * (size_t)nw, st) != cudaSuccess) return DQ_ERR_CUDA;
   const SolveOpts o{flags, nullptr, nullptr};
