@@ -104,3 +104,22 @@ def test_invalid_arguments_rejected_without_launch(L):
     odd = ctypes.c_void_p(0x1001)
     assert L.dq_w4a4_linear(odd, fake, fake, fake, fake, fake, None, fake, 1, 16, 128, 256,
                             3, None) == 1
+
+
+def test_header_is_plain_c_and_links(L, tmp_path):
+    """include/dq.h compiles as strict C99 and a C program linked against
+    libdq.so gets the documented results from calls that need no GPU."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.join(ROOT, "w4a4_post_quantization_dual_b200", "lib")
+    exe = str(tmp_path / "c_abi_check")
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", exe,
+                    "-L", libdir, "-ldq", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    assert "c abi ok" in out.stdout
