@@ -22,8 +22,12 @@ import numpy as np
 from . import build as _build
 
 INT4, MXINT4, MXFP4, NVFP4 = 0, 1, 2, 3
-FORMAT_NAMES = {"int4": INT4, "mxint4": MXINT4, "mxfp4": MXFP4, "nvfp4": NVFP4}
-NATIVE_GROUP = {INT4: 64, MXINT4: 32, MXFP4: 32, NVFP4: 16}
+INT8, MXINT8, MXFP8 = 4, 5, 6          # 8-bit variants (Appendix G.2, Table 9)
+FORMAT_NAMES = {"int4": INT4, "mxint4": MXINT4, "mxfp4": MXFP4, "nvfp4": NVFP4,
+                "int8": INT8, "mxint8": MXINT8, "mxfp8": MXFP8}
+NATIVE_GROUP = {INT4: 64, MXINT4: 32, MXFP4: 32, NVFP4: 16, INT8: 128, MXINT8: 32, MXFP8: 32}
+EIGHT_BIT = (INT8, MXINT8, MXFP8)
+BF16_SCALED = (INT4, INT8)
 
 _lib = None
 
@@ -46,6 +50,10 @@ def lib():
             "oracle_int4_value": (ctypes.c_double, [ctypes.c_int]),
             "oracle_int4_encode": (ctypes.c_int, [ctypes.c_float]),
             "oracle_e4m3_value": (ctypes.c_double, [ctypes.c_int]),
+            "oracle_int8_value": (ctypes.c_double, [ctypes.c_int]),
+            "oracle_int8_encode": (ctypes.c_int, [ctypes.c_float]),
+            "oracle_e4m3_elem_value": (ctypes.c_double, [ctypes.c_int]),
+            "oracle_e4m3_elem_encode": (ctypes.c_int, [ctypes.c_float]),
             "oracle_ue4m3_rne": (ctypes.c_int, [ctypes.c_double]),
             "oracle_ue4m3_proj": (ctypes.c_int, [ctypes.c_double]),
             "oracle_e8m0_value": (ctypes.c_double, [ctypes.c_int]),
@@ -152,8 +160,28 @@ def proj_beta(fmt, u):
     return lib().oracle_proj_beta(fmt, float(u))
 
 
+def int8_value(code):
+    return lib().oracle_int8_value(int(code))
+
+
+def int8_encode(t):
+    return lib().oracle_int8_encode(float(np.float32(t)))
+
+
+def e4m3_elem_value(code):
+    return lib().oracle_e4m3_elem_value(int(code))
+
+
+def e4m3_elem_encode(t):
+    return lib().oracle_e4m3_elem_encode(float(np.float32(t)))
+
+
 def elem_value_table(fmt):
-    """Value of each of the 16 element codes."""
+    """Value of each element code (16 for the 4-bit grids, 256 for 8-bit)."""
+    if fmt in (INT8, MXINT8):
+        return np.array([int8_value(k) for k in range(256)], dtype=np.float64)
+    if fmt == MXFP8:
+        return np.array([e4m3_elem_value(k) for k in range(256)], dtype=np.float64)
     f = int4_value if fmt in (INT4, MXINT4) else e2m1_value
     return np.array([f(k) for k in range(16)], dtype=np.float64)
 
@@ -285,11 +313,12 @@ def sf_bytes(rows, S):
 
 
 def pack_weight(W, fmt, G, r, c, s_T=1.0):
-    """Packed codes (m, n/2) u8 and scales (GEMM layout bytes, or (m, n/G) u16 bf16 for INT4)."""
+    """Packed codes (m, n/2) u8 ((m, n) for 8-bit formats) and scales (GEMM layout
+    bytes, or (m, n/G) u16 bf16 for INT4 / INT8)."""
     W = _f32(W)
     m, n = W.shape
-    cod = np.empty((m, n // 2), np.uint8)
-    if fmt == INT4:
+    cod = np.empty((m, n if fmt in EIGHT_BIT else n // 2), np.uint8)
+    if fmt in BF16_SCALED:
         sc = np.empty((m, n // G), np.uint16)
     else:
         sc = np.empty(sf_bytes(m, n // G), np.uint8)
@@ -299,11 +328,12 @@ def pack_weight(W, fmt, G, r, c, s_T=1.0):
 
 
 def quantize_act(X, c, fmt, G):
-    """Rescale by c and quantise.  Returns (codes (M, K/2) u8, scales, s_tok (M,) f32)."""
+    """Rescale by c and quantise.  Returns (codes (M, K/2) u8 ((M, K) for 8-bit
+    formats), scales, s_tok (M,) f32)."""
     X = _f32(X)
     M, K = X.shape
-    cod = np.empty((M, K // 2), np.uint8)
-    if fmt == INT4:
+    cod = np.empty((M, K if fmt in EIGHT_BIT else K // 2), np.uint8)
+    if fmt in BF16_SCALED:
         sc = np.empty((M, K // G), np.uint16)
     else:
         sc = np.empty(sf_bytes(M, K // G), np.uint8)
@@ -315,8 +345,11 @@ def quantize_act(X, c, fmt, G):
 
 # ---------------------------------------------------------------- reference GEMM
 def unpack_codes(packed, K):
-    """(R, K/2) bytes -> (R, K) codes, element 2k in the low nibble of byte k."""
+    """(R, K/2) bytes -> (R, K) codes, element 2k in the low nibble of byte k
+    ((R, K) bytes of an 8-bit format are returned as they are)."""
     packed = np.asarray(packed, np.uint8)
+    if packed.shape[1] == K:
+        return packed.copy()
     out = np.empty((packed.shape[0], K), np.uint8)
     out[:, 0::2] = packed & 0xF
     out[:, 1::2] = packed >> 4
@@ -341,7 +374,10 @@ def scale_values(sf, rows, S, fmt):
 def dequant(packed, sf, rows, K, fmt, G, row_scale=None):
     """Dequantised operand (rows, K) fp64 = code value x block scale (x per-row scale)."""
     q = elem_value_table(fmt)[unpack_codes(packed, K)]
-    s = scale_values(sf, rows, K // G, fmt)
+    if fmt in BF16_SCALED:
+        s = np.vectorize(bf16_value)(np.asarray(sf).reshape(rows, K // G).astype(np.int64))
+    else:
+        s = scale_values(sf, rows, K // G, fmt)
     v = q * np.repeat(s, G, axis=1)
     if row_scale is not None:
         v = v * np.asarray(row_scale, np.float64)[:, None]
@@ -370,7 +406,7 @@ def act_error_sums(X, c, fmt, G):
     M, K = X.shape
     cc = np.ones(K, np.float32) if c is None else _f32(c)
     cod, sc, st = quantize_act(X, cc, fmt, G)
-    if fmt == INT4:
+    if fmt in BF16_SCALED:
         q = elem_value_table(fmt)[unpack_codes(cod, K)]
         s = np.vectorize(bf16_value)(sc.astype(np.int64))
         xt = q * np.repeat(s, G, axis=1)

@@ -28,7 +28,21 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { F_INT4 = 0, F_MXINT4 = 1, F_MXFP4 = 2, F_NVFP4 = 3 };
+enum { F_INT4 = 0, F_MXINT4 = 1, F_MXFP4 = 2, F_NVFP4 = 3,
+       F_INT8 = 4, F_MXINT8 = 5, F_MXFP8 = 6 };
+
+/* Format families.  The 8-bit variants (Appendix G.2, Table 9: INT8 with
+ * G = 128, MXINT8 and MXFP8 with G = 32) reuse Algorithm 1 unchanged with
+ * their own element grids: INT8 integers -128..127 (Section 3's integer grid
+ * with B = 8), FP8 E4M3 (OCP MX v1.0 MXFP8 element type). */
+static int is_mx(int fmt) {
+  return fmt == F_MXINT4 || fmt == F_MXFP4 || fmt == F_MXINT8 || fmt == F_MXFP8;
+}
+static int is_8bit(int fmt) { return fmt == F_INT8 || fmt == F_MXINT8 || fmt == F_MXFP8; }
+/* OCP MX shared-exponent rule X = 2^(floor(log2 amax) - emax_elem):
+ * emax_elem = exponent of the element grid's largest power of two
+ * (E2M1 6 -> 2, INT4 7 -> 2, INT8 127 -> 6, E4M3 448 -> 8). */
+static int mx_emax(int fmt) { return fmt == F_MXINT8 ? 6 : (fmt == F_MXFP8 ? 8 : 2); }
 
 /* ------------------------------------------------------------------ */
 /* Element grids (Section 3: "canonical, unit-scale grid")            */
@@ -76,11 +90,44 @@ int oracle_int4_encode(float t) {
   return best & 0xF;
 }
 
+/* INT8 grid: integers -128..127 (Section 3 with B = 8); code = the
+ * two's-complement byte. */
+double oracle_int8_value(int code) {
+  int v = code & 0xFF;
+  return (double)(v >= 128 ? v - 256 : v);
+}
+
+/* proj_G for INT8: nearest integer, ties to even (the IEEE default
+ * rounding of nearbyint), clipped to [-128, 127]. */
+int oracle_int8_encode(float t) {
+  double v = nearbyint((double)t);
+  if (v < -128.0) v = -128.0;
+  if (v > 127.0) v = 127.0;
+  return ((int)v) & 0xFF;
+}
+
+static int elem_encode_e4m3(float t);
+static double elem_value_e4m3(int code);
+
 static int elem_encode(int fmt, float t) {
-  return (fmt == F_MXINT4 || fmt == F_INT4) ? oracle_int4_encode(t) : oracle_e2m1_encode(t);
+  switch (fmt) {
+    case F_INT4:
+    case F_MXINT4: return oracle_int4_encode(t);
+    case F_INT8:
+    case F_MXINT8: return oracle_int8_encode(t);
+    case F_MXFP8: return elem_encode_e4m3(t);
+    default: return oracle_e2m1_encode(t);
+  }
 }
 static double elem_value(int fmt, int code) {
-  return (fmt == F_MXINT4 || fmt == F_INT4) ? oracle_int4_value(code) : oracle_e2m1_value(code);
+  switch (fmt) {
+    case F_INT4:
+    case F_MXINT4: return oracle_int4_value(code);
+    case F_INT8:
+    case F_MXINT8: return oracle_int8_value(code);
+    case F_MXFP8: return elem_value_e4m3(code);
+    default: return oracle_e2m1_value(code);
+  }
 }
 
 /* ------------------------------------------------------------------ */
@@ -117,6 +164,16 @@ int oracle_ue4m3_proj(double u) {
   }
   return best;
 }
+
+/* FP8 E4M3 element (MXFP8): value of the byte (sign bit 7), and the nearest
+ * finite value to t, ties to the even byte, saturating at +-448, the sign
+ * kept from t (a negative t that rounds to 0 gives 0x80). */
+static double elem_value_e4m3(int code) { return oracle_e4m3_value(code & 0xFF); }
+static int elem_encode_e4m3(float t) {
+  return oracle_ue4m3_rne(fabs((double)t)) | (signbit(t) ? 0x80 : 0);
+}
+double oracle_e4m3_elem_value(int code) { return elem_value_e4m3(code); }
+int oracle_e4m3_elem_encode(float t) { return elem_encode_e4m3(t); }
 
 /* E8M0: 2^(b-127), b in 0..254. */
 double oracle_e8m0_value(int b) { return ldexp(1.0, b - 127); }
@@ -183,8 +240,8 @@ double oracle_bf16_proj(double u) {
 /* ------------------------------------------------------------------ */
 /* Projections Pi_F (Section 4.3 "projected onto the admissible set";  */
 /* Appendix C, Remark 1: nearest value of the scale's inverse).        */
-/* F_alpha / F_beta per format (Section 4.2): BF16 for INT4, E8M0 for  */
-/* MXINT4 / MXFP4, UE4M3 for NVFP4 (F_alpha = s_T * UE4M3 with the     */
+/* F_alpha / F_beta per format (Section 4.2): BF16 for INT4 / INT8,     */
+/* E8M0 for the MX formats, UE4M3 for NVFP4 (F_alpha = s_T * UE4M3 with the */
 /* per-tensor fp32 scale s_T fixed at initialisation).                 */
 /* ------------------------------------------------------------------ */
 
@@ -205,7 +262,9 @@ static float proj_alpha(int fmt, double u, float s_T) {
       return (float)((double)s_T * v); /* one fp32 rounding of s_T * v */
     }
     case F_MXFP4:
-    case F_MXINT4: return (float)oracle_e8m0_value(u32 > 0.0f ? oracle_e8m0_proj((double)u32) : 0);
+    case F_MXINT4:
+    case F_MXINT8:
+    case F_MXFP8: return (float)oracle_e8m0_value(u32 > 0.0f ? oracle_e8m0_proj((double)u32) : 0);
     default: return (float)oracle_bf16_proj((double)u32);
   }
 }
@@ -216,7 +275,9 @@ static float proj_beta(int fmt, double u) {
   switch (fmt) {
     case F_NVFP4: return (float)oracle_e4m3_value(oracle_ue4m3_proj((double)u32));
     case F_MXFP4:
-    case F_MXINT4: return (float)oracle_e8m0_value(u32 > 0.0f ? oracle_e8m0_proj((double)u32) : 0);
+    case F_MXINT4:
+    case F_MXINT8:
+    case F_MXFP8: return (float)oracle_e8m0_value(u32 > 0.0f ? oracle_e8m0_proj((double)u32) : 0);
     default: return (float)oracle_bf16_proj((double)u32);
   }
 }
@@ -290,14 +351,20 @@ static float rtn_block_scale(int fmt, float a, float s_T) {
       return proj_alpha(fmt, (double)q, s_T);
     }
     case F_MXFP4:
-    case F_MXINT4: {
-      /* OCP MX: X = 2^(floor(log2 amax) - emax_elem), emax_elem = 2. */
+    case F_MXINT4:
+    case F_MXINT8:
+    case F_MXFP8: {
+      /* OCP MX: X = 2^(floor(log2 amax) - emax_elem). */
       int E;
       frexp((double)a, &E);
-      int k = (E - 1) - 2;
+      int k = (E - 1) - mx_emax(fmt);
       if (k < -127) k = -127;
       if (k > 127) k = 127;
       return (float)ldexp(1.0, k);
+    }
+    case F_INT8: {
+      volatile float q = a / 127.0f;
+      return proj_alpha(fmt, (double)q, s_T);
     }
     default: {
       volatile float q = a / 7.0f;
@@ -574,13 +641,20 @@ int64_t oracle_sf_bytes(int64_t rows, int64_t S) { return ((rows + 127) / 128) *
 
 /* ------------------------------------------------------------------ */
 /* Weight packing (Section 4.4 artefacts; Appendix I "packed offline") */
-/* codes: m x n/2 bytes, element 2k in the low nibble of byte k.       */
+/* codes: m x n/2 bytes, element 2k in the low nibble of byte k        */
+/*        (8-bit formats: m x n bytes, one per element).                */
 /* scales: NVFP4/MX -> one byte per (row, block) in the GEMM layout;   */
 /*         INT4 -> bf16 bits, row-major m x n/G (uint16).               */
 /* ------------------------------------------------------------------ */
 void oracle_pack_weight(const float* W, int64_t m, int64_t n, int fmt, int G, const float* r,
                         const float* c, float s_T, uint8_t* codes, uint8_t* scales) {
   int64_t nb = n / G;
+  if (is_8bit(fmt)) {   /* one byte per element */
+    for (int64_t i = 0; i < m; ++i)
+      for (int64_t j = 0; j < n; ++j)
+        codes[i * n + j] = (uint8_t)elem_encode(
+            fmt, quant_arg(W[i * n + j], inv32(c[j]), inv32(r[i * nb + j / G])));
+  } else
   for (int64_t i = 0; i < m; ++i)
     for (int64_t j = 0; j < n; j += 2) {
       int lo = elem_encode(fmt, quant_arg(W[i * n + j], inv32(c[j]), inv32(r[i * nb + j / G])));
@@ -588,7 +662,7 @@ void oracle_pack_weight(const float* W, int64_t m, int64_t n, int fmt, int G, co
                                           inv32(r[i * nb + (j + 1) / G])));
       codes[i * (n / 2) + j / 2] = (uint8_t)(lo | (hi << 4));
     }
-  if (fmt == F_INT4) {
+  if (fmt == F_INT4 || fmt == F_INT8) {
     uint16_t* s16 = (uint16_t*)scales;
     for (int64_t i = 0; i < m; ++i)
       for (int64_t b = 0; b < nb; ++b) s16[i * nb + b] = (uint16_t)oracle_bf16_rne(r[i * nb + b]);
@@ -623,13 +697,16 @@ void oracle_pack_weight(const float* W, int64_t m, int64_t n, int fmt, int G, co
 /*   MXFP4 / MXINT4: block byte = floor(log2 amax_blk) - 2 + 127;      */
 /*          code = grid(x~ * 2^-e).                                    */
 /*   INT4:  block scale bf16(amax_blk / 7), code = INT4(x~ / scale).   */
+/*   8-bit: MXINT8 / MXFP8 as MX with emax_elem 6 / 8, INT8 with         */
+/*          bf16(amax_blk / 127); codes one byte per element.          */
 /* All products / quotients are single fp32 operations.                */
 /* ------------------------------------------------------------------ */
 void oracle_quantize_act(const float* X, int64_t M, int64_t K, const float* c, int fmt, int G,
                          uint8_t* codes, uint8_t* scales, float* s_tok) {
   int64_t S = K / G;
   float* xt = (float*)malloc(sizeof(float) * (size_t)K);
-  if (fmt != F_INT4) memset(scales, 0, (size_t)oracle_sf_bytes(M, S));
+  const int bf16_scales = fmt == F_INT4 || fmt == F_INT8;
+  if (!bf16_scales) memset(scales, 0, (size_t)oracle_sf_bytes(M, S));
   for (int64_t t = 0; t < M; ++t) {
     float amax = 0.0f;
     for (int64_t j = 0; j < K; ++j) {
@@ -657,12 +734,12 @@ void oracle_quantize_act(const float* X, int64_t M, int64_t K, const float* c, i
         scales[oracle_sf_offset(t, s, S)] = (uint8_t)byte;
         volatile float sblk = (float)oracle_e4m3_value(byte) * st;
         if (sblk == 0.0f) zero = 1; else inv = inv32(sblk);
-      } else if (fmt == F_MXFP4 || fmt == F_MXINT4) {
+      } else if (is_mx(fmt)) {
         int e = -127;
         if (ab > 0.0f) {
           int E;
           frexp((double)ab, &E);
-          e = (E - 1) - 2;
+          e = (E - 1) - mx_emax(fmt);
           if (e < -127) e = -127;
           if (e > 127) e = 127;
         } else {
@@ -671,11 +748,22 @@ void oracle_quantize_act(const float* X, int64_t M, int64_t K, const float* c, i
         scales[oracle_sf_offset(t, s, S)] = (uint8_t)(e + 127);
         inv = (float)ldexp(1.0, -e);
       } else {
-        volatile float q = ab / 7.0f;
+        volatile float q = ab / (fmt == F_INT8 ? 127.0f : 7.0f);
         int h = oracle_bf16_rne((double)q);
         ((uint16_t*)scales)[t * S + s] = (uint16_t)h;
         float sc = (float)oracle_bf16_value(h);
         if (sc == 0.0f) zero = 1; else inv = inv32(sc);
+      }
+      if (is_8bit(fmt)) {   /* one byte per element */
+        for (int j = 0; j < G; ++j) {
+          int q = 0;
+          if (!zero) {
+            volatile float a0 = xt[s * G + j] * inv;
+            q = elem_encode(fmt, a0);
+          }
+          codes[t * K + s * G + j] = (uint8_t)q;
+        }
+        continue;
       }
       for (int j = 0; j < G; j += 2) {
         int lo = 0, hi = 0;
