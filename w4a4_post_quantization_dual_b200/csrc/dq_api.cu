@@ -66,9 +66,15 @@ inline bool valid_group(int f, int G) {
     case DQ_MXFP4:
     case DQ_MXINT4: return G == 32;
     case DQ_INT4: return G == 32 || G == 64 || G == 128;
+    case DQ_MXINT8:
+    case DQ_MXFP8: return G == 32;
+    case DQ_INT8: return G == 32 || G == 64 || G == 128;
   }
   return false;
 }
+
+// 8-bit variants: the solver only, so far
+inline bool is_8bit(int f) { return f == DQ_INT8 || f == DQ_MXINT8 || f == DQ_MXFP8; }
 
 inline int resolve_group(int f, int group) { return group > 0 ? group : dq_native_group((dq_format)f); }
 
@@ -98,6 +104,9 @@ int dq_native_group(dq_format f) {
     case DQ_MXINT4:
     case DQ_MXFP4: return 32;
     case DQ_NVFP4: return 16;
+    case DQ_INT8: return 128;
+    case DQ_MXINT8:
+    case DQ_MXFP8: return 32;
   }
   return 0;
 }
@@ -106,7 +115,7 @@ size_t dq_scales_bytes(int64_t rows, int64_t k, dq_format f, int group) {
   const int G = resolve_group(f, group);
   if (rows < 0 || k <= 0 || !valid_group(f, G) || k % G) return 0;
   const int64_t S = k / G;
-  if (f == DQ_INT4) return (size_t)(rows * S * 2);
+  if (f == DQ_INT4 || f == DQ_INT8) return (size_t)(rows * S * 2);
   return (size_t)(((rows + 127) / 128) * ((S + 3) / 4) * 512);
 }
 
@@ -167,6 +176,7 @@ int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format 
 int dq_quantize_weight(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f, int group,
                        const float* r, const float* c, const float* s_tensor, uint8_t* codes,
                        void* scales, void* stream) {
+  if (is_8bit(f)) return DQ_ERR_UNSUPPORTED;
   const int G = resolve_group(f, group);
   if (!W || !r || !c || !codes || !scales || m <= 0 || n <= 0 || !valid_dtype(wt) ||
       !valid_group(f, G) || n % G || !aligned(W, 16) || !aligned(codes, 16) ||
@@ -179,6 +189,7 @@ int dq_quantize_weight(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_form
 int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, const float* c,
                     dq_format f, int group, uint8_t* codes, void* scales, float* s_tok,
                     void* stream) {
+  if (is_8bit(f)) return DQ_ERR_UNSUPPORTED;
   const int G = resolve_group(f, group);
   if (!X || !codes || !scales || M <= 0 || K <= 0 || !valid_dtype(xt) || !valid_group(f, G) ||
       K % G || !aligned(X, 16) || !aligned(codes, 16) || !aligned(scales, 16) ||
@@ -190,6 +201,7 @@ int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, const floa
 int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, const float* c,
                        dq_format f, int group, const uint8_t* codes, const void* scales,
                        const float* s_tok, double* sums, void* stream) {
+  if (is_8bit(f)) return DQ_ERR_UNSUPPORTED;
   const int G = resolve_group(f, group);
   if (!X || !codes || !scales || !sums || M <= 0 || K <= 0 || !valid_dtype(xt) ||
       !valid_group(f, G) || K % G || K % 8 || !aligned(X, 16) || !aligned(codes, 4) ||
@@ -202,6 +214,7 @@ int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, const f
 int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                    const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                    dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream) {
+  if (is_8bit(f)) return DQ_ERR_UNSUPPORTED;
   if (f == DQ_INT4) return DQ_ERR_UNSUPPORTED;
   if (f != DQ_NVFP4 && f != DQ_MXFP4 && f != DQ_MXINT4) return DQ_ERR_ARG;
   if (!A || !sA || !B || !sB || !Y || M <= 0 || N <= 0 || K <= 0 || !valid_dtype(yt) ||

@@ -15,9 +15,20 @@
 
 namespace dq {
 
-enum Fmt : int { INT4 = 0, MXINT4 = 1, MXFP4 = 2, NVFP4 = 3 };
+enum Fmt : int { INT4 = 0, MXINT4 = 1, MXFP4 = 2, NVFP4 = 3, INT8 = 4, MXINT8 = 5, MXFP8 = 6 };
 
+// 4-bit integer grid (-8..7)
 __host__ __device__ constexpr bool is_int_grid(int f) { return f == INT4 || f == MXINT4; }
+// 8-bit variants (INT8 / MXINT8: integers -128..127; MXFP8: FP8 E4M3)
+__host__ __device__ constexpr bool is_int8_grid(int f) { return f == INT8 || f == MXINT8; }
+__host__ __device__ constexpr bool is_8bit(int f) { return f == INT8 || f == MXINT8 || f == MXFP8; }
+// E8M0 block scales
+__host__ __device__ constexpr bool is_mx(int f) {
+  return f == MXINT4 || f == MXFP4 || f == MXINT8 || f == MXFP8;
+}
+// OCP MX shared-exponent rule 2^(floor(log2 amax) - emax): exponent of the
+// element grid's largest power of two (E2M1 / INT4 2, INT8 6, E4M3 8)
+__host__ __device__ constexpr int mx_emax(int f) { return f == MXINT8 ? 6 : (f == MXFP8 ? 8 : 2); }
 
 // ---------------------------------------------------------------- E2M1
 // Two fp32 -> one byte: x0 in the low nibble, x1 in the high nibble.
@@ -131,7 +142,7 @@ __device__ __forceinline__ float proj_alpha(float u, float sT) {
   if constexpr (F == NVFP4) {
     float v = proj_ue4m3(__fdiv_rn(u, sT));
     return __fmul_rn(sT, v);
-  } else if constexpr (F == MXFP4 || F == MXINT4) {
+  } else if constexpr (is_mx(F)) {
     return proj_e8m0(u);
   } else {
     return proj_bf16(u);
@@ -141,7 +152,7 @@ __device__ __forceinline__ float proj_alpha(float u, float sT) {
 template <int F>
 __device__ __forceinline__ float proj_beta(float u) {
   if constexpr (F == NVFP4) return proj_ue4m3(u);
-  else if constexpr (F == MXFP4 || F == MXINT4) return proj_e8m0(u);
+  else if constexpr (is_mx(F)) return proj_e8m0(u);
   else return proj_bf16(u);
 }
 
@@ -152,12 +163,12 @@ __device__ __forceinline__ float rtn_block_scale(float a, float sT) {
   if (a == 0.0f) return proj_alpha<F>(1.0f, sT);
   if constexpr (F == NVFP4) {
     return proj_alpha<F>(__fdiv_rn(a, 6.0f), sT);
-  } else if constexpr (F == MXFP4 || F == MXINT4) {
-    int k = ilog2f(a) - 2;
+  } else if constexpr (is_mx(F)) {
+    int k = ilog2f(a) - mx_emax(F);
     k = k < -127 ? -127 : (k > 127 ? 127 : k);
     return pow2f(k);
   } else {
-    return proj_bf16(__fdiv_rn(a, 7.0f));
+    return proj_bf16(__fdiv_rn(a, F == INT8 ? 127.0f : 7.0f));
   }
 }
 

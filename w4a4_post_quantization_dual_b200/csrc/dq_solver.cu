@@ -90,23 +90,6 @@ __device__ __forceinline__ void load8<float>(const float* __restrict__ W, int64_
   x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 
-// Quantise 8 fp32 arguments z to grid VALUES (E2M1 or INT4).
-template <int F>
-__device__ __forceinline__ void grid8(const float* z, float* q) {
-  if constexpr (is_int_grid(F)) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) q[k] = int4_value_rn(z[k]);
-  } else {
-    uint32_t codes = e2m1x8(z);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float2 v = __half22float2(e2m1x2_to_half2((codes >> (8 * k)) & 0xFFu));
-      q[2 * k] = v.x;
-      q[2 * k + 1] = v.y;
-    }
-  }
-}
-
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -209,7 +192,7 @@ __device__ __forceinline__ bool near_tie_beta(float u, uint32_t win) {
     // UE4M3: 3 mantissa bits above 2^-6; below it (subnormal steps of 2^-9,
     // a rare range) every update takes the exact path
     return u < 0.015625f || near_half(__float_as_uint(u), 20, win);
-  } else if constexpr (F == MXFP4 || F == MXINT4) {
+  } else if constexpr (is_mx(F)) {
     return near_half(__float_as_uint(u), 23, win);      // E8M0: midpoint 1.5 * 2^k
   } else {
     return near_half(__float_as_uint(u), 16, win);      // bf16
@@ -349,7 +332,7 @@ struct RowProj {
       b = b ? b : 1u;
       r = rtab[b];
       a = atab[b];
-    } else if constexpr (F == MXFP4 || F == MXINT4) {
+    } else if constexpr (is_mx(F)) {
       uint32_t bits = __float_as_uint(u);
       int e = (int)((bits >> 23) & 0xFFu);
       int k = e ? e - 127 + ((bits & 0x7FFFFFu) >= 0x400000u ? 1 : 0)
@@ -364,34 +347,23 @@ struct RowProj {
   }
 };
 
-template <int F>
-__device__ __forceinline__ void grid8_packed(const float2* z, float2* q) {
-  if constexpr (is_int_grid(F)) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      q[k].x = rintf(fminf(fmaxf(z[k].x, -8.0f), 7.0f));
-      q[k].y = rintf(fminf(fmaxf(z[k].y, -8.0f), 7.0f));
-    }
-  } else {
-    // nearest E2M1 value of each argument (RNE, saturating): the pair's code
-    // byte goes straight back to an f16x2 of its values (exact), then to fp32
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint32_t h;
-      asm("{\n\t.reg .b8 t;\n\t"
-          "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
-          "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
-          : "=r"(h) : "f"(z[k].x), "f"(z[k].y));
-      q[k] = __half22float2(*reinterpret_cast<__half2*>(&h));
-    }
-  }
-}
-
-// Grid value of one pair of arguments (as grid8_packed).
+// Grid values of one pair of quantiser arguments: nearest grid point (ties
+// to even), saturating.  E2M1 / E4M3 pairs go through the hardware
+// conversion to their code bytes and straight back to an exact f16x2.
 template <int F>
 __device__ __forceinline__ float2 grid2_packed(float2 z) {
   if constexpr (is_int_grid(F)) {
     return make_float2(rintf(fminf(fmaxf(z.x, -8.0f), 7.0f)), rintf(fminf(fmaxf(z.y, -8.0f), 7.0f)));
+  } else if constexpr (is_int8_grid(F)) {
+    return make_float2(rintf(fminf(fmaxf(z.x, -128.0f), 127.0f)),
+                       rintf(fminf(fmaxf(z.y, -128.0f), 127.0f)));
+  } else if constexpr (F == MXFP8) {
+    uint32_t h;
+    asm("{\n\t.reg .b16 t;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 t, %2, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h) : "f"(z.x), "f"(z.y));
+    return __half22float2(*reinterpret_cast<__half2*>(&h));
   } else {
     uint32_t h;
     asm("{\n\t.reg .b8 t;\n\t"
@@ -400,6 +372,12 @@ __device__ __forceinline__ float2 grid2_packed(float2 z) {
         : "=r"(h) : "f"(z.x), "f"(z.y));
     return __half22float2(*reinterpret_cast<__half2*>(&h));
   }
+}
+
+template <int F>
+__device__ __forceinline__ void grid8_packed(const float2* z, float2* q) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) q[k] = grid2_packed<F>(z[k]);
 }
 
 template <typename WT>
@@ -947,7 +925,10 @@ static int check_solver(int f, int G, int64_t m, int64_t n) {
   switch (f) {
     case NVFP4: return solver_supported<16, WT>(m, n);
     case MXFP4:
-    case MXINT4: return solver_supported<32, WT>(m, n);
+    case MXINT4:
+    case MXINT8:
+    case MXFP8: return solver_supported<32, WT>(m, n);
+    case INT8:
     case INT4:
       if (G == 32) return solver_supported<32, WT>(m, n);
       if (G == 64) return solver_supported<64, WT>(m, n);
@@ -967,6 +948,12 @@ static int dispatch_solver(int f, int G, const SolveBatch& bt, int count, int64_
       if (G == 32) return launch_solver<INT4, 32, WT>(bt, count, m, T, o, traces, st);
       if (G == 64) return launch_solver<INT4, 64, WT>(bt, count, m, T, o, traces, st);
       return launch_solver<INT4, 128, WT>(bt, count, m, T, o, traces, st);
+    case MXINT8: return launch_solver<MXINT8, 32, WT>(bt, count, m, T, o, traces, st);
+    case MXFP8: return launch_solver<MXFP8, 32, WT>(bt, count, m, T, o, traces, st);
+    case INT8:
+      if (G == 32) return launch_solver<INT8, 32, WT>(bt, count, m, T, o, traces, st);
+      if (G == 64) return launch_solver<INT8, 64, WT>(bt, count, m, T, o, traces, st);
+      return launch_solver<INT8, 128, WT>(bt, count, m, T, o, traces, st);
   }
   return DQ_ERR_ARG;
 }

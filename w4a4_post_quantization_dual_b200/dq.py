@@ -15,8 +15,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libdq.so")
 
 DQ_INT4, DQ_MXINT4, DQ_MXFP4, DQ_NVFP4 = 0, 1, 2, 3
+DQ_INT8, DQ_MXINT8, DQ_MXFP8 = 4, 5, 6
 DQ_F32, DQ_BF16 = 0, 1
-FORMATS = {"int4": DQ_INT4, "mxint4": DQ_MXINT4, "mxfp4": DQ_MXFP4, "nvfp4": DQ_NVFP4}
+FORMATS = {"int4": DQ_INT4, "mxint4": DQ_MXINT4, "mxfp4": DQ_MXFP4, "nvfp4": DQ_NVFP4,
+           "int8": DQ_INT8, "mxint8": DQ_MXINT8, "mxfp8": DQ_MXFP8}
 STATUS = {0: "DQ_OK", 1: "DQ_ERR_ARG", 2: "DQ_ERR_UNSUPPORTED", 3: "DQ_ERR_CUDA",
           4: "DQ_ERR_DEVICE_TIMEOUT", 5: "DQ_ERR_WORKSPACE"}
 
