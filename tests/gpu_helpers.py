@@ -15,18 +15,22 @@ def to_dev(a, dtype=None):
     return t.to(DEV)
 
 
+EIGHT_BIT = (dq.DQ_INT8, dq.DQ_MXINT8, dq.DQ_MXFP8)
+BF16_SCALED = (dq.DQ_INT4, dq.DQ_INT8)
+
+
 def gpu_act(X, c, fmt, G, xdtype=torch.bfloat16):
     M, K = X.shape
     Xd = to_dev(X.astype(np.float32), xdtype)
     cd = to_dev(np.asarray(c, np.float32)) if c is not None else None
-    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=DEV)
+    codes = torch.empty((M, K if fmt in EIGHT_BIT else K // 2), dtype=torch.uint8, device=DEV)
     nbytes = dq.scales_bytes(M, K, fmt, G)
     scales = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device=DEV)  # poison padding
     st = torch.full((M,), -1.0, dtype=torch.float32, device=DEV) if fmt == dq.DQ_NVFP4 else None
     dq.dq_quantize_act(Xd, fmt, cd, codes, scales, st, group=G)
     torch.cuda.synchronize()
     sc = scales.cpu().numpy()
-    if fmt == dq.DQ_INT4:
+    if fmt in BF16_SCALED:
         sc = sc.view(np.uint16).reshape(M, K // G)
     return codes.cpu().numpy(), sc, (st.cpu().numpy() if st is not None else None)
 
@@ -34,14 +38,14 @@ def gpu_act(X, c, fmt, G, xdtype=torch.bfloat16):
 def gpu_pack(W, r, c, sT, fmt, G, wdtype=torch.bfloat16):
     m, n = W.shape
     Wd = to_dev(W.astype(np.float32), wdtype)
-    codes = torch.empty((m, n // 2), dtype=torch.uint8, device=DEV)
+    codes = torch.empty((m, n if fmt in EIGHT_BIT else n // 2), dtype=torch.uint8, device=DEV)
     scales = torch.full((dq.scales_bytes(m, n, fmt, G),), 0xAB, dtype=torch.uint8, device=DEV)
     sTd = to_dev(np.array([sT], np.float32))
     dq.dq_quantize_weight(Wd, fmt, to_dev(np.asarray(r, np.float32)),
                           to_dev(np.asarray(c, np.float32)), sTd, codes, scales, group=G)
     torch.cuda.synchronize()
     sc = scales.cpu().numpy()
-    if fmt == dq.DQ_INT4:
+    if fmt in BF16_SCALED:
         sc = sc.view(np.uint16).reshape(m, n // G)
     return codes.cpu().numpy(), sc
 

@@ -73,7 +73,7 @@ inline bool valid_group(int f, int G) {
   return false;
 }
 
-// 8-bit variants: the solver only, so far
+// 8-bit variants: no tensor-core linear yet
 inline bool is_8bit(int f) { return f == DQ_INT8 || f == DQ_MXINT8 || f == DQ_MXFP8; }
 
 inline int resolve_group(int f, int group) { return group > 0 ? group : dq_native_group((dq_format)f); }
@@ -176,7 +176,6 @@ int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format 
 int dq_quantize_weight(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f, int group,
                        const float* r, const float* c, const float* s_tensor, uint8_t* codes,
                        void* scales, void* stream) {
-  if (is_8bit(f)) return DQ_ERR_UNSUPPORTED;
   const int G = resolve_group(f, group);
   if (!W || !r || !c || !codes || !scales || m <= 0 || n <= 0 || !valid_dtype(wt) ||
       !valid_group(f, G) || n % G || !aligned(W, 16) || !aligned(codes, 16) ||
@@ -189,11 +188,11 @@ int dq_quantize_weight(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_form
 int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, const float* c,
                     dq_format f, int group, uint8_t* codes, void* scales, float* s_tok,
                     void* stream) {
-  if (is_8bit(f)) return DQ_ERR_UNSUPPORTED;
   const int G = resolve_group(f, group);
   if (!X || !codes || !scales || M <= 0 || K <= 0 || !valid_dtype(xt) || !valid_group(f, G) ||
       K % G || !aligned(X, 16) || !aligned(codes, 16) || !aligned(scales, 16) ||
-      (f == DQ_NVFP4 && !s_tok) || (f != DQ_INT4 && K % (4 * G)) || K / G > 4096)
+      (f == DQ_NVFP4 && !s_tok) || (f != DQ_INT4 && f != DQ_INT8 && K % (4 * G)) ||
+      K / G > 4096)
     return DQ_ERR_ARG;
   return dq::quantize_act(X, xt, M, K, c, f, G, codes, scales, s_tok, (cudaStream_t)stream);
 }
@@ -201,10 +200,10 @@ int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, const floa
 int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, const float* c,
                        dq_format f, int group, const uint8_t* codes, const void* scales,
                        const float* s_tok, double* sums, void* stream) {
-  if (is_8bit(f)) return DQ_ERR_UNSUPPORTED;
   const int G = resolve_group(f, group);
   if (!X || !codes || !scales || !sums || M <= 0 || K <= 0 || !valid_dtype(xt) ||
-      !valid_group(f, G) || K % G || K % 8 || !aligned(X, 16) || !aligned(codes, 4) ||
+      !valid_group(f, G) || K % G || K % 8 || !aligned(X, 16) ||
+      !aligned(codes, is_8bit(f) ? 8 : 4) ||
       !aligned(scales, 2) || !aligned(sums, 8) || !aligned(c, 4) || (f == DQ_NVFP4 && !s_tok))
     return DQ_ERR_ARG;
   return dq::act_quant_error(X, xt, M, K, c, f, G, codes, scales, s_tok, sums,

@@ -42,10 +42,17 @@ act_error_kernel(const XT* __restrict__ X, int64_t M, int64_t K, const float* __
       x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
       x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
     }
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + row * (K / 2) + col / 2);
+    uint32_t w = 0, w2 = 0;   // 8-bit formats: eight bytes in w (0-3), w2 (4-7)
+    if constexpr (is_8bit(F)) {
+      const uint2 v = *reinterpret_cast<const uint2*>(codes + row * K + col);
+      w = v.x;
+      w2 = v.y;
+    } else {
+      w = *reinterpret_cast<const uint32_t*>(codes + row * (K / 2) + col / 2);
+    }
     const int64_t s = col / G;
     double scale;
-    if constexpr (F == INT4) {
+    if constexpr (F == INT4 || F == INT8) {
       const uint16_t h = reinterpret_cast<const uint16_t*>(scales)[row * S + s];
       scale = (double)__uint_as_float((uint32_t)h << 16);
     } else {
@@ -55,8 +62,19 @@ act_error_kernel(const XT* __restrict__ X, int64_t M, int64_t K, const float* __
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const uint32_t code = (w >> (4 * k)) & 0xFu;
-      const double q = is_int_grid(F) ? (double)((int)(code << 28) >> 28) : e2m1_value_f64(code);
+      double q;
+      if constexpr (is_8bit(F)) {
+        const uint32_t code = ((k < 4 ? w : w2) >> (8 * (k & 3))) & 0xFFu;
+        if constexpr (F == MXFP8) {
+          const float mag = ue4m3_value(code & 0x7Fu);
+          q = (code & 0x80u) ? -(double)mag : (double)mag;
+        } else {
+          q = (double)((int)(code << 24) >> 24);
+        }
+      } else {
+        const uint32_t code = (w >> (4 * k)) & 0xFu;
+        q = is_int_grid(F) ? (double)((int)(code << 28) >> 28) : e2m1_value_f64(code);
+      }
       double xh = q * scale;
       if (c != nullptr) xh = xh / (double)c[col + k];
       const double xv = (double)x[k], e = xv - xh;
@@ -107,6 +125,12 @@ int act_quant_error(const void* X, int xt, int64_t M, int64_t K, const float* c,
       if (G == 32) return launch_error<INT4, 32>(X, xt, M, K, c, codes, scales, s_tok, sums, st);
       if (G == 64) return launch_error<INT4, 64>(X, xt, M, K, c, codes, scales, s_tok, sums, st);
       return launch_error<INT4, 128>(X, xt, M, K, c, codes, scales, s_tok, sums, st);
+    case MXINT8: return launch_error<MXINT8, 32>(X, xt, M, K, c, codes, scales, s_tok, sums, st);
+    case MXFP8: return launch_error<MXFP8, 32>(X, xt, M, K, c, codes, scales, s_tok, sums, st);
+    case INT8:
+      if (G == 32) return launch_error<INT8, 32>(X, xt, M, K, c, codes, scales, s_tok, sums, st);
+      if (G == 64) return launch_error<INT8, 64>(X, xt, M, K, c, codes, scales, s_tok, sums, st);
+      return launch_error<INT8, 128>(X, xt, M, K, c, codes, scales, s_tok, sums, st);
   }
   return DQ_ERR_ARG;
 }

@@ -50,6 +50,35 @@ __device__ __forceinline__ void load_block_smem(const XT* p, float* x) {
   }
 }
 
+// 8-bit codes of G grid arguments z -> G bytes written to dst (16-byte
+// aligned): INT8 two's-complement bytes (nearest even, clipped), FP8 E4M3
+// bytes (nearest even, saturating).
+template <int F, int G>
+__device__ __forceinline__ void store_codes8(uint8_t* dst, const float* z) {
+  uint32_t w[G / 4];
+#pragma unroll
+  for (int u = 0; u < G / 4; ++u) {
+    if constexpr (F == MXFP8) {
+      uint16_t lo, hi;   // element 2k in the low byte of each pair
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(lo) : "f"(z[4 * u]), "f"(z[4 * u + 1]));
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(hi)
+          : "f"(z[4 * u + 2]), "f"(z[4 * u + 3]));
+      w[u] = (uint32_t)lo | ((uint32_t)hi << 16);
+    } else {
+      uint32_t v = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int q = (int)rintf(fminf(fmaxf(z[4 * u + k], -128.0f), 127.0f));
+        v |= ((uint32_t)q & 0xFFu) << (8 * k);
+      }
+      w[u] = v;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < G / 16; ++u)
+    reinterpret_cast<uint4*>(dst)[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+}
+
 // Codes of G grid arguments z -> G/2 bytes written to dst (16-byte aligned for G >= 32).
 template <int F, int G>
 __device__ __forceinline__ void store_codes(uint8_t* dst, const float* z) {
@@ -89,7 +118,7 @@ quantize_act_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int64_t K
   const int64_t S = K / G;
   for (int64_t t = blockIdx.x; t < Mpad; t += gridDim.x) {
     if (t >= M) {  // padding rows of the tensor-core scale layout
-      if constexpr (F != INT4) {
+      if constexpr (F != INT4 && F != INT8) {
         for (int j = 0; j < BPT; ++j) {
           int64_t s = tid + (int64_t)j * NT;
           if (s < S) scales[sf_offset(t, s, S)] = 0;
@@ -146,10 +175,10 @@ quantize_act_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int64_t K
         float sblk = __fmul_rn(ue4m3_value(byte), st);
         zero = (sblk == 0.0f);
         inv = zero ? 0.0f : __frcp_rn(sblk);
-      } else if constexpr (F == MXFP4 || F == MXINT4) {
+      } else if constexpr (is_mx(F)) {
         int e = -127;
         if (ab[j] > 0.0f) {
-          e = ilog2f(ab[j]) - 2;
+          e = ilog2f(ab[j]) - mx_emax(F);
           e = e < -127 ? -127 : (e > 127 ? 127 : e);
         } else {
           zero = true;
@@ -157,7 +186,7 @@ quantize_act_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int64_t K
         scales[sf_offset(t, s, S)] = (uint8_t)(e + 127);
         inv = pow2f(-e);
       } else {
-        __nv_bfloat16 h = __float2bfloat16_rn(__fdiv_rn(ab[j], 7.0f));
+        __nv_bfloat16 h = __float2bfloat16_rn(__fdiv_rn(ab[j], F == INT8 ? 127.0f : 7.0f));
         reinterpret_cast<__nv_bfloat16*>(scales)[t * S + s] = h;
         float sc = __bfloat162float(h);
         zero = (sc == 0.0f);
@@ -166,7 +195,8 @@ quantize_act_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int64_t K
       float z[G];
 #pragma unroll
       for (int k = 0; k < G; ++k) z[k] = zero ? 0.0f : __fmul_rn(xt[j][k], inv);
-      store_codes<F, G>(codes + t * (K / 2) + s * (G / 2), z);
+      if constexpr (is_8bit(F)) store_codes8<F, G>(codes + t * K + s * G, z);
+      else store_codes<F, G>(codes + t * (K / 2) + s * (G / 2), z);
     }
   }
 }
@@ -667,10 +697,11 @@ pack_weight_kernel(const WT* __restrict__ W, int64_t m, int64_t n, const float* 
 #pragma unroll
   for (int k = 0; k < G; ++k)
     z[k] = __fmul_rn(__fmul_rn(x[k], __frcp_rn(__ldg(c + b * G + k))), alpha);
-  store_codes<F, G>(codes + i * (n / 2) + b * (G / 2), z);
+  if constexpr (is_8bit(F)) store_codes8<F, G>(codes + i * n + b * G, z);
+  else store_codes<F, G>(codes + i * (n / 2) + b * (G / 2), z);
   if constexpr (F == NVFP4) {
     scales[sf_offset(i, b, nb)] = (uint8_t)ue4m3_rn(__fdiv_rn(rr, *sTp));
-  } else if constexpr (F == MXFP4 || F == MXINT4) {
+  } else if constexpr (is_mx(F)) {
     uint32_t e = (__float_as_uint(rr) >> 23) & 0xFFu;  // exponent of a power of two
     scales[sf_offset(i, b, nb)] = (uint8_t)(e > 254u ? 254u : e);
   } else {
@@ -706,9 +737,9 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
   const int64_t S = K / G;
   int NT = (int)((S < 1024 ? S : 1024) + 31) / 32 * 32;
   const int bpt = (int)((S + NT - 1) / NT);
-  const int64_t Mpad = (F == INT4) ? M : ((M + 127) / 128) * 128;
+  const int64_t Mpad = (F == INT4 || F == INT8) ? M : ((M + 127) / 128) * 128;
   const XT* Xp = reinterpret_cast<const XT*>(X);
-  if constexpr (F != INT4) {
+  if constexpr (F != INT4 && !is_8bit(F)) {
     if constexpr (sizeof(XT) == 2) {
       // ring kernel: NTS threads per row, BPT blocks per thread, at most MAXT
       // threads and MINB CTAs per SM (the register budget of each variant)
@@ -819,6 +850,12 @@ int quantize_act(const void* X, int xt, int64_t M, int64_t K, const float* c, in
       if (G == 32) { DQ_ACT(INT4, 32); }
       if (G == 64) { DQ_ACT(INT4, 64); }
       DQ_ACT(INT4, 128);
+    case MXINT8: DQ_ACT(MXINT8, 32);
+    case MXFP8: DQ_ACT(MXFP8, 32);
+    case INT8:
+      if (G == 32) { DQ_ACT(INT8, 32); }
+      if (G == 64) { DQ_ACT(INT8, 64); }
+      DQ_ACT(INT8, 128);
   }
 #undef DQ_ACT
   return DQ_ERR_ARG;
@@ -828,7 +865,7 @@ template <int F, int G, typename WT>
 static int launch_pack(const void* W, int64_t m, int64_t n, const float* r, const float* c,
                        const float* sT, uint8_t* codes, uint8_t* scales, cudaStream_t st) {
   const int64_t nb = n / G;
-  if (F != INT4) {
+  if (F != INT4 && F != INT8) {
     // padding rows / scale columns of the tensor-core layout are zeroed first
     int64_t bytes = (int64_t)(((m + 127) / 128) * ((nb + 3) / 4) * 512);
     if ((m & 127) || (nb & 3)) {
@@ -857,6 +894,12 @@ int quantize_weight(const void* W, int wt, int64_t m, int64_t n, int f, int G, c
       if (G == 32) { DQ_PACK(INT4, 32); }
       if (G == 64) { DQ_PACK(INT4, 64); }
       DQ_PACK(INT4, 128);
+    case MXINT8: DQ_PACK(MXINT8, 32);
+    case MXFP8: DQ_PACK(MXFP8, 32);
+    case INT8:
+      if (G == 32) { DQ_PACK(INT8, 32); }
+      if (G == 64) { DQ_PACK(INT8, 64); }
+      DQ_PACK(INT8, 128);
   }
 #undef DQ_PACK
   return DQ_ERR_ARG;
