@@ -73,7 +73,8 @@ inline bool valid_group(int f, int G) {
   return false;
 }
 
-// 8-bit variants: no tensor-core linear yet
+// 8-bit variants (MXFP8 has a tensor-core linear; INT8 / MXINT8 do not:
+// sm_100a's block-scaled MMA takes FP8/FP6/FP4 operands only)
 inline bool is_8bit(int f) { return f == DQ_INT8 || f == DQ_MXINT8 || f == DQ_MXFP8; }
 
 inline int resolve_group(int f, int group) { return group > 0 ? group : dq_native_group((dq_format)f); }
@@ -213,9 +214,9 @@ int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, const f
 int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                    const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                    dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream) {
-  if (is_8bit(f)) return DQ_ERR_UNSUPPORTED;
+  if (f == DQ_INT8 || f == DQ_MXINT8) return DQ_ERR_UNSUPPORTED;
   if (f == DQ_INT4) return DQ_ERR_UNSUPPORTED;
-  if (f != DQ_NVFP4 && f != DQ_MXFP4 && f != DQ_MXINT4) return DQ_ERR_ARG;
+  if (f != DQ_NVFP4 && f != DQ_MXFP4 && f != DQ_MXINT4 && f != DQ_MXFP8) return DQ_ERR_ARG;
   if (!A || !sA || !B || !sB || !Y || M <= 0 || N <= 0 || K <= 0 || !valid_dtype(yt) ||
       N % 128 || K % 256 || !aligned(A, 16) || !aligned(B, 16) || !aligned(sA, 16) ||
       !aligned(sB, 16) || !aligned(Y, 16) || (f == DQ_NVFP4 && !s_tok) ||

@@ -1207,7 +1207,9 @@ __device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t
 }
 }  // namespace i4
 
-template <int YT>
+// FP8: MXFP8 operands (E4M3 codes in global memory): TMA places them
+// straight into the swizzled operand tiles and the converter warps idle.
+template <int YT, bool FP8>
 __global__ void __launch_bounds__(i4::THREADS, 1)
 w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const uint8_t* __restrict__ sfA,
@@ -1270,9 +1272,15 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
         const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(&full[stage], STG_A + STG_B + SF_A + SF_B);
-          tma_load_2d(stA + stage * STG_A, &tmA, &full[stage], kt * (BKE / 2), m0);
-          tma_load_2d(stB + stage * STG_B, &tmB, &full[stage], kt * (BKE / 2), n0);
+          if constexpr (FP8) {
+            mbar_expect_tx(&full[stage], OP_A + OP_B + SF_A + SF_B);
+            tma_load_2d(opA + stage * OP_A, &tmA, &full[stage], kt * BKE, m0);
+            tma_load_2d(opB + stage * OP_B, &tmB, &full[stage], kt * BKE, n0);
+          } else {
+            mbar_expect_tx(&full[stage], STG_A + STG_B + SF_A + SF_B);
+            tma_load_2d(stA + stage * STG_A, &tmA, &full[stage], kt * (BKE / 2), m0);
+            tma_load_2d(stB + stage * STG_B, &tmB, &full[stage], kt * (BKE / 2), n0);
+          }
           bulk_load(sSFA + stage * SF_A, sfA + ((size_t)(m0 / 128) * S4 + kt) * 512, SF_A,
                     &full[stage]);
           bulk_load(sSFB + stage * SF_B, sfB + ((size_t)(n0 / 128) * S4 + kt) * 512, SF_B,
@@ -1297,7 +1305,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
         if (!mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag)) break;
         fence_after_sync();
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&conv[stage], phase, abort_flag) ||
+          if (!mbar_wait(FP8 ? &full[stage] : &conv[stage], phase, abort_flag) ||
               !mbar_wait(&sfready[stage], phase, abort_flag)) { ok = false; break; }
           fence_after_sync();
           const uint32_t a_base = smem_u32(opA + stage * OP_A);
@@ -1338,6 +1346,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
   } else if (warp >= 7) {
+    if constexpr (!FP8) {
     // converters: packed INT4 staging -> swizzled E4M3 operand tiles
     const int ct = threadIdx.x - 7 * 32;        // 0..127
     int stage = 0;
@@ -1369,6 +1378,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
         if (lane == 0) mbar_arrive(&conv[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
+    }
     }
   } else {
     // epilogue (warps 2..5)
@@ -1663,14 +1673,18 @@ static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, con
   return launch<FMT, 128, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
 }
 
-template <int YT>
+// FP8: MXFP8 codes (one byte per element, 128-byte swizzled TMA boxes);
+// otherwise packed MXINT4 codes (64-byte boxes into the staging buffers).
+template <int YT, bool FP8>
 static int launch_mxint4(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB,
                          const float* r_row, void* Y, int64_t M, int64_t N, int64_t K,
                          cudaStream_t st) {
   CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K / 2, BM, i4::BKE / 2) || !make_map(&tb, B, N, K / 2, i4::BN, i4::BKE / 2))
+  const int64_t kb = FP8 ? K : K / 2;
+  const int box = FP8 ? i4::BKE : i4::BKE / 2;
+  if (!make_map(&ta, A, M, kb, BM, box) || !make_map(&tb, B, N, kb, i4::BN, box))
     return DQ_ERR_CUDA;
-  auto kern = w4a4_gemm_mxint4_kernel<YT>;
+  auto kern = w4a4_gemm_mxint4_kernel<YT, FP8>;
   if (!ensure_kernel_attrs((const void*)kern, i4::SMEM, false)) return DQ_ERR_CUDA;
   const int64_t tiles = ((M + BM - 1) / BM) * (N / i4::BN);
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
@@ -1691,8 +1705,11 @@ int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const u
     return yt == 1 ? gemm::dispatch<MXFP4, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
                    : gemm::dispatch<MXFP4, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
   if (f == MXINT4)
-    return yt == 1 ? gemm::launch_mxint4<1>(A, sA, B, sB, r_row, Y, M, N, K, st)
-                   : gemm::launch_mxint4<0>(A, sA, B, sB, r_row, Y, M, N, K, st);
+    return yt == 1 ? gemm::launch_mxint4<1, false>(A, sA, B, sB, r_row, Y, M, N, K, st)
+                   : gemm::launch_mxint4<0, false>(A, sA, B, sB, r_row, Y, M, N, K, st);
+  if (f == MXFP8)
+    return yt == 1 ? gemm::launch_mxint4<1, true>(A, sA, B, sB, r_row, Y, M, N, K, st)
+                   : gemm::launch_mxint4<0, true>(A, sA, B, sB, r_row, Y, M, N, K, st);
   return DQ_ERR_UNSUPPORTED;
 }
 

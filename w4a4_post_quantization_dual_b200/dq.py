@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_HERE, "lib", "libdq.so")
 
 DQ_INT4, DQ_MXINT4, DQ_MXFP4, DQ_NVFP4 = 0, 1, 2, 3
 DQ_INT8, DQ_MXINT8, DQ_MXFP8 = 4, 5, 6
+EIGHT_BIT = (DQ_INT8, DQ_MXINT8, DQ_MXFP8)
 DQ_F32, DQ_BF16 = 0, 1
 FORMATS = {"int4": DQ_INT4, "mxint4": DQ_MXINT4, "mxfp4": DQ_MXFP4, "nvfp4": DQ_NVFP4,
            "int8": DQ_INT8, "mxint8": DQ_MXINT8, "mxfp8": DQ_MXFP8}
@@ -193,10 +194,11 @@ def dq_quantize_act(X, fmt, c, codes, scales, s_tok=None, group=0, stream=None):
 
 
 def dq_w4a4_linear(A, sA, s_tok, B, sB, s_w, Y, fmt, r_row=None, stream=None):
-    M, K2 = A.shape
+    M, KB = A.shape                 # code bytes per row: K/2 (4-bit) or K (8-bit)
     N = B.shape[0]
+    K = KB if _fmt(fmt) in (DQ_INT8, DQ_MXINT8, DQ_MXFP8) else 2 * KB
     _check(lib().dq_w4a4_linear(_ptr(A), _ptr(sA), _ptr(s_tok), _ptr(B), _ptr(sB), _ptr(s_w),
-                                _ptr(r_row), _ptr(Y), _dtype(Y), M, N, 2 * K2, _fmt(fmt),
+                                _ptr(r_row), _ptr(Y), _dtype(Y), M, N, K, _fmt(fmt),
                                 _stream(stream)),
            "dq_w4a4_linear")
 
@@ -238,7 +240,8 @@ def quantize_linear(W, fmt, T, group=0, mse_trace=False):
     tr = torch.empty(T + 1, dtype=torch.float64, device=dev) if mse_trace else None
     ws = torch.empty(solve_workspace_size(T), dtype=torch.uint8, device=dev)
     dq_solve_scales(W, fmt, T, r, c, sT, tr, ws, group=G)
-    codes = torch.empty((m, n // 2), dtype=torch.uint8, device=dev)
+    codes = torch.empty((m, n if _fmt(fmt) in EIGHT_BIT else n // 2), dtype=torch.uint8,
+                        device=dev)
     scales = torch.empty(scales_bytes(m, n, fmt, G), dtype=torch.uint8, device=dev)
     dq_quantize_weight(W, fmt, r, c, sT, codes, scales, group=G)
     return QuantizedLinear(codes, scales, c, sT, fmt, G, (m, n)), r, tr
@@ -251,7 +254,8 @@ def act_sqnr_db(X, fmt, c=None, group=0):
     M, K = X.shape
     dev = X.device
     G = group or native_group(fmt)
-    A = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    A = torch.empty((M, K if _fmt(fmt) in EIGHT_BIT else K // 2), dtype=torch.uint8,
+                    device=dev)
     sA = torch.empty(scales_bytes(M, K, fmt, G), dtype=torch.uint8, device=dev)
     st = torch.empty(M, dtype=torch.float32, device=dev) if _fmt(fmt) == DQ_NVFP4 else None
     sums = torch.empty(2, dtype=torch.float64, device=dev)
@@ -265,7 +269,7 @@ def linear(X, q: QuantizedLinear, out_dtype=torch.bfloat16, r_row=None):
     """Y = X W^T through the W4A4 path: fused rescale+quantise, block-scaled GEMM."""
     M, K = X.shape
     dev = X.device
-    A = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    A = torch.empty((M, K if q.fmt in EIGHT_BIT else K // 2), dtype=torch.uint8, device=dev)
     sA = torch.empty(scales_bytes(M, K, q.fmt, q.group), dtype=torch.uint8, device=dev)
     st = torch.empty(M, dtype=torch.float32, device=dev) if q.fmt == DQ_NVFP4 else None
     dq_quantize_act(X, q.fmt, q.c, A, sA, st, group=q.group)
