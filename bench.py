@@ -470,6 +470,49 @@ def run_ours(args, rank, world, local_rank):
     # scaling); the time is the slowest rank's
     value = world * lin_flops * args.steps / (lin_ms * 1e-3) / 1e12
 
+    # 8-bit variant (Appendix G.2): the MXFP8 linear on the largest weight at
+    # the prefill shape -- solve, pack, then the activation quantiser and the
+    # GEMM timed like the others.  Auxiliary: an error is reported, not raised.
+    mxfp8 = None
+    try:
+        Wm = Wd[j0]
+        N8, K8 = Wm.shape
+        r8 = torch.empty((N8, K8 // 32), device=dev)
+        c8 = torch.empty(K8, device=dev)
+        s8 = torch.empty(1, device=dev)
+        dq.dq_solve_scales(Wm, dq.DQ_MXFP8, T, r8, c8, s8, None, ws, group=32)
+        B8 = torch.empty((N8, K8), dtype=torch.uint8, device=dev)
+        sB8 = torch.empty(dq.scales_bytes(N8, K8, dq.DQ_MXFP8, 32), dtype=torch.uint8, device=dev)
+        dq.dq_quantize_weight(Wm, dq.DQ_MXFP8, r8, c8, s8, B8, sB8, group=32)
+        X8 = Xd[prefill_M]
+        A8 = torch.empty((prefill_M, K8), dtype=torch.uint8, device=dev)
+        sA8 = torch.empty(dq.scales_bytes(prefill_M, K8, dq.DQ_MXFP8, 32), dtype=torch.uint8,
+                          device=dev)
+        Y8 = torch.empty((prefill_M, N8), dtype=torch.bfloat16, device=dev)
+        nx8 = max(2, min(16, -(-2 * L2_BYTES // (X8.numel() * 2))))
+        Xc8 = [X8.clone() for _ in range(nx8)]
+        t_act8 = per_launch_us(lambda i: dq.dq_quantize_act(
+            Xc8[i % nx8], dq.DQ_MXFP8, c8, A8, sA8, None, group=32), nx8)
+        nb8 = max(2, min(64, -(-2 * L2_BYTES // (B8.numel() + sB8.numel()))))
+        Bc8 = [(B8.clone(), sB8.clone()) for _ in range(nb8)]
+        t_gemm8 = per_launch_us(lambda i: dq.dq_w4a4_linear(
+            A8, sA8, None, Bc8[i][0], Bc8[i][1], None, Y8, dq.DQ_MXFP8), nb8)
+        err8 = dq.dq_device_error(clear=True)
+        fl8 = 2.0 * prefill_M * N8 * K8 / (t_gemm8 * 1e-6) / 1e12
+        a8_bytes = prefill_M * K8 * (2 + 1 + 1.0 / 32)
+        mxfp8 = {"shape": f"M={prefill_M} x N={N8} x K={K8}", "T": T,
+                 "gemm": {"kernel": "w4a4_gemm_mxint4_kernel<FP8>", "us_per_launch": t_gemm8,
+                          "achieved": fl8, "peak": 2.0 * bf16_tf, "unit": "TFLOP/s",
+                          "frac": fl8 / (2.0 * bf16_tf),
+                          "peak_kind": f"{peak_kind} bf16 burst x 2 (nominal fp8:bf16)"},
+                 "act_quant": {"us_per_launch": t_act8, "achieved": a8_bytes / (t_act8 * 1e-6) / 1e9,
+                               "peak": hbm, "unit": "GB/s",
+                               "frac": a8_bytes / (t_act8 * 1e-6) / 1e9 / hbm},
+                 "device_error": err8}
+        del Xc8, Bc8
+    except Exception as ex:  # auxiliary measurement: report, do not fail the bench line
+        mxfp8 = {"error": str(ex)[:300]}
+
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         oracle_prepare(wl, Ws)
@@ -529,6 +572,7 @@ def run_ours(args, rank, world, local_rank):
                            "weights": "q, k, v, o 4096/1024 x 4096; gate, up 14336 x 4096; "
                                       "down 4096 x 14336 (one Llama-3.1-8B layer)",
                            "launches": {"separate": 14, "batched": 6}},
+        "mxfp8": mxfp8,
         "act_sqnr": {"per_weight": act_sqnr, "rows": prefill_M,
                      "note": "SQNR of the dequantised activations mapped back by 1/c vs X, "
                              "measured on the device (dq_act_quant_error); synthetic "
