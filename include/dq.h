@@ -21,15 +21,17 @@
  *  - 4-bit codes are packed two per byte, element 2k in the low nibble of
  *    byte k.  E2M1 codes: bit 3 sign, bits 0-2 magnitude index of
  *    {0, .5, 1, 1.5, 2, 3, 4, 6}.  INT4 / MXINT4 codes: two's complement
- *    nibble, values -8..7.
- *  - Block scales for NVFP4 / MXFP4 / MXINT4 operands are one byte per
+ *    nibble, values -8..7.  8-bit codes are one byte per element: INT8 /
+ *    MXINT8 two's complement (-128..127), MXFP8 FP8 E4M3 (OCP), rows K
+ *    bytes long.
+ *  - Block scales for NVFP4 and the MX formats are one byte per
  *    (row, block) (UE4M3 for NVFP4, E8M0 for MX) stored in the layout the
  *    block-scaled tensor-core MMA reads: 512-byte atoms of 128 rows x 4
  *    scales, atoms ordered row-block-major then along K; inside an atom the
  *    scale (row, s) sits at byte (row%32)*16 + ((row%128)/32)*4 + s%4.
  *    Rows are padded to a multiple of 128 and scale columns to a multiple
- *    of 4; dq_scales_bytes() gives the size.  INT4 block scales are bf16,
- *    row-major rows x (k/G).
+ *    of 4; dq_scales_bytes() gives the size.  INT4 and INT8 block scales
+ *    are bf16, row-major rows x (k/G).
  *  - Inputs must be finite.  For NVFP4 and INT4 activations a row (NVFP4)
  *    or block (INT4) whose absmax is below about 1e-30 is outside the
  *    supported range: its fp32 reciprocal block scale overflows.  Arguments are validated before any launch; a
@@ -179,7 +181,7 @@ DQ_API int dq_solve_scales_ex(const void* W, dq_dtype wt, int64_t m, int64_t n, 
  *           s_tensor * UE4M3 for NVFP4, a bf16 value for INT4).
  *  s_tensor device pointer to the NVFP4 per-tensor scale (ignored, may be
  *           NULL, for other formats).
- *  codes    out, m x n/2 bytes.
+ *  codes    out, m x n/2 bytes (m x n for the 8-bit formats).
  *  scales   out, dq_scales_bytes(m, n, f, G) bytes: the row-block scales
  *           encoded (UE4M3 of r/s_tensor, E8M0 exponent of r, bf16 of r).
  * Element code = grid(fl(fl(W_ij * fl(1/c_j)) * fl(1/r_ib))), round to
@@ -197,7 +199,7 @@ DQ_API int dq_quantize_weight(const void* W, dq_dtype wt, int64_t m, int64_t n, 
  *
  *  X        M x K (dtype xt: DQ_BF16 or DQ_F32); K % G == 0.
  *  c        K fp32 column scales (NULL = all ones).
- *  codes    out, M x K/2 bytes.
+ *  codes    out, M x K/2 bytes (M x K for the 8-bit formats).
  *  scales   out, dq_scales_bytes(M, K, f, G) bytes; padding rows of the
  *           tensor-core layout are written as zero.
  *  s_tok    out, M fp32 (NVFP4 only, else may be NULL): per-token scale
@@ -222,7 +224,8 @@ DQ_API int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, con
  * (Section 4.4: "Q(X~) What^T Diag(alpha)^-1"):
  *   Y[t, o] = s_tok[t] * s_w * r_row[o] * sum_k a[t,k] sa[t,k/G] b[o,k] sb[o,k/G]
  *
- *  A, sA    activation codes (M x K/2) and scales from dq_quantize_act.
+ *  A, sA    activation codes (M x K/2; M x K for MXFP8) and scales from
+ *           dq_quantize_act.
  *  s_tok    M fp32 per-token scales (NVFP4; ignored for MX, may be NULL).
  *  B, sB    weight codes (N x K/2) and scales from dq_quantize_weight.
  *  s_w      device pointer to the weight's per-tensor scale (NVFP4; may be
