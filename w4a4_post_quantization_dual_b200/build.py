@@ -52,7 +52,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     os.makedirs(LIB_DIR, exist_ok=True)
     obj_dir = os.path.join(HERE, "_build")
     os.makedirs(obj_dir, exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     for src in _sources():
         obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
         cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-c", src,
@@ -60,8 +60,13 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
         objs.append(obj)
+    # the translation units are independent: compile them side by side
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as pool:
+        for res in pool.map(lambda c: subprocess.run(c, check=True), cmds):
+            del res
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.run([_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
                     "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-lcudart"], check=True)
