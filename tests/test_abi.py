@@ -80,6 +80,14 @@ def test_invalid_arguments_rejected_without_launch(L):
                                      two, None, ws, 4096, None) == 1
     assert L.dq_solve_scales_batched(2, two, 1, i64(64, 64), i64(64, 64), 3, 16, 5, 0, two, two,
                                      two, None, ws, 100, None) == 5
+    # 8-bit formats: INT8 has no tensor-core linear; MXFP8 follows the MX shape rules
+    assert L.dq_w4a4_linear(fake, fake, fake, fake, fake, fake, None, fake, 1, 16, 128, 256,
+                            4, None) == 2
+    assert L.dq_w4a4_linear(fake, fake, None, fake, fake, None, None, fake, 1, 16, 100, 256,
+                            6, None) == 1
+    assert L.dq_scales_bytes(10, 256, 4, 128) == 10 * 2 * 2          # INT8: bf16 row-major
+    assert L.dq_scales_bytes(130, 256, 6, 32) == 2 * 2 * 512          # MXFP8: padded atoms
+    assert [L.dq_native_group(f) for f in (4, 5, 6)] == [128, 32, 32]
     # more column blocks than one launch grid holds: refused before anything is enqueued
     wide = 16 * 65536
     assert L.dq_solve_scales(fake, 1, 64, wide, 3, 16, 5, fake, fake, fake, None, ws, 4096,
