@@ -72,6 +72,9 @@ def lib():
             "oracle_solve_ex": (None, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_int, _f32p, _f32p, _i64p, _i64,
                                        _f32p, _f32p, _f32p, _f64p, _f64p]),
+            "oracle_solve_qtrace": (None, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, _f32p, _f32p, _i64p, _i64,
+                                           _f32p, _f32p, _f32p, _f64p, _f64p, _f64p, _f64p]),
             "oracle_error": (ctypes.c_double, [_f32p, _i64, _i64, ctypes.c_int, ctypes.c_int,
                                                _f32p, _f32p]),
             "oracle_error_fixed_q": (ctypes.c_double, [_f32p, _u8p, _i64, _i64, ctypes.c_int,
@@ -266,6 +269,36 @@ def solve_ex(W, fmt, G, T, flags=0, r0=None, c0=None, s_T=None, tiles=None):
                           _p(w2, _f64p))
     trace = err / w2[0] if w2[0] > 0 else err
     return {"r": r, "c": c, "s_T": float(sT[0]), "trace": trace, "err": err, "w2": float(w2[0])}
+
+
+def solve_qtrace(W, fmt, G, T, flags=0, tiles=None):
+    """solve_ex plus the relative code change of Fig. 2(a) / Fig. 3(a):
+    result["qchange"][t] = ||Qhat(t) - Qhat(t-1)||_F / ||Qhat(t-1)||_F for
+    t = 1..T (entry 0 is nan), Qhat(t) the code values at the scales after
+    round t, over the solved tiles."""
+    W = _f32(W)
+    m, n = W.shape
+    nb = n // G
+    r = np.empty((m, nb), np.float32)
+    c = np.empty(n, np.float32)
+    sT = np.zeros(1, np.float32)
+    err = np.zeros(T + 1, np.float64)
+    w2 = np.zeros(1, np.float64)
+    qn = np.zeros(T + 1, np.float64)
+    qd = np.zeros(T + 1, np.float64)
+    if tiles is None:
+        tp, nt = None, 0
+    else:
+        tarr = np.ascontiguousarray(tiles, dtype=np.int64)
+        tp, nt = _p(tarr, _i64p), len(tarr)
+    lib().oracle_solve_qtrace(_p(W, _f32p), m, n, fmt, G, T, flags, None, None, tp, nt,
+                              _p(r, _f32p), _p(c, _f32p), _p(sT, _f32p), _p(err, _f64p),
+                              _p(w2, _f64p), _p(qn, _f64p), _p(qd, _f64p))
+    qc = np.full(T + 1, np.nan)
+    qc[1:] = np.sqrt(qn[1:] / np.where(qd[1:] > 0, qd[1:], np.nan))
+    trace = err / w2[0] if w2[0] > 0 else err
+    return {"r": r, "c": c, "s_T": float(sT[0]), "trace": trace, "err": err, "w2": float(w2[0]),
+            "qchange": qc}
 
 
 def error(W, fmt, G, r, c):

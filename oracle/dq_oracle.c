@@ -439,12 +439,35 @@ static double tile_error(const float* W, int64_t m, int64_t n, int fmt, int G, i
 /* error at the scales after round t (t = 0: initialisation).          */
 /* flags skip the row (BETA_ONLY) or column (ALPHA_ONLY) half-step.    */
 /* ------------------------------------------------------------------ */
+/* Grid values of the tile's codes at the current scales, into q (m x G). */
+static void tile_codes(const float* W, int64_t m, int64_t n, int fmt, int G, int64_t b,
+                       const float* r, const float* c, double* q) {
+  int64_t nb = n / G;
+  for (int64_t i = 0; i < m; ++i)
+    for (int j = 0; j < G; ++j) {
+      int64_t col = b * G + j;
+      q[i * G + j] = elem_value(fmt, elem_encode(fmt, quant_arg(W[i * n + col], inv32(c[col]),
+                                                                  inv32(r[i * nb + b]))));
+    }
+}
+
+/* qnum / qden (T+1 entries, nullable): for t >= 1 they accumulate
+ * ||Qhat(t) - Qhat(t-1)||_F^2 and ||Qhat(t-1)||_F^2, Qhat(t) being the code
+ * values at the scales after round t (the relative change of Fig. 2(a) /
+ * Fig. 3(a) is sqrt(qnum / qden)). */
 static void solve_tile_flags(const float* W, int64_t m, int64_t n, int fmt, int G, int T,
                              int64_t b, float s_T, float* r, float* c, double* err_trace,
-                             int flags) {
+                             int flags, double* qnum, double* qden) {
   int64_t nb = n / G;
   double* num = (double*)malloc(sizeof(double) * (size_t)G);
   double* den = (double*)malloc(sizeof(double) * (size_t)G);
+  double* qprev = NULL;
+  double* qcur = NULL;
+  if (qnum && qden) {
+    qprev = (double*)malloc(sizeof(double) * (size_t)(m * G));
+    qcur = (double*)malloc(sizeof(double) * (size_t)(m * G));
+    tile_codes(W, m, n, fmt, G, b, r, c, qprev);
+  }
   if (err_trace) err_trace[0] += tile_error(W, m, n, fmt, G, b, r, c);
   for (int t = 1; t <= T; ++t) {
     /* row half-step */
@@ -478,14 +501,27 @@ static void solve_tile_flags(const float* W, int64_t m, int64_t n, int fmt, int 
     for (int j = 0; j < G && !(flags & ORACLE_ALPHA_ONLY); ++j)
       c[b * G + j] = (den[j] > 0.0) ? proj_beta(fmt, num[j] / den[j]) : proj_beta(fmt, 1.0);
     if (err_trace) err_trace[t] += tile_error(W, m, n, fmt, G, b, r, c);
+    if (qprev) {
+      tile_codes(W, m, n, fmt, G, b, r, c, qcur);
+      for (int64_t k = 0; k < m * G; ++k) {
+        double d = qcur[k] - qprev[k];
+        qnum[t] += d * d;
+        qden[t] += qprev[k] * qprev[k];
+      }
+      double* tmp = qprev;
+      qprev = qcur;
+      qcur = tmp;
+    }
   }
   free(num);
   free(den);
+  free(qprev);
+  free(qcur);
 }
 
 static void solve_tile(const float* W, int64_t m, int64_t n, int fmt, int G, int T, int64_t b,
                        float s_T, float* r, float* c, double* err_trace) {
-  solve_tile_flags(W, m, n, fmt, G, T, b, s_T, r, c, err_trace, 0);
+  solve_tile_flags(W, m, n, fmt, G, T, b, s_T, r, c, err_trace, 0, NULL, NULL);
 }
 
 /* Full solve of the listed tiles (all tiles when tiles == NULL).
@@ -530,9 +566,34 @@ void oracle_solve(const float* W, int64_t m, int64_t n, int fmt, int G, int T,
  * result (r, c, s_T) continues it exactly.  r0 (m x n/G, nullable): initial
  * row-block scales, projected onto F_alpha; replaces the RTN
  * initialisation. */
+static void solve_ex_impl(const float* W, int64_t m, int64_t n, int fmt, int G, int T, int flags,
+                          const float* r0, const float* c0, const int64_t* tiles, int64_t ntiles,
+                          float* r, float* c, float* s_T, double* err_trace, double* w2,
+                          double* qnum, double* qden);
+
 void oracle_solve_ex(const float* W, int64_t m, int64_t n, int fmt, int G, int T, int flags,
                      const float* r0, const float* c0, const int64_t* tiles, int64_t ntiles,
                      float* r, float* c, float* s_T, double* err_trace, double* w2) {
+  solve_ex_impl(W, m, n, fmt, G, T, flags, r0, c0, tiles, ntiles, r, c, s_T, err_trace, w2, NULL,
+                NULL);
+}
+
+/* oracle_solve_ex plus the code-change trace of Fig. 2(a): qnum[t], qden[t]
+ * (T+1 entries each, entry 0 unused) as described at solve_tile_flags, summed
+ * over the solved tiles. */
+void oracle_solve_qtrace(const float* W, int64_t m, int64_t n, int fmt, int G, int T, int flags,
+                         const float* r0, const float* c0, const int64_t* tiles, int64_t ntiles,
+                         float* r, float* c, float* s_T, double* err_trace, double* w2,
+                         double* qnum, double* qden) {
+  for (int t = 0; t <= T; ++t) { qnum[t] = 0.0; qden[t] = 0.0; }
+  solve_ex_impl(W, m, n, fmt, G, T, flags, r0, c0, tiles, ntiles, r, c, s_T, err_trace, w2, qnum,
+                qden);
+}
+
+static void solve_ex_impl(const float* W, int64_t m, int64_t n, int fmt, int G, int T, int flags,
+                          const float* r0, const float* c0, const int64_t* tiles, int64_t ntiles,
+                          float* r, float* c, float* s_T, double* err_trace, double* w2,
+                          double* qnum, double* qden) {
   int64_t nb = n / G;
   if (c0) {
     for (int64_t j = 0; j < n; ++j) c[j] = proj_beta(fmt, (double)c0[j]);
@@ -560,7 +621,7 @@ void oracle_solve_ex(const float* W, int64_t m, int64_t n, int fmt, int G, int T
   }
   for (int64_t k = 0; k < cnt; ++k) {
     int64_t b = tiles ? tiles[k] : k;
-    solve_tile_flags(W, m, n, fmt, G, T, b, sT, r, c, err_trace, flags);
+    solve_tile_flags(W, m, n, fmt, G, T, b, sT, r, c, err_trace, flags, qnum, qden);
   }
 }
 
