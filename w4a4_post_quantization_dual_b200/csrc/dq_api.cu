@@ -214,9 +214,10 @@ int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, const f
 int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                    const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                    dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream) {
-  if (f == DQ_INT8 || f == DQ_MXINT8) return DQ_ERR_UNSUPPORTED;
+  if (f == DQ_INT8) return DQ_ERR_UNSUPPORTED;
   if (f == DQ_INT4) return DQ_ERR_UNSUPPORTED;
-  if (f != DQ_NVFP4 && f != DQ_MXFP4 && f != DQ_MXINT4 && f != DQ_MXFP8) return DQ_ERR_ARG;
+  if (f != DQ_NVFP4 && f != DQ_MXFP4 && f != DQ_MXINT4 && f != DQ_MXFP8 && f != DQ_MXINT8)
+    return DQ_ERR_ARG;
   if (!A || !sA || !B || !sB || !Y || M <= 0 || N <= 0 || K <= 0 || !valid_dtype(yt) ||
       N % 128 || K % 256 || !aligned(A, 16) || !aligned(B, 16) || !aligned(sA, 16) ||
       !aligned(sB, 16) || !aligned(Y, 16) || (f == DQ_NVFP4 && !s_tok) ||

@@ -1196,6 +1196,32 @@ __device__ __forceinline__ uint2 widen8(uint32_t w) {
   return make_uint2(out[0], out[1]);
 }
 
+// kind::f16 MMA (bf16 A and B from shared memory, fp32 accumulator), K = 16.
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Sixteen int8 codes (a 16-byte chunk) times the block's power of two ->
+// sixteen bf16 values, exact (8 significant bits), packed two per word.
+__device__ __forceinline__ void dequant16_bf16(uint4 v, float scale, uint32_t* out) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int lo = (int)(w[i] << (24 - 16 * h)) >> 24;       // byte 2h of the word
+      const int hi = (int)(w[i] << (16 - 16 * h)) >> 24;       // byte 2h + 1
+      const uint32_t blo = __float_as_uint(__fmul_rn((float)lo, scale)) >> 16;
+      const uint32_t bhi = __float_as_uint(__fmul_rn((float)hi, scale)) >> 16;
+      out[2 * i + h] = blo | (bhi << 16);
+    }
+}
+
 __device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate, uint32_t tsfa,
                                        uint32_t tsfb) {
@@ -1207,9 +1233,16 @@ __device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t
 }
 }  // namespace i4
 
-// FP8: MXFP8 operands (E4M3 codes in global memory): TMA places them
-// straight into the swizzled operand tiles and the converter warps idle.
-template <int YT, bool FP8>
+// MODE 0: MXINT4 (as described above).
+// MODE 1: MXFP8 operands (E4M3 codes in global memory): TMA places them
+//         straight into the swizzled operand tiles and the converter warps idle.
+// MODE 2: MXINT8 operands: an int8 code times its block's power of two is a
+//         bf16 value exactly, so the converters dequantise each 64-element
+//         k-tile (int8 staging, scale bytes read from global memory) into
+//         128-byte-swizzled bf16 operand tiles, and kind::f16 MMAs with fp32
+//         accumulation compute the block-scaled product exactly; no scale
+//         copies into tensor memory.
+template <int YT, int MODE>
 __global__ void __launch_bounds__(i4::THREADS, 1)
 w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const uint8_t* __restrict__ sfA,
@@ -1236,7 +1269,9 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (M + BM - 1) / BM, tiles_n = N / BN, num_tiles = tiles_m * tiles_n;
-  const int KT = K / BKE;
+  constexpr bool FP8 = MODE == 1, I8 = MODE == 2;
+  constexpr int KTE = I8 ? 64 : BKE;                 // elements per k-tile
+  const int KT = K / KTE;
   const int S4 = (K / 32) / 4;
 
   if (threadIdx.x == 0) {
@@ -1272,7 +1307,13 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
         const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-          if constexpr (FP8) {
+          if constexpr (I8) {          // int8 staging, 64 bytes per row; no scale copies
+            mbar_expect_tx(&full[stage], STG_A + STG_B);
+            tma_load_2d(stA + stage * STG_A, &tmA, &full[stage], kt * KTE, m0);
+            tma_load_2d(stB + stage * STG_B, &tmB, &full[stage], kt * KTE, n0);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            continue;
+          } else if constexpr (FP8) {
             mbar_expect_tx(&full[stage], OP_A + OP_B + SF_A + SF_B);
             tma_load_2d(opA + stage * OP_A, &tmA, &full[stage], kt * BKE, m0);
             tma_load_2d(opB + stage * OP_B, &tmB, &full[stage], kt * BKE, n0);
@@ -1301,10 +1342,28 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
       bool ok = true;
       // kind::mxf8f6f4: E4M3 A and B (format 0), E8M0 scales, K-major, M = 128
       const uint32_t idesc0 = ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24);
+      // kind::f16: fp32 accumulator (c_format 1), bf16 A and B (format 1), K-major
+      const uint32_t idesc_bf16 = (1u << 4) | (1u << 7) | (1u << 10) |
+                                  ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
         if (!mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag)) break;
         fence_after_sync();
         for (int kt = 0; kt < KT; ++kt) {
+          if constexpr (I8) {
+            if (!mbar_wait(&conv[stage], phase, abort_flag)) { ok = false; break; }
+            fence_after_sync();
+            const uint32_t a_base = smem_u32(opA + stage * OP_A);
+            const uint32_t b_base = smem_u32(opB + stage * OP_B);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {    // K = 16 bf16 (32 bytes) per MMA
+              const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, LAYOUT_SW128);
+              const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, LAYOUT_SW128);
+              mma_bf16(tmem, ad, bd, idesc_bf16, (kt > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            continue;
+          }
           if (!mbar_wait(FP8 ? &full[stage] : &conv[stage], phase, abort_flag) ||
               !mbar_wait(&sfready[stage], phase, abort_flag)) { ok = false; break; }
           fence_after_sync();
@@ -1328,7 +1387,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
   } else if (warp == 6) {
-    if (lane == 0) {
+    if (lane == 0 && !I8) {
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -1346,7 +1405,46 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
   } else if (warp >= 7) {
-    if constexpr (!FP8) {
+    if constexpr (I8) {
+    // converters: int8 staging x block power of two -> swizzled bf16 operand tiles
+    const int ct = threadIdx.x - 7 * 32;        // 0..127
+    const int64_t S = K / 32;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
+      for (int kt = 0; kt < KT; ++kt) {
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&full[stage], phase, abort_flag) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        // 16-byte int8 chunks: A rows 0..127 (4 chunks each), then B rows
+#pragma unroll 2
+        for (int c = ct; c < (BM + BN) * 4; c += 128) {
+          const bool isB = c >= BM * 4;
+          const int cc = isB ? c - BM * 4 : c;
+          const int r = cc >> 2, kc = cc & 3;
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              (isB ? stB + stage * STG_B : stA + stage * STG_A) + r * 64 + kc * 16);
+          // chunks 0-1 hold block 2kt of the row, chunks 2-3 block 2kt + 1; rows
+          // past M read the zero scale bytes of the padded layout
+          const int64_t grow = (isB ? n0 : m0) + r;
+          const uint32_t e = __ldg((isB ? sfB : sfA) + sf_offset(grow, 2 * kt + (kc >> 1), S));
+          uint32_t o[8];
+          dequant16_bf16(v, pow2f((int)e - 127), o);
+          unsigned char* rowp = (isB ? opB + stage * OP_B : opA + stage * OP_A) + r * 128;
+          const int sw = r & 7;
+          *reinterpret_cast<uint4*>(rowp + (((2 * kc) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(rowp + (((2 * kc + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&conv[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    } else if constexpr (!FP8) {
     // converters: packed INT4 staging -> swizzled E4M3 operand tiles
     const int ct = threadIdx.x - 7 * 32;        // 0..127
     int stage = 0;
@@ -1673,18 +1771,20 @@ static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, con
   return launch<FMT, 128, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
 }
 
-// FP8: MXFP8 codes (one byte per element, 128-byte swizzled TMA boxes);
-// otherwise packed MXINT4 codes (64-byte boxes into the staging buffers).
-template <int YT, bool FP8>
+// MODE 1: MXFP8 codes (one byte per element, 128-byte swizzled TMA boxes);
+// MODE 2: MXINT8 codes (one byte per element, 64-byte boxes of 64 elements
+// into the staging buffers); MODE 0: packed MXINT4 codes (64-byte boxes of
+// 128 elements into the staging buffers).
+template <int YT, int MODE>
 static int launch_mxint4(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB,
                          const float* r_row, void* Y, int64_t M, int64_t N, int64_t K,
                          cudaStream_t st) {
   CUtensorMap ta, tb;
-  const int64_t kb = FP8 ? K : K / 2;
-  const int box = FP8 ? i4::BKE : i4::BKE / 2;
+  const int64_t kb = MODE == 0 ? K / 2 : K;
+  const int box = MODE == 1 ? i4::BKE : i4::BKE / 2;
   if (!make_map(&ta, A, M, kb, BM, box) || !make_map(&tb, B, N, kb, i4::BN, box))
     return DQ_ERR_CUDA;
-  auto kern = w4a4_gemm_mxint4_kernel<YT, FP8>;
+  auto kern = w4a4_gemm_mxint4_kernel<YT, MODE>;
   if (!ensure_kernel_attrs((const void*)kern, i4::SMEM, false)) return DQ_ERR_CUDA;
   const int64_t tiles = ((M + BM - 1) / BM) * (N / i4::BN);
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
@@ -1705,11 +1805,14 @@ int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const u
     return yt == 1 ? gemm::dispatch<MXFP4, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
                    : gemm::dispatch<MXFP4, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
   if (f == MXINT4)
-    return yt == 1 ? gemm::launch_mxint4<1, false>(A, sA, B, sB, r_row, Y, M, N, K, st)
-                   : gemm::launch_mxint4<0, false>(A, sA, B, sB, r_row, Y, M, N, K, st);
+    return yt == 1 ? gemm::launch_mxint4<1, 0>(A, sA, B, sB, r_row, Y, M, N, K, st)
+                   : gemm::launch_mxint4<0, 0>(A, sA, B, sB, r_row, Y, M, N, K, st);
   if (f == MXFP8)
-    return yt == 1 ? gemm::launch_mxint4<1, true>(A, sA, B, sB, r_row, Y, M, N, K, st)
-                   : gemm::launch_mxint4<0, true>(A, sA, B, sB, r_row, Y, M, N, K, st);
+    return yt == 1 ? gemm::launch_mxint4<1, 1>(A, sA, B, sB, r_row, Y, M, N, K, st)
+                   : gemm::launch_mxint4<0, 1>(A, sA, B, sB, r_row, Y, M, N, K, st);
+  if (f == MXINT8)
+    return yt == 1 ? gemm::launch_mxint4<1, 2>(A, sA, B, sB, r_row, Y, M, N, K, st)
+                   : gemm::launch_mxint4<0, 2>(A, sA, B, sB, r_row, Y, M, N, K, st);
   return DQ_ERR_UNSUPPORTED;
 }
 
