@@ -300,6 +300,25 @@ DQ_API int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, 
                               const float* s_tok, double* sums, void* stream);
 
 /* ------------------------------------------------------------------------
+ * dq_w4a4_linear_fused -- dq_quantize_act followed by dq_w4a4_linear in one
+ * kernel, for small token counts (decode): the activation rescale by c and
+ * the NVFP4 quantisation (per-token scale over the whole row, UE4M3 block
+ * scales, E2M1 codes, the arithmetic of dq_quantize_act) run in the GEMM's
+ * producer warps, so no activation codes travel through memory.  Y equals
+ * the unfused pair's output bit for bit.
+ *
+ *  X        M x K bf16 activations (xt must be DQ_BF16); c K fp32 or NULL.
+ *  B, sB, s_w, r_row, Y, yt, N, K   as dq_w4a4_linear (NVFP4 only).
+ * Returns DQ_ERR_UNSUPPORTED when no split of K across a cluster leaves each
+ * CTA at most its pipeline depth of k-tiles within one wave of the GPU (use
+ * the unfused pair then), or for a format other than NVFP4.
+ * ---------------------------------------------------------------------- */
+DQ_API int dq_w4a4_linear_fused(const void* X, dq_dtype xt, const float* c, const uint8_t* B,
+                                const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
+                                dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f,
+                                void* stream);
+
+/* ------------------------------------------------------------------------
  * dq_solve_scales_noalloc -- dq_solve_scales for callers that cannot
  * allocate device memory (the paper has no counterpart: this is a library
  * convenience).  Some callers have no way to provide the workspace: a

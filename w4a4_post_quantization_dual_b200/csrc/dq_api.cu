@@ -211,6 +211,19 @@ int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, const f
                              (cudaStream_t)stream);
 }
 
+int dq_w4a4_linear_fused(const void* X, dq_dtype xt, const float* c, const uint8_t* B,
+                         const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
+                         dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f,
+                         void* stream) {
+  if (f != DQ_NVFP4 || xt != DQ_BF16) return DQ_ERR_UNSUPPORTED;
+  if (!X || !B || !sB || !s_w || !Y || M <= 0 || N <= 0 || K <= 0 || !valid_dtype(yt) ||
+      N % 128 || K % 256 || !aligned(X, 16) || !aligned(B, 16) || !aligned(sB, 16) ||
+      !aligned(Y, 16) || !aligned(c, 4) || M > ((int64_t)1 << 31) - 128 ||
+      N > ((int64_t)1 << 31) || K > ((int64_t)1 << 20))
+    return DQ_ERR_ARG;
+  return dq::w4a4_linear_fused(X, c, B, sB, s_w, r_row, Y, yt, M, N, K, (cudaStream_t)stream);
+}
+
 int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                    const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                    dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream) {
