@@ -150,6 +150,10 @@ DQ_API int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_
  *           that solve exactly: T1 rounds then T2 resumed rounds give the
  *           scales and trace tail of T1 + T2 rounds.  Ignored (s_tensor
  *           receives 1.0) for the other formats.
+ *  DQ_SOLVE_TRACE_CODES  mse_trace (then required) holds 2 (T+1) doubles:
+ *           the MSE trace, then the relative code change of Fig. 2(a) /
+ *           Fig. 3(a), ||Qhat(t) - Qhat(t-1)||_F / ||Qhat(t-1)||_F with
+ *           Qhat(t) the codes at the scales after round t (entry 0 NaN).
  *  r0       nullable, device, m x (n/G) fp32, positive and finite: initial
  *           row-block scales (the initialisation (alpha_0, beta_0) of
  *           Section 5.3 given by the caller), each projected onto F_alpha
@@ -164,7 +168,8 @@ DQ_API int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_
 typedef enum {
   DQ_SOLVE_ALPHA_ONLY = 1,
   DQ_SOLVE_BETA_ONLY = 2,
-  DQ_SOLVE_KEEP_TENSOR_SCALE = 4
+  DQ_SOLVE_KEEP_TENSOR_SCALE = 4,
+  DQ_SOLVE_TRACE_CODES = 8
 } dq_solve_flags;
 DQ_API int dq_solve_scales_ex(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f,
                               int group, int T, unsigned flags, const float* r0, const float* c0,
@@ -340,7 +345,7 @@ DQ_API int dq_w4a4_linear_fused(const void* X, dq_dtype xt, const float* c, cons
  *    them) race on the array and may corrupt each other's trace and NVFP4
  *    tensor scale; serialise them.
  * ---------------------------------------------------------------------- */
-#define DQ_NOALLOC_SCRATCH_BYTES 16384
+#define DQ_NOALLOC_SCRATCH_BYTES 49152
 #define DQ_NOALLOC_MAX_ROUNDS 2045
 DQ_API int dq_solve_scales_noalloc(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f,
                                    int group, int T, float* r, float* c, float* s_tensor,

@@ -127,8 +127,10 @@ int dq_solve_scales_ex(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_form
                        float* c, float* s_tensor, double* mse_trace, void* workspace,
                        size_t ws_bytes, void* stream) {
   const int G = resolve_group(f, group);
-  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE;
-  if (!W || !r || !c || !s_tensor || m <= 0 || n <= 0 || T < 0 || !valid_dtype(wt) ||
+  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE |
+                         DQ_SOLVE_TRACE_CODES;
+  if (((flags & DQ_SOLVE_TRACE_CODES) && !mse_trace) ||
+      !W || !r || !c || !s_tensor || m <= 0 || n <= 0 || T < 0 || !valid_dtype(wt) ||
       !valid_group(f, G) || n % G || !aligned(W, 16) || !aligned(r, 4) || !aligned(c, 4) ||
       !aligned(r0, 4) || !aligned(c0, 4) || (flags & ~known) ||
       ((flags & DQ_SOLVE_ALPHA_ONLY) && (flags & DQ_SOLVE_BETA_ONLY)) ||
@@ -150,8 +152,10 @@ int dq_solve_scales_batched(int nw, const void* const* W, dq_dtype wt, const int
                             double* const* mse_trace, void* workspace, size_t ws_bytes,
                             void* stream) {
   const int G = resolve_group(f, group);
-  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE;
-  if (nw <= 0 || !W || !m || !n || !r || !c || !s_tensor || T < 0 || !valid_dtype(wt) ||
+  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE |
+                         DQ_SOLVE_TRACE_CODES;
+  if (((flags & DQ_SOLVE_TRACE_CODES) && !mse_trace) ||
+      nw <= 0 || !W || !m || !n || !r || !c || !s_tensor || T < 0 || !valid_dtype(wt) ||
       !valid_group(f, G) || (flags & ~known) ||
       ((flags & DQ_SOLVE_ALPHA_ONLY) && (flags & DQ_SOLVE_BETA_ONLY)))
     return DQ_ERR_ARG;

@@ -130,6 +130,7 @@ def dq_solve_scales(W, fmt, T, r, c, s_tensor, mse_trace=None, workspace=None, g
 
 
 DQ_SOLVE_ALPHA_ONLY, DQ_SOLVE_BETA_ONLY, DQ_SOLVE_KEEP_TENSOR_SCALE = 1, 2, 4
+DQ_SOLVE_TRACE_CODES = 8
 
 
 def dq_solve_scales_ex(W, fmt, T, r, c, s_tensor, flags=0, r0=None, c0=None, mse_trace=None,
