@@ -150,6 +150,10 @@ DQ_API int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_
  *           that solve exactly: T1 rounds then T2 resumed rounds give the
  *           scales and trace tail of T1 + T2 rounds.  Ignored (s_tensor
  *           receives 1.0) for the other formats.
+ *  DQ_SOLVE_TRACE_CODES  mse_trace (then required) holds 2 (T+1) doubles:
+ *           the MSE trace, then the relative code change of Fig. 2(a) /
+ *           Fig. 3(a), ||Qhat(t) - Qhat(t-1)||_F / ||Qhat(t-1)||_F with
+ *           Qhat(t) the codes at the scales after round t (entry 0 NaN).
  *  r0       nullable, device, m x (n/G) fp32, positive and finite: initial
  *           row-block scales (the initialisation (alpha_0, beta_0) of
  *           Section 5.3 given by the caller), each projected onto F_alpha
@@ -164,7 +168,8 @@ DQ_API int dq_solve_scales(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_
 typedef enum {
   DQ_SOLVE_ALPHA_ONLY = 1,
   DQ_SOLVE_BETA_ONLY = 2,
-  DQ_SOLVE_KEEP_TENSOR_SCALE = 4
+  DQ_SOLVE_KEEP_TENSOR_SCALE = 4,
+  DQ_SOLVE_TRACE_CODES = 8
 } dq_solve_flags;
 DQ_API int dq_solve_scales_ex(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f,
                               int group, int T, unsigned flags, const float* r0, const float* c0,
@@ -300,6 +305,25 @@ DQ_API int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, 
                               const float* s_tok, double* sums, void* stream);
 
 /* ------------------------------------------------------------------------
+ * dq_w4a4_linear_fused -- dq_quantize_act followed by dq_w4a4_linear in one
+ * kernel, for small token counts (decode): the activation rescale by c and
+ * the NVFP4 quantisation (per-token scale over the whole row, UE4M3 block
+ * scales, E2M1 codes, the arithmetic of dq_quantize_act) run in the GEMM's
+ * producer warps, so no activation codes travel through memory.  Y equals
+ * the unfused pair's output bit for bit.
+ *
+ *  X        M x K bf16 activations (xt must be DQ_BF16); c K fp32 or NULL.
+ *  B, sB, s_w, r_row, Y, yt, N, K   as dq_w4a4_linear (NVFP4 only).
+ * Returns DQ_ERR_UNSUPPORTED when no split of K across a cluster leaves each
+ * CTA at most its pipeline depth of k-tiles within one wave of the GPU (use
+ * the unfused pair then), or for a format other than NVFP4.
+ * ---------------------------------------------------------------------- */
+DQ_API int dq_w4a4_linear_fused(const void* X, dq_dtype xt, const float* c, const uint8_t* B,
+                                const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
+                                dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f,
+                                void* stream);
+
+/* ------------------------------------------------------------------------
  * dq_solve_scales_noalloc -- dq_solve_scales for callers that cannot
  * allocate device memory (the paper has no counterpart: this is a library
  * convenience).  Some callers have no way to provide the workspace: a
@@ -321,7 +345,7 @@ DQ_API int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, 
  *    them) race on the array and may corrupt each other's trace and NVFP4
  *    tensor scale; serialise them.
  * ---------------------------------------------------------------------- */
-#define DQ_NOALLOC_SCRATCH_BYTES 16384
+#define DQ_NOALLOC_SCRATCH_BYTES 49152
 #define DQ_NOALLOC_MAX_ROUNDS 2045
 DQ_API int dq_solve_scales_noalloc(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_format f,
                                    int group, int T, float* r, float* c, float* s_tensor,

@@ -53,22 +53,24 @@ def test_act_error_8bit_parity(fmt, G):
     np.testing.assert_allclose(sums.cpu().numpy(), O.act_error_sums(X, c, fmt, G), rtol=1e-9)
 
 
+@pytest.mark.parametrize("fmt", [O.MXFP8, O.MXINT8])
 @pytest.mark.parametrize("M,N,K", [(1, 256, 512), (130, 256, 512), (300, 1024, 2048)])
 @pytest.mark.parametrize("ydtype", [torch.float32, torch.bfloat16])
-def test_mxfp8_linear_parity(M, N, K, ydtype):
-    """MXFP8 linear (E4M3 codes, E8M0 32-blocks, tcgen05 kind::mxf8f6f4) on
-    the device's own codes vs the fp64 reference product: relative Frobenius
-    error <= 1e-3 (fp32 output) / bf16 rounding of the reference (bf16)."""
+def test_mx8_linear_parity(fmt, M, N, K, ydtype):
+    """MXFP8 linear (E4M3 codes, E8M0 32-blocks, tcgen05 kind::mxf8f6f4) and
+    MXINT8 linear (int8 codes dequantised exactly to bf16 on chip, kind::f16)
+    on the device's own codes vs the fp64 reference product: relative
+    Frobenius error <= 1e-3 (fp32 output) / bf16 rounding of the reference."""
     X, _ = synth.activations(M, K, 95, n_outliers=4, outlier_scale=50.0)
     X = torch.from_numpy(X).to(torch.bfloat16).to(torch.float32).numpy()
     W, _ = synth.student_t_weight(N, K, 96, outlier_cols=3, outlier_scale=20.0, bf16=True)
-    r, c, sT, _ = gpu_solve(W, O.MXFP8, 32, 5, trace=False)
-    A, sA, _ = gpu_act(X, c, O.MXFP8, 32)
-    B, sB = gpu_pack(W, r, c, sT, O.MXFP8, 32)
+    r, c, sT, _ = gpu_solve(W, fmt, 32, 5, trace=False)
+    A, sA, _ = gpu_act(X, c, fmt, 32)
+    B, sB = gpu_pack(W, r, c, sT, fmt, 32)
     Y = torch.empty((M, N), dtype=ydtype, device=DEV)
-    dq.dq_w4a4_linear(to_dev(A), to_dev(sA), None, to_dev(B), to_dev(sB), None, Y, O.MXFP8)
+    dq.dq_w4a4_linear(to_dev(A), to_dev(sA), None, to_dev(B), to_dev(sB), None, Y, fmt)
     torch.cuda.synchronize()
-    ref = O.linear(A, sA, None, B, sB, 1.0, M, N, K, O.MXFP8)
+    ref = O.linear(A, sA, None, B, sB, 1.0, M, N, K, fmt)
     got = Y.float().cpu().numpy().astype(np.float64)
     if ydtype == torch.float32:
         assert np.linalg.norm(got - ref) <= 1e-3 * np.linalg.norm(ref)

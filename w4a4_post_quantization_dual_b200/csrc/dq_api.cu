@@ -127,8 +127,10 @@ int dq_solve_scales_ex(const void* W, dq_dtype wt, int64_t m, int64_t n, dq_form
                        float* c, float* s_tensor, double* mse_trace, void* workspace,
                        size_t ws_bytes, void* stream) {
   const int G = resolve_group(f, group);
-  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE;
-  if (!W || !r || !c || !s_tensor || m <= 0 || n <= 0 || T < 0 || !valid_dtype(wt) ||
+  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE |
+                         DQ_SOLVE_TRACE_CODES;
+  if (((flags & DQ_SOLVE_TRACE_CODES) && !mse_trace) ||
+      !W || !r || !c || !s_tensor || m <= 0 || n <= 0 || T < 0 || !valid_dtype(wt) ||
       !valid_group(f, G) || n % G || !aligned(W, 16) || !aligned(r, 4) || !aligned(c, 4) ||
       !aligned(r0, 4) || !aligned(c0, 4) || (flags & ~known) ||
       ((flags & DQ_SOLVE_ALPHA_ONLY) && (flags & DQ_SOLVE_BETA_ONLY)) ||
@@ -150,8 +152,10 @@ int dq_solve_scales_batched(int nw, const void* const* W, dq_dtype wt, const int
                             double* const* mse_trace, void* workspace, size_t ws_bytes,
                             void* stream) {
   const int G = resolve_group(f, group);
-  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE;
-  if (nw <= 0 || !W || !m || !n || !r || !c || !s_tensor || T < 0 || !valid_dtype(wt) ||
+  const unsigned known = DQ_SOLVE_ALPHA_ONLY | DQ_SOLVE_BETA_ONLY | DQ_SOLVE_KEEP_TENSOR_SCALE |
+                         DQ_SOLVE_TRACE_CODES;
+  if (((flags & DQ_SOLVE_TRACE_CODES) && !mse_trace) ||
+      nw <= 0 || !W || !m || !n || !r || !c || !s_tensor || T < 0 || !valid_dtype(wt) ||
       !valid_group(f, G) || (flags & ~known) ||
       ((flags & DQ_SOLVE_ALPHA_ONLY) && (flags & DQ_SOLVE_BETA_ONLY)))
     return DQ_ERR_ARG;
@@ -211,12 +215,26 @@ int dq_act_quant_error(const void* X, dq_dtype xt, int64_t M, int64_t K, const f
                              (cudaStream_t)stream);
 }
 
+int dq_w4a4_linear_fused(const void* X, dq_dtype xt, const float* c, const uint8_t* B,
+                         const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
+                         dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f,
+                         void* stream) {
+  if (f != DQ_NVFP4 || xt != DQ_BF16) return DQ_ERR_UNSUPPORTED;
+  if (!X || !B || !sB || !s_w || !Y || M <= 0 || N <= 0 || K <= 0 || !valid_dtype(yt) ||
+      N % 128 || K % 256 || !aligned(X, 16) || !aligned(B, 16) || !aligned(sB, 16) ||
+      !aligned(Y, 16) || !aligned(c, 4) || M > ((int64_t)1 << 31) - 128 ||
+      N > ((int64_t)1 << 31) || K > ((int64_t)1 << 20))
+    return DQ_ERR_ARG;
+  return dq::w4a4_linear_fused(X, c, B, sB, s_w, r_row, Y, yt, M, N, K, (cudaStream_t)stream);
+}
+
 int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                    const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                    dq_dtype yt, int64_t M, int64_t N, int64_t K, dq_format f, void* stream) {
-  if (f == DQ_INT8 || f == DQ_MXINT8) return DQ_ERR_UNSUPPORTED;
+  if (f == DQ_INT8) return DQ_ERR_UNSUPPORTED;
   if (f == DQ_INT4) return DQ_ERR_UNSUPPORTED;
-  if (f != DQ_NVFP4 && f != DQ_MXFP4 && f != DQ_MXINT4 && f != DQ_MXFP8) return DQ_ERR_ARG;
+  if (f != DQ_NVFP4 && f != DQ_MXFP4 && f != DQ_MXINT4 && f != DQ_MXFP8 && f != DQ_MXINT8)
+    return DQ_ERR_ARG;
   if (!A || !sA || !B || !sB || !Y || M <= 0 || N <= 0 || K <= 0 || !valid_dtype(yt) ||
       N % 128 || K % 256 || !aligned(A, 16) || !aligned(B, 16) || !aligned(sA, 16) ||
       !aligned(sB, 16) || !aligned(Y, 16) || (f == DQ_NVFP4 && !s_tok) ||

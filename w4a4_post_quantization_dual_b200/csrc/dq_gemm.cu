@@ -530,18 +530,36 @@ __device__ __forceinline__ void st_dsmem_f32x4(uint32_t local_addr, uint32_t ran
                : "memory");
 }
 
+// A float of CTA `rank`'s shared memory (ordered after the peer's write by a
+// cluster barrier).
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
+  uint32_t a = (uint32_t)__cvta_generic_to_shared(local), ra;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+
 constexpr int SK_BN = 128;
 // partial slices received from the S CTAs of the cluster: [S][BM][BN / S] floats
 constexpr int SK_PART_BYTES = BM * SK_BN * 4;
 
-template <int FMT, int YT>
+// FUSED (NVFP4, bf16 activations): the activation rescale and quantisation
+// run inside the kernel.  Each CTA takes the per-token maximum of |x c| over
+// its K slice, the cluster combines them over DSMEM into s_tok, and warps
+// 2..5 write the A operand tiles (128-byte swizzled E2M1 codes) and the A
+// scale atoms (UE4M3) of every k-tile of the slice straight into the stage
+// buffers, with the arithmetic of the standalone activation quantiser; TMA
+// brings only the weights.  Requires kt_per_slice <= STAGES.
+template <int FMT, int YT, bool FUSED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const uint8_t* __restrict__ sfA,
                         const uint8_t* __restrict__ sfB, const float* __restrict__ s_tok,
                         const float* __restrict__ s_w, const float* __restrict__ r_row,
                         void* __restrict__ Y, int M, int N, int K, int kt_per_slice,
-                        int a_rows) {
+                        int a_rows, const __nv_bfloat16* __restrict__ X,
+                        const float* __restrict__ cvec) {
   constexpr int BN = SK_BN;
   using C = Cfg<FMT, BN, SK_PART_BYTES>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -560,6 +578,8 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
   __shared__ float s_rs[BM];       // per-row output scale
   __shared__ float s_rr[SK_BN];    // per-output-column factor of this tile
+  __shared__ float s_pamax[FUSED ? BM : 1];   // FUSED: this CTA's row maxima of |x c|
+  __shared__ float s_stok[FUSED ? BM : 1];    // FUSED: per-token scale of the m-tile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -573,7 +593,8 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      // FUSED: the weights' TMA plus one arrival per A-producer warp
+      mbar_init(&full[s], FUSED ? 5 : 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sfready[s], COPIERS);
     }
@@ -594,8 +615,51 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
   const uint32_t tmem = *tmem_base_slot;
   pdl_trigger();   // weights are fetched before the dependency wait (see the 1-CTA kernel)
 
+  if constexpr (FUSED) {
+    // weights of every k-tile of the slice first (they do not depend on X)
+    if (warp == 0 && lane == 0) {
+      for (int kt = 0; kt < kt_per_slice; ++kt) {
+        mbar_expect_tx(&full[kt], C::B_BYTES + C::SFB_BYTES);
+        tma_load_2d(sB + kt * C::B_BYTES, &tmB, &full[kt], (kt0 + kt) * BKB, n0);
+        bulk_load(sSFB + kt * C::SFB_BYTES,
+                  sfB + ((size_t)(n0 / 128) * S4 + (size_t)(kt0 + kt) * C::SF_ATOMS) * 512,
+                  C::SFB_BYTES, &full[kt]);
+      }
+    }
+    pdl_wait();   // X and c may come from the kernel launched just before
+    // row maxima of |x c| over this CTA's K slice: one warp per row, lanes
+    // over 8-element pieces
+    const int rows_here = (M - m0) < a_rows ? (M - m0) : a_rows;
+    const int64_t k_lo = (int64_t)kt0 * BK, k_n = (int64_t)kt_per_slice * BK;
+    for (int r = warp; r < a_rows; r += NUM_THREADS / 32) {
+      float a = 0.0f;
+      if (r < rows_here) {
+        const __nv_bfloat16* xr = X + (size_t)(m0 + r) * K + k_lo;
+        for (int64_t p = lane * 8; p < k_n; p += 256) {
+          float x[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(xr + p), x);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float cv = cvec ? __ldg(cvec + k_lo + p + k) : 1.0f;
+            a = fmaxf(a, fabsf(__fmul_rn(x[k], cv)));
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      if (lane == 0) s_pamax[r] = a;
+    }
+    cluster_barrier();   // every CTA's partial maxima are visible to the cluster
+    if ((int)threadIdx.x < a_rows) {
+      float a = 0.0f;
+      for (uint32_t q = 0; q < S; ++q) a = fmaxf(a, ld_dsmem_f32(&s_pamax[threadIdx.x], q));
+      s_stok[threadIdx.x] = __fdiv_rn(a, 2688.0f);
+    }
+    __syncthreads();
+  }
+
   if (warp == 0) {
-    if (lane == 0) {
+    if (lane == 0 && !FUSED) {
       // A tiles carry only the a_rows rows that exist (rounded up to 16): the
       // MMA's other rows feed accumulator rows that are never stored
       const uint32_t tx = C::STAGE_BYTES - (BM - a_rows) * BKB;
@@ -695,6 +759,52 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     __syncwarp();
     const int quad = warp & 3;
+    if (FUSED && !copier) {
+      // A producers: codes and scale bytes of every (row, 16-block) of every
+      // k-tile of the slice, rows past M as zeros
+      const int pt = (warp - 2) * 32 + lane;            // 0..127
+      const int rows_here = (M - m0) < a_rows ? (M - m0) : a_rows;
+      for (int kt = 0; kt < kt_per_slice; ++kt) {
+        unsigned char* tA = sA + kt * C::A_BYTES;
+        unsigned char* tS = sSFA + kt * C::SFA_BYTES;
+        const int64_t kb = (int64_t)(kt0 + kt) * BK;
+        for (int idx = pt; idx < a_rows * (BK / 16); idx += 128) {
+          const int r = idx / (BK / 16), j = idx % (BK / 16);
+          uint32_t byte = 0u;
+          uint2 codes = make_uint2(0u, 0u);
+          if (r < rows_here) {
+            const float st = s_stok[r];
+            const __nv_bfloat16* xr = X + (size_t)(m0 + r) * K + kb + j * 16;
+            float xt[16];
+            bf16x8_to_f32(reinterpret_cast<const uint4*>(xr)[0], xt);
+            bf16x8_to_f32(reinterpret_cast<const uint4*>(xr)[1], xt + 8);
+            float ab = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float cv = cvec ? __ldg(cvec + kb + j * 16 + k) : 1.0f;
+              xt[k] = __fmul_rn(xt[k], cv);
+              ab = fmaxf(ab, fabsf(xt[k]));
+            }
+            byte = st > 0.0f ? ue4m3_rn(__fdiv_rn(ab, __fmul_rn(6.0f, st))) : 0u;
+            const float sblk = __fmul_rn(ue4m3_value(byte), st);
+            if (sblk != 0.0f) {
+              const float inv = __frcp_rn(sblk);
+#pragma unroll
+              for (int k = 0; k < 16; ++k) xt[k] = __fmul_rn(xt[k], inv);
+              codes = make_uint2(e2m1x8(xt), e2m1x8(xt + 8));
+            }
+          }
+          // 8 code bytes at byte j * 8 of the row, 16-byte chunks swizzled by row
+          *reinterpret_cast<uint2*>(tA + r * 128 + ((((j >> 1) ^ (r & 7))) << 4) + (j & 1) * 8) =
+              codes;
+          tS[(j >> 2) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (j & 3)] = (uint8_t)byte;
+        }
+        // generic-proxy writes -> visible to the tensor core and tcgen05.cp
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[kt]);
+      }
+    }
     if (!copier) {
       // per-row scale and the tile's output-row factors, staged before the
       // accumulator wait so the reduction below reads shared memory only
@@ -703,7 +813,11 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
       pdl_wait();
       const int rr = quad * 32 + lane;
       float rs = (FMT == NVFP4 && s_w) ? *s_w : 1.0f;
-      if (FMT == NVFP4 && s_tok && m0 + rr < M) rs = __fmul_rn(s_tok[m0 + rr], rs);
+      if constexpr (FUSED) {
+        if (m0 + rr < M && rr < a_rows) rs = __fmul_rn(s_stok[rr], rs);
+      } else {
+        if (FMT == NVFP4 && s_tok && m0 + rr < M) rs = __fmul_rn(s_tok[m0 + rr], rs);
+      }
       s_rs[rr] = rs;
       s_rr[rr] = r_row ? __ldg(r_row + n0 + rr) : 1.0f;
     }
@@ -1196,6 +1310,32 @@ __device__ __forceinline__ uint2 widen8(uint32_t w) {
   return make_uint2(out[0], out[1]);
 }
 
+// kind::f16 MMA (bf16 A and B from shared memory, fp32 accumulator), K = 16.
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Sixteen int8 codes (a 16-byte chunk) times the block's power of two ->
+// sixteen bf16 values, exact (8 significant bits), packed two per word.
+__device__ __forceinline__ void dequant16_bf16(uint4 v, float scale, uint32_t* out) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int lo = (int)(w[i] << (24 - 16 * h)) >> 24;       // byte 2h of the word
+      const int hi = (int)(w[i] << (16 - 16 * h)) >> 24;       // byte 2h + 1
+      const uint32_t blo = __float_as_uint(__fmul_rn((float)lo, scale)) >> 16;
+      const uint32_t bhi = __float_as_uint(__fmul_rn((float)hi, scale)) >> 16;
+      out[2 * i + h] = blo | (bhi << 16);
+    }
+}
+
 __device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate, uint32_t tsfa,
                                        uint32_t tsfb) {
@@ -1207,9 +1347,16 @@ __device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t
 }
 }  // namespace i4
 
-// FP8: MXFP8 operands (E4M3 codes in global memory): TMA places them
-// straight into the swizzled operand tiles and the converter warps idle.
-template <int YT, bool FP8>
+// MODE 0: MXINT4 (as described above).
+// MODE 1: MXFP8 operands (E4M3 codes in global memory): TMA places them
+//         straight into the swizzled operand tiles and the converter warps idle.
+// MODE 2: MXINT8 operands: an int8 code times its block's power of two is a
+//         bf16 value exactly, so the converters dequantise each 64-element
+//         k-tile (int8 staging, scale bytes read from global memory) into
+//         128-byte-swizzled bf16 operand tiles, and kind::f16 MMAs with fp32
+//         accumulation compute the block-scaled product exactly; no scale
+//         copies into tensor memory.
+template <int YT, int MODE>
 __global__ void __launch_bounds__(i4::THREADS, 1)
 w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const uint8_t* __restrict__ sfA,
@@ -1236,7 +1383,9 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (M + BM - 1) / BM, tiles_n = N / BN, num_tiles = tiles_m * tiles_n;
-  const int KT = K / BKE;
+  constexpr bool FP8 = MODE == 1, I8 = MODE == 2;
+  constexpr int KTE = I8 ? 64 : BKE;                 // elements per k-tile
+  const int KT = K / KTE;
   const int S4 = (K / 32) / 4;
 
   if (threadIdx.x == 0) {
@@ -1272,7 +1421,13 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
         const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-          if constexpr (FP8) {
+          if constexpr (I8) {          // int8 staging, 64 bytes per row; no scale copies
+            mbar_expect_tx(&full[stage], STG_A + STG_B);
+            tma_load_2d(stA + stage * STG_A, &tmA, &full[stage], kt * KTE, m0);
+            tma_load_2d(stB + stage * STG_B, &tmB, &full[stage], kt * KTE, n0);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            continue;
+          } else if constexpr (FP8) {
             mbar_expect_tx(&full[stage], OP_A + OP_B + SF_A + SF_B);
             tma_load_2d(opA + stage * OP_A, &tmA, &full[stage], kt * BKE, m0);
             tma_load_2d(opB + stage * OP_B, &tmB, &full[stage], kt * BKE, n0);
@@ -1301,10 +1456,28 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
       bool ok = true;
       // kind::mxf8f6f4: E4M3 A and B (format 0), E8M0 scales, K-major, M = 128
       const uint32_t idesc0 = ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24);
+      // kind::f16: fp32 accumulator (c_format 1), bf16 A and B (format 1), K-major
+      const uint32_t idesc_bf16 = (1u << 4) | (1u << 7) | (1u << 10) |
+                                  ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
         if (!mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag)) break;
         fence_after_sync();
         for (int kt = 0; kt < KT; ++kt) {
+          if constexpr (I8) {
+            if (!mbar_wait(&conv[stage], phase, abort_flag)) { ok = false; break; }
+            fence_after_sync();
+            const uint32_t a_base = smem_u32(opA + stage * OP_A);
+            const uint32_t b_base = smem_u32(opB + stage * OP_B);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {    // K = 16 bf16 (32 bytes) per MMA
+              const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, LAYOUT_SW128);
+              const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, LAYOUT_SW128);
+              mma_bf16(tmem, ad, bd, idesc_bf16, (kt > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            continue;
+          }
           if (!mbar_wait(FP8 ? &full[stage] : &conv[stage], phase, abort_flag) ||
               !mbar_wait(&sfready[stage], phase, abort_flag)) { ok = false; break; }
           fence_after_sync();
@@ -1328,7 +1501,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
   } else if (warp == 6) {
-    if (lane == 0) {
+    if (lane == 0 && !I8) {
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -1346,7 +1519,46 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
   } else if (warp >= 7) {
-    if constexpr (!FP8) {
+    if constexpr (I8) {
+    // converters: int8 staging x block power of two -> swizzled bf16 operand tiles
+    const int ct = threadIdx.x - 7 * 32;        // 0..127
+    const int64_t S = K / 32;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
+      for (int kt = 0; kt < KT; ++kt) {
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&full[stage], phase, abort_flag) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        // 16-byte int8 chunks: A rows 0..127 (4 chunks each), then B rows
+#pragma unroll 2
+        for (int c = ct; c < (BM + BN) * 4; c += 128) {
+          const bool isB = c >= BM * 4;
+          const int cc = isB ? c - BM * 4 : c;
+          const int r = cc >> 2, kc = cc & 3;
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              (isB ? stB + stage * STG_B : stA + stage * STG_A) + r * 64 + kc * 16);
+          // chunks 0-1 hold block 2kt of the row, chunks 2-3 block 2kt + 1; rows
+          // past M read the zero scale bytes of the padded layout
+          const int64_t grow = (isB ? n0 : m0) + r;
+          const uint32_t e = __ldg((isB ? sfB : sfA) + sf_offset(grow, 2 * kt + (kc >> 1), S));
+          uint32_t o[8];
+          dequant16_bf16(v, pow2f((int)e - 127), o);
+          unsigned char* rowp = (isB ? opB + stage * OP_B : opA + stage * OP_A) + r * 128;
+          const int sw = r & 7;
+          *reinterpret_cast<uint4*>(rowp + (((2 * kc) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(rowp + (((2 * kc + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&conv[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    } else if constexpr (!FP8) {
     // converters: packed INT4 staging -> swizzled E4M3 operand tiles
     const int ct = threadIdx.x - 7 * 32;        // 0..127
     int stage = 0;
@@ -1532,12 +1744,35 @@ static int launch_splitk(const uint8_t* A, const uint8_t* sA, const float* s_tok
   const int a_rows = M < BM ? (int)((M + 15) / 16 * 16) : BM;
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, M, K / 2, a_rows) || !make_map(&tb, B, N, K / 2, SK_BN)) return DQ_ERR_CUDA;
-  auto kern = w4a4_gemm_splitk_kernel<FMT, YT>;
+  auto kern = w4a4_gemm_splitk_kernel<FMT, YT, false>;
   if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
   const int kt_per_slice = (int)(K / BK) / S;
   if (launch_ex(kern, dim3(S, (unsigned)(N / SK_BN), (unsigned)((M + BM - 1) / BM)),
                 dim3(NUM_THREADS), C::SMEM_BYTES, st, (unsigned)S, ta, tb, sA, sB, s_tok, s_w,
-                r_row, Y, (int)M, (int)N, (int)K, kt_per_slice, a_rows) != cudaSuccess)
+                r_row, Y, (int)M, (int)N, (int)K, kt_per_slice, a_rows,
+                (const __nv_bfloat16*)nullptr, (const float*)nullptr) != cudaSuccess)
+    return DQ_ERR_CUDA;
+  return DQ_OK;
+}
+
+// Fused activation quantisation + split-K GEMM (NVFP4, bf16 X): the A tensor
+// map is not used (a placeholder on the weights keeps the parameter valid).
+template <int YT>
+static int launch_splitk_fused(const __nv_bfloat16* X, const float* c, const uint8_t* B,
+                               const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
+                               int64_t M, int64_t N, int64_t K, int S, cudaStream_t st) {
+  using C = Cfg<NVFP4, SK_BN, SK_PART_BYTES>;
+  const int a_rows = M < BM ? (int)((M + 15) / 16 * 16) : BM;
+  const int kt_per_slice = (int)(K / BK) / S;
+  if (kt_per_slice > C::STAGES) return DQ_ERR_UNSUPPORTED;
+  CUtensorMap tb;
+  if (!make_map(&tb, B, N, K / 2, SK_BN)) return DQ_ERR_CUDA;
+  auto kern = w4a4_gemm_splitk_kernel<NVFP4, YT, true>;
+  if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
+  if (launch_ex(kern, dim3(S, (unsigned)(N / SK_BN), (unsigned)((M + BM - 1) / BM)),
+                dim3(NUM_THREADS), C::SMEM_BYTES, st, (unsigned)S, tb, tb,
+                (const uint8_t*)nullptr, sB, (const float*)nullptr, s_w, r_row, Y, (int)M,
+                (int)N, (int)K, kt_per_slice, a_rows, X, c) != cudaSuccess)
     return DQ_ERR_CUDA;
   return DQ_OK;
 }
@@ -1614,7 +1849,7 @@ static int splitk_max_clusters(int S) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16 || S < 1 || S > 8) return 0;
   if (cache[dev][S]) return cache[dev][S] > 0 ? cache[dev][S] : 0;
   using C = Cfg<FMT, SK_BN, SK_PART_BYTES>;
-  auto kern = w4a4_gemm_splitk_kernel<FMT, YT>;
+  auto kern = w4a4_gemm_splitk_kernel<FMT, YT, false>;
   int n = 0;
   if (ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) {
     cudaLaunchAttribute attr[1];
@@ -1673,18 +1908,20 @@ static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, con
   return launch<FMT, 128, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
 }
 
-// FP8: MXFP8 codes (one byte per element, 128-byte swizzled TMA boxes);
-// otherwise packed MXINT4 codes (64-byte boxes into the staging buffers).
-template <int YT, bool FP8>
+// MODE 1: MXFP8 codes (one byte per element, 128-byte swizzled TMA boxes);
+// MODE 2: MXINT8 codes (one byte per element, 64-byte boxes of 64 elements
+// into the staging buffers); MODE 0: packed MXINT4 codes (64-byte boxes of
+// 128 elements into the staging buffers).
+template <int YT, int MODE>
 static int launch_mxint4(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB,
                          const float* r_row, void* Y, int64_t M, int64_t N, int64_t K,
                          cudaStream_t st) {
   CUtensorMap ta, tb;
-  const int64_t kb = FP8 ? K : K / 2;
-  const int box = FP8 ? i4::BKE : i4::BKE / 2;
+  const int64_t kb = MODE == 0 ? K / 2 : K;
+  const int box = MODE == 1 ? i4::BKE : i4::BKE / 2;
   if (!make_map(&ta, A, M, kb, BM, box) || !make_map(&tb, B, N, kb, i4::BN, box))
     return DQ_ERR_CUDA;
-  auto kern = w4a4_gemm_mxint4_kernel<YT, FP8>;
+  auto kern = w4a4_gemm_mxint4_kernel<YT, MODE>;
   if (!ensure_kernel_attrs((const void*)kern, i4::SMEM, false)) return DQ_ERR_CUDA;
   const int64_t tiles = ((M + BM - 1) / BM) * (N / i4::BN);
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
@@ -1705,12 +1942,37 @@ int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const u
     return yt == 1 ? gemm::dispatch<MXFP4, 1>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
                    : gemm::dispatch<MXFP4, 0>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
   if (f == MXINT4)
-    return yt == 1 ? gemm::launch_mxint4<1, false>(A, sA, B, sB, r_row, Y, M, N, K, st)
-                   : gemm::launch_mxint4<0, false>(A, sA, B, sB, r_row, Y, M, N, K, st);
+    return yt == 1 ? gemm::launch_mxint4<1, 0>(A, sA, B, sB, r_row, Y, M, N, K, st)
+                   : gemm::launch_mxint4<0, 0>(A, sA, B, sB, r_row, Y, M, N, K, st);
   if (f == MXFP8)
-    return yt == 1 ? gemm::launch_mxint4<1, true>(A, sA, B, sB, r_row, Y, M, N, K, st)
-                   : gemm::launch_mxint4<0, true>(A, sA, B, sB, r_row, Y, M, N, K, st);
+    return yt == 1 ? gemm::launch_mxint4<1, 1>(A, sA, B, sB, r_row, Y, M, N, K, st)
+                   : gemm::launch_mxint4<0, 1>(A, sA, B, sB, r_row, Y, M, N, K, st);
+  if (f == MXINT8)
+    return yt == 1 ? gemm::launch_mxint4<1, 2>(A, sA, B, sB, r_row, Y, M, N, K, st)
+                   : gemm::launch_mxint4<0, 2>(A, sA, B, sB, r_row, Y, M, N, K, st);
   return DQ_ERR_UNSUPPORTED;
+}
+
+// Fused activation rescale + quantise + linear for small M (NVFP4, bf16 X):
+// the split of K is chosen as for the split-K GEMM, and must leave at most
+// STAGES k-tiles per CTA.
+int w4a4_linear_fused(const void* X, const float* c, const uint8_t* B, const uint8_t* sB,
+                      const float* s_w, const float* r_row, void* Y, int yt, int64_t M,
+                      int64_t N, int64_t K, cudaStream_t st) {
+  using C = gemm::Cfg<NVFP4, gemm::SK_BN, gemm::SK_PART_BYTES>;
+  const int sms = gemm::num_sms();
+  const int64_t tm = (M + gemm::BM - 1) / gemm::BM;
+  const int64_t t128 = tm * (N / gemm::SK_BN);
+  const int KT = (int)(K / gemm::BK);
+  int S = 0;
+  for (int cand : {8, 4, 2})
+    if (S == 0 && KT % cand == 0 && KT / cand <= C::STAGES && t128 * cand <= sms &&
+        t128 <= gemm::splitk_max_clusters<NVFP4, 1>(cand))
+      S = cand;
+  if (S == 0) return DQ_ERR_UNSUPPORTED;
+  const __nv_bfloat16* Xb = reinterpret_cast<const __nv_bfloat16*>(X);
+  return yt == 1 ? gemm::launch_splitk_fused<1>(Xb, c, B, sB, s_w, r_row, Y, M, N, K, S, st)
+                 : gemm::launch_splitk_fused<0>(Xb, c, B, sB, s_w, r_row, Y, M, N, K, S, st);
 }
 
 int read_device_error(int clear) {

@@ -20,6 +20,9 @@ int solve_scales_batched(int nw, const void* const* W, int wt, const int64_t* m,
                          const int64_t* n, int f, int G, int T, unsigned flags, float* const* r,
                          float* const* c, float* const* sT, double* const* trace, void* ws,
                          cudaStream_t st);
+int w4a4_linear_fused(const void* X, const float* c, const uint8_t* B, const uint8_t* sB,
+                      const float* s_w, const float* r_row, void* Y, int yt, int64_t M,
+                      int64_t N, int64_t K, cudaStream_t st);
 int act_quant_error(const void* X, int xt, int64_t M, int64_t K, const float* c, int f, int G,
                     const uint8_t* codes, const void* scales, const float* s_tok, double* sums,
                     cudaStream_t st);

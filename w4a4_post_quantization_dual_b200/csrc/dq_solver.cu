@@ -41,7 +41,8 @@ struct SolverShape {
   static constexpr int RPS = NW * RPW;         // rows per CTA per step
 };
 
-// Workspace layout (bytes): [0] u32 amax bits, [8] f64 ||W||^2, [16..] f64 err[T+1].
+// Workspace layout (bytes): [0] u32 amax bits, [8] f64 ||W||^2, [16..] f64
+// err[T+1], then f64 qnum[T+1] and qden[T+1] (code-change trace sums).
 struct SolverWs {
   uint32_t amax_bits;
   uint32_t pad;
@@ -57,7 +58,8 @@ struct SolveOpts {
   const float* r0;   // nullable, m x (n/G)
   const float* c0;   // nullable, n
 };
-constexpr unsigned SOLVE_ALPHA_ONLY = 1u, SOLVE_BETA_ONLY = 2u, SOLVE_KEEP_S = 4u;
+constexpr unsigned SOLVE_ALPHA_ONLY = 1u, SOLVE_BETA_ONLY = 2u, SOLVE_KEEP_S = 4u,
+                   SOLVE_TRACE_CODES = 8u;
 
 // The weights of one launch (all with the same row count m): launch z-index
 // i solves weight i.  Passed by value (kernel parameter space).
@@ -444,6 +446,8 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   constexpr bool WSMEM = STG != 0;
   using ST = typename std::conditional<STG == 2, float, WT>::type;  // staged element type
   ST* wch = reinterpret_cast<ST*>(atab + 128);      // staged rows
+  // TRACE: alpha of the previous round per row-step (code-change trace)
+  float* ap_s = reinterpret_cast<float*>(wch + (WSMEM ? (size_t)steps * S::RPS * G : 0));
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int oct = lane % S::OPB, rslot = warp * S::RPW + lane / S::OPB;
@@ -513,6 +517,9 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   const int64_t xgl_step = (int64_t)S::RPS * n;
   float* rsl = r_s + rslot;
   float* asl = a_s + rslot;
+  float* apl = ap_s + rslot;
+  const bool trace_codes = TRACE && (o.flags & SOLVE_TRACE_CODES);
+  float2 beta_prev[4];   // TRACE: beta of the previous round
   auto load_x = [&](int s, float2* x) {
     if constexpr (WSMEM) unpack8<ST>(xsm + s * XSM_STEP, x);
     else unpack8_global<WT>(xgl + s * xgl_step, x);
@@ -570,12 +577,14 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   for (int t = 0; t <= T; ++t) {
     // ---- row half-step (t < T) / error at the current scales ----
     float e_acc = 0.0f;
+    float2 qn2 = make_float2(0.f, 0.f), qd2 = qn2;   // TRACE: code-change sums
     bool any_tie = false;
     if ((t < T && !beta_only) || TRACE) {
       for (int s = 0; s < steps; ++s) {
         const bool valid = s < s_end;
         float2 num2 = make_float2(0.f, 0.f), den2 = num2, err2 = num2;
         const float rr = rsl[s * S::RPS], alpha = asl[s * S::RPS];
+        const float alpha_prev = (TRACE && t > 0) ? apl[s * S::RPS] : 0.0f;
         if (valid) {
           float2 x[4], z[4], q[4];
           load_x(s, x);
@@ -593,6 +602,19 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
               err2 = __ffma2_rn(d, d, err2);
             }
           }
+          if constexpr (TRACE) {
+            // Qhat(t) - Qhat(t-1): the codes at the previous round's scales
+            if (trace_codes && t > 0) {
+              const float2 ap2 = make_float2(alpha_prev, alpha_prev);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float2 qp = grid2_packed<F>(__fmul2_rn(__fmul2_rn(x[k], beta_prev[k]), ap2));
+                const float2 d = make_float2(q[k].x - qp.x, q[k].y - qp.y);
+                qn2 = __ffma2_rn(d, d, qn2);
+                qd2 = __ffma2_rn(qp, qp, qd2);
+              }
+            }
+          }
         }
         float num = num2.x + num2.y, den = den2.x + den2.y, err = err2.x + err2.y;
 #pragma unroll
@@ -602,6 +624,8 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
           if constexpr (TRACE) err += __shfl_xor_sync(0xffffffffu, err, o);
         }
         if (TRACE && oct == 0) e_acc += err;
+        // the alpha these codes were taken with serves the next round's trace
+        if (TRACE && trace_codes && oct == 0) apl[s * S::RPS] = alpha;
         if (t < T && !beta_only) {
           const float u = den > 0.0f ? __fdividef(num, den) : 1.0f;
           // all lanes of a row-block hold the same sums, hence the same flag
@@ -659,6 +683,21 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
 #pragma unroll
       for (int o = 16; o; o >>= 1) e_acc += __shfl_xor_sync(0xffffffffu, e_acc, o);
       if (lane == 0) atomicAdd(&ws->err[t], (double)e_acc);
+      if (trace_codes) {
+        // sums of this warp; qnum / qden follow err[T+1] in the workspace
+        float qn = qn2.x + qn2.y, qd = qd2.x + qd2.y;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          qn += __shfl_xor_sync(0xffffffffu, qn, o);
+          qd += __shfl_xor_sync(0xffffffffu, qd, o);
+        }
+        if (lane == 0 && t > 0) {
+          atomicAdd(&ws->err[(T + 1) + t], (double)qn);
+          atomicAdd(&ws->err[2 * (T + 1) + t], (double)qd);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) beta_prev[k] = beta[k];
+      }
     }
     if (t == T) break;
     __syncwarp();
@@ -794,19 +833,30 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   cluster_sync_all();  // no CTA leaves while a peer may still read its cpart
 }
 
-__global__ void solve_finalize_kernel(const SolverWs* ws, int T, double* mse_trace) {
+// mse_trace[t] = err[t] / ||W||^2; with the code-change trace also
+// mse_trace[T + 1 + t] = sqrt(qnum[t] / qden[t]) for t >= 1 (NaN at t = 0).
+__global__ void solve_finalize_kernel(const SolverWs* ws, int T, double* mse_trace, int codes) {
   int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t <= T) mse_trace[t] = ws->w2 > 0.0 ? ws->err[t] / ws->w2 : 0.0;
+  if (t <= T) {
+    mse_trace[t] = ws->w2 > 0.0 ? ws->err[t] / ws->w2 : 0.0;
+    if (codes) {
+      const double qn = ws->err[(T + 1) + t], qd = ws->err[2 * (T + 1) + t];
+      mse_trace[(T + 1) + t] = t == 0 ? __longlong_as_double(0x7FF8000000000000ll)
+                                      : (qd > 0.0 ? sqrt(qn / qd) : 0.0);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+// trace: one more float per row-step (the previous round's alpha, for the
+// code-change trace), after the staged rows.
 template <int G>
-static size_t solver_smem_bytes(int steps, size_t staged_elem_bytes) {
+static size_t solver_smem_bytes(int steps, size_t staged_elem_bytes, bool trace = false) {
   const size_t rows = (size_t)steps * SolverShape<G>::RPS;
   return sizeof(SolverSmem<G>) + 2 * sizeof(float) * rows + 2 * 128 * sizeof(float) +
-         rows * G * staged_elem_bytes;
+         rows * G * staged_elem_bytes + (trace ? sizeof(float) * rows : 0);
 }
 
 // Launch geometry: the tile's rows are split over C CTAs of one cluster,
@@ -855,16 +905,16 @@ static int launch_solver(const SolveBatch& bt, int count, int64_t m, int T, cons
   using S = SolverShape<G>;
   int steps, C, stg;
   solver_geometry<G, WT>(m, steps, C, stg);
-  const size_t sm_init = sizeof(SolverSmem<G>),
-               sm_main = solver_smem_bytes<G>(
-                   steps, stg == 2 ? sizeof(float) : (stg == 1 ? sizeof(WT) : 0));
-  if (sm_main > 227 * 1024) return DQ_ERR_UNSUPPORTED;
   int64_t tiles = 0;
   bool any_trace = false;
   for (int i = 0; i < count; ++i) {
     tiles = bt.item[i].n / G > tiles ? bt.item[i].n / G : tiles;
     any_trace = any_trace || (traces && traces[i]);
   }
+  const size_t sm_init = sizeof(SolverSmem<G>),
+               sm_main = solver_smem_bytes<G>(
+                   steps, stg == 2 ? sizeof(float) : (stg == 1 ? sizeof(WT) : 0), any_trace);
+  if (sm_main > 227 * 1024) return DQ_ERR_UNSUPPORTED;
   if (tiles > 65535) return DQ_ERR_UNSUPPORTED;
 
   cudaLaunchAttribute attr[1];
@@ -903,7 +953,8 @@ static int launch_solver(const SolveBatch& bt, int count, int64_t m, int T, cons
   if (e != cudaSuccess) return DQ_ERR_CUDA;
   for (int i = 0; i < count && any_trace; ++i) {
     if (!traces[i]) continue;
-    solve_finalize_kernel<<<(T + 1 + 127) / 128, 128, 0, st>>>(bt.item[i].ws, T, traces[i]);
+    solve_finalize_kernel<<<(T + 1 + 127) / 128, 128, 0, st>>>(
+        bt.item[i].ws, T, traces[i], (o.flags & SOLVE_TRACE_CODES) ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return DQ_ERR_CUDA;
   }
   return DQ_OK;
@@ -915,8 +966,8 @@ template <int G, typename WT>
 static int solver_supported(int64_t m, int64_t n) {
   int steps, C, stg;
   solver_geometry<G, WT>(m, steps, C, stg);
-  const size_t sm_main =
-      solver_smem_bytes<G>(steps, stg == 2 ? sizeof(float) : (stg == 1 ? sizeof(WT) : 0));
+  const size_t sm_main =   // with the trace array: the largest variant
+      solver_smem_bytes<G>(steps, stg == 2 ? sizeof(float) : (stg == 1 ? sizeof(WT) : 0), true);
   return (sm_main > 227 * 1024 || n / G > 65535) ? DQ_ERR_UNSUPPORTED : DQ_OK;
 }
 
@@ -959,7 +1010,7 @@ static int dispatch_solver(int f, int G, const SolveBatch& bt, int count, int64_
 }
 
 size_t solve_workspace_bytes(int T) {
-  size_t b = 16 + 8 * (size_t)(T + 1);
+  size_t b = 16 + 3 * 8 * (size_t)(T + 1);
   return (b + 255) & ~(size_t)255;
 }
 

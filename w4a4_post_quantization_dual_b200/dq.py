@@ -46,6 +46,8 @@ SIGNATURES = {
     "dq_solve_batched_workspace_size": (_sz, [_int, _int]),
     "dq_solve_scales_batched": (_int, [_int, _vp, _int, _vp, _vp, _int, _int, _int, ctypes.c_uint,
                                        _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "dq_w4a4_linear_fused": (_int, [_vp, _int, _vp, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64,
+                                    _i64, _int, _vp]),
     "dq_act_quant_error": (_int, [_vp, _int, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp, _vp,
                                   _vp]),
     "dq_device_error": (_int, [_int]),
@@ -128,6 +130,7 @@ def dq_solve_scales(W, fmt, T, r, c, s_tensor, mse_trace=None, workspace=None, g
 
 
 DQ_SOLVE_ALPHA_ONLY, DQ_SOLVE_BETA_ONLY, DQ_SOLVE_KEEP_TENSOR_SCALE = 1, 2, 4
+DQ_SOLVE_TRACE_CODES = 8
 
 
 def dq_solve_scales_ex(W, fmt, T, r, c, s_tensor, flags=0, r0=None, c0=None, mse_trace=None,
@@ -210,6 +213,16 @@ def dq_act_quant_error(X, fmt, c, codes, scales, s_tok, sums, group=0, stream=No
                                     _ptr(codes), _ptr(scales), _ptr(s_tok), _ptr(sums),
                                     _stream(stream)),
            "dq_act_quant_error")
+
+
+def dq_w4a4_linear_fused(X, c, B, sB, s_w, Y, fmt, r_row=None, stream=None):
+    """Activation quantisation + linear in one kernel (small M, NVFP4, bf16 X)."""
+    M, K = X.shape
+    N = B.shape[0]
+    _check(lib().dq_w4a4_linear_fused(_ptr(X), _dtype(X), _ptr(c), _ptr(B), _ptr(sB), _ptr(s_w),
+                                      _ptr(r_row), _ptr(Y), _dtype(Y), M, N, K, _fmt(fmt),
+                                      _stream(stream)),
+           "dq_w4a4_linear_fused")
 
 
 def dq_device_error(clear=True):
