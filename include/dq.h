@@ -339,6 +339,8 @@ DQ_API int dq_w4a4_linear_fused(const void* X, dq_dtype xt, const float* c, cons
  *  - The first call on each device looks up the array's device address with
  *    that device current (a host-side step); make that first call before any
  *    stream capture.
+ *  - The scratch used is the current device's: a non-null stream must belong
+ *    to the current device, else DQ_ERR_ARG before anything is enqueued.
  *  - Every call on a device shares the one array, which keeps the contents
  *    of the last call (each call clears what it uses first).  Calls whose
  *    execution overlaps on the GPU (different streams, no ordering between

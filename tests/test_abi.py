@@ -109,6 +109,11 @@ def test_invalid_arguments_rejected_without_launch(L):
                             3, None) == 1
     assert L.dq_w4a4_linear(fake, fake, fake, fake, fake, fake, None, fake, 1, 16, 128, 128,
                             3, None) == 1
+    # N must stay below 2^31 (the kernels index output columns with 32-bit ints)
+    assert L.dq_w4a4_linear(fake, fake, fake, fake, fake, fake, None, fake, 1, 16, 1 << 31, 256,
+                            3, None) == 1
+    assert L.dq_w4a4_linear_fused(fake, 1, None, fake, fake, fake, None, fake, 1, 16, 1 << 31,
+                                  256, 3, None) == 1
     odd = ctypes.c_void_p(0x1001)
     assert L.dq_w4a4_linear(odd, fake, fake, fake, fake, fake, None, fake, 1, 16, 128, 256,
                             3, None) == 1

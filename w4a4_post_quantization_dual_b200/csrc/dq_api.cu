@@ -223,7 +223,7 @@ int dq_w4a4_linear_fused(const void* X, dq_dtype xt, const float* c, const uint8
   if (!X || !B || !sB || !s_w || !Y || M <= 0 || N <= 0 || K <= 0 || !valid_dtype(yt) ||
       N % 128 || K % 256 || !aligned(X, 16) || !aligned(B, 16) || !aligned(sB, 16) ||
       !aligned(Y, 16) || !aligned(c, 4) || M > ((int64_t)1 << 31) - 128 ||
-      N > ((int64_t)1 << 31) || K > ((int64_t)1 << 20))
+      N > ((int64_t)1 << 31) - 128 || K > ((int64_t)1 << 20))
     return DQ_ERR_ARG;
   return dq::w4a4_linear_fused(X, c, B, sB, s_w, r_row, Y, yt, M, N, K, (cudaStream_t)stream);
 }
@@ -238,7 +238,7 @@ int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, cons
   if (!A || !sA || !B || !sB || !Y || M <= 0 || N <= 0 || K <= 0 || !valid_dtype(yt) ||
       N % 128 || K % 256 || !aligned(A, 16) || !aligned(B, 16) || !aligned(sA, 16) ||
       !aligned(sB, 16) || !aligned(Y, 16) || (f == DQ_NVFP4 && !s_tok) ||
-      M > ((int64_t)1 << 31) - 128 || N > ((int64_t)1 << 31) || K > ((int64_t)1 << 20))
+      M > ((int64_t)1 << 31) - 128 || N > ((int64_t)1 << 31) - 128 || K > ((int64_t)1 << 20))
     return DQ_ERR_ARG;
   return dq::w4a4_linear(A, sA, s_tok, B, sB, s_w, r_row, Y, yt, M, N, K, f,
                          (cudaStream_t)stream);

@@ -39,6 +39,14 @@ extern "C" int dq_solve_scales_noalloc(const void* W, dq_dtype wt, int64_t m, in
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return DQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DQ_ERR_UNSUPPORTED;
+  // The scratch address belongs to the current device, so the stream must be
+  // one of that device's streams (the legacy / per-thread default streams,
+  // passed as null, always are).
+  if (stream) {
+    int sdev = -1;
+    if (cudaStreamGetDevice((cudaStream_t)stream, &sdev) != cudaSuccess) return DQ_ERR_CUDA;
+    if (sdev != dev) return DQ_ERR_ARG;
+  }
   // First call on this device: resolve the array's device address with the
   // device current.  Later calls reuse it.
   std::call_once(g_setup_once[dev], [dev]() {
