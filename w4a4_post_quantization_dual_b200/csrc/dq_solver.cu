@@ -6,21 +6,15 @@
 //
 // With the row scale alpha being the format's native block scale, every
 // m x G column-block tile of W is an independent problem: r_ib touches only
-// tile b and every column lies in one tile.  One thread-block CLUSTER owns
-// one tile; its C CTAs split the tile's rows.  The whole iteration loop runs
-// on the device:
-//   row half-step   : each thread owns 8 contiguous columns of a row; the
-//                     G/8 threads of a row-block combine <W,R> and ||R||^2
-//                     with warp shuffles; the projected update is written to
-//                     shared memory.
-//   column half-step: per-thread column partials -> transposed shared-memory
-//                     reduction in fp64 -> per-CTA sums in cluster-visible
-//                     shared memory -> every CTA reads all C partial sums
-//                     over DSMEM in rank order (identical c in every CTA).
-// Each CTA stages its rows of the tile in shared memory once, converted to
-// fp32 (clusters of up to 16 CTAs keep the share <= 96 KB), and reads them
-// from there in every pass; tiles too tall for that stream their rows through the read-only
-// global path (L1 / L2 hits after the first round).  HBM sees W about once.
+// tile b and every column lies in one tile.  One CTA (or, for tiles taller
+// than one SM's shared memory holds, one thread-block cluster) owns one tile;
+// the whole iteration loop runs on the device with the tile resident in
+// shared memory.  Each thread owns 8 contiguous columns of a row per
+// row-step; the G/8 threads of a row-block are lanes of one warp.  A round
+// is one pass over the tile: per row-block the row update (warp shuffles
+// over the row-block's lanes) and, at the new row scale, the thread's column
+// partials; then the column update from the partials (warp reduce-scatter,
+// fp64 over warps, DSMEM over the cluster in rank order).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -34,11 +28,16 @@ namespace dq {
 
 template <int G>
 struct SolverShape {
-  static constexpr int OPB = G / 8;            // 8-column octets per row-block
-  static constexpr int NT = (G >= 64) ? 512 : 256;
+  static constexpr int OPB = G / 8;            // 8-column octets per row-block (lanes per row-block)
+  static constexpr int NT = 512;
   static constexpr int NW = NT / 32;
   static constexpr int RPW = 32 / OPB;         // rows per warp per step
   static constexpr int RPS = NW * RPW;         // rows per CTA per step
+  // column reduce-scatter over the RPW lanes that share an octet: LV shuffle
+  // levels, after which each lane holds VPL of the octet's 16 (num, den) sums
+  static constexpr int LV = RPW == 16 ? 4 : RPW == 8 ? 3 : RPW == 4 ? 2 : RPW == 2 ? 1 : 0;
+  static constexpr int VPL = 16 / RPW;
+  static_assert((1 << LV) == RPW && RPW <= 16, "reduce-scatter shape");
 };
 
 // Workspace layout (bytes): [0] u32 amax bits, [8] f64 ||W||^2, [16..] f64
@@ -112,40 +111,8 @@ __device__ __forceinline__ double ld_dsmem_f64(const double* local, uint32_t ran
   return v;
 }
 
-// Reduce V fp32 partials per thread over the CTA's threads that share an
-// octet.  Thread (oct, rslot) contributes acc[v] to value gv = oct*V + v.
-// out[gv] (shared, fp64) receives the CTA total, summed in a fixed order.
-template <int G, int V>
-__device__ __forceinline__ void cta_octet_reduce(const float* acc, float* scr, double* part,
-                                                 double* out) {
-  using S = SolverShape<G>;
-  constexpr int NV = S::OPB * V;           // values per CTA
-  constexpr int P = S::NT / NV;            // parts per value
-  constexpr int SPP = S::RPS / P;          // slots per part
-  static_assert(S::NT % NV == 0 && S::RPS % P == 0, "reduction shape");
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int oct = lane % S::OPB, rslot = warp * S::RPW + lane / S::OPB;
-#pragma unroll
-  for (int v = 0; v < V; ++v) scr[(oct * V + v) * (S::RPS + 1) + rslot] = acc[v];
-  __syncthreads();
-  {
-    const int gv = tid % NV, p = tid / NV;
-    double s = 0.0;
-    const float* src = scr + gv * (S::RPS + 1) + p * SPP;
-#pragma unroll 4
-    for (int i = 0; i < SPP; ++i) s += (double)src[i];
-    part[gv * P + p] = s;
-  }
-  __syncthreads();
-  if (tid < NV) {
-    double s = 0.0;
-    for (int p = 0; p < P; ++p) s += part[tid * P + p];
-    out[tid] = s;
-  }
-  __syncthreads();
-}
-
-// Same reduction for V fp64 partials per thread; scr (the float scratch of
+// Reduce V fp64 partials per thread over the CTA's threads that share an
+// octet (initialisation: column l1 norms); scr (the float scratch of
 // SolverSmem) is reused as OPB * V * (RPS + 1) doubles, V <= 8.
 template <int G, int V>
 __device__ __forceinline__ void cta_octet_reduce_f64(const double* acc, double* scr,
@@ -316,13 +283,25 @@ solve_init_kernel(SolveBatch bt, int64_t m, int steps, SolveOpts o) {
 // ---------------------------------------------------------------------------
 // Main kernel: r0 and T rounds of Algorithm 1, final error, outputs.
 //
-// WSMEM: the CTA's rows of the tile are staged once in shared memory and
-// every pass reads them from there; otherwise they are re-read through the
-// read-only global path (L1 / L2).  Element arithmetic uses the packed
+// One pass over the tile per round.  A row's update depends only on that
+// row, and the column update needs every row's new scale, so each row-block
+// is taken through the whole round at once: x -> y = x beta (used by both
+// half-steps of the round) -> codes at the old alpha -> <W_i, R_i>,
+// ||R_i||^2 over the row-block's lanes -> projected row scale -> codes at
+// the new alpha -> the thread's column partials <S_j, W_j>, ||S_j||^2.
+// After the pass the column partials are reduce-scattered over the lanes of
+// each warp that share an octet (shuffles), summed over the warps in fp64
+// and, when the tile spans a cluster, over its CTAs in rank order (DSMEM).
+//
+// Each CTA keeps its rows of the tile in shared memory in the weight's own
+// type for all T rounds (tiles too tall for that stream their rows through
+// the read-only global path); rows past m are zeros, so every loop runs the
+// same number of steps in every lane.  Element arithmetic uses the packed
 // fp32x2 instructions of sm_100 (each lane of a pair is an ordinary
 // correctly-rounded fp32 operation, so the quantiser argument
 // (w * beta) * alpha is bit-identical to the scalar definition).
-// TRACE: accumulate the reconstruction error for the MSE trace.
+// TRACE: accumulate the reconstruction error for the MSE trace (and, with
+// DQ_SOLVE_TRACE_CODES, the code change between rounds).
 // ---------------------------------------------------------------------------
 template <int F>
 struct RowProj {
@@ -376,60 +355,32 @@ __device__ __forceinline__ float2 grid2_packed(float2 z) {
   }
 }
 
-template <int F>
-__device__ __forceinline__ void grid8_packed(const float2* z, float2* q) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) q[k] = grid2_packed<F>(z[k]);
-}
-
-template <typename WT>
-__device__ __forceinline__ void unpack8(const WT* p, float2* x);
-template <>
-__device__ __forceinline__ void unpack8<__nv_bfloat16>(const __nv_bfloat16* p, float2* x) {
-  uint4 v = *reinterpret_cast<const uint4*>(p);
+__device__ __forceinline__ void bf16x8_to_f2(const uint4& v, float2* x) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-}
-template <>
-__device__ __forceinline__ void unpack8<float>(const float* p, float2* x) {
-  float4 a = reinterpret_cast<const float4*>(p)[0];
-  float4 b = reinterpret_cast<const float4*>(p)[1];
-  x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w);
-  x[2] = make_float2(b.x, b.y); x[3] = make_float2(b.z, b.w);
-}
-template <typename WT>
-__device__ __forceinline__ void unpack8_global(const WT* __restrict__ p, float2* x) {
-  if constexpr (sizeof(WT) == 2) {
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-  } else {
-    float4 a = __ldg(reinterpret_cast<const float4*>(p));
-    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w);
-    x[2] = make_float2(b.x, b.y); x[3] = make_float2(b.z, b.w);
-  }
+  for (int i = 0; i < 4; ++i)
+    x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
 }
 
-// Columns 2k, 2k+1 of an 8-column piece, as fp32.
-template <typename T>
-__device__ __forceinline__ float2 load_pair(const T* p, int k) {
-  if constexpr (sizeof(T) == 2) {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(p + 2 * k);
-    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-  } else {
-    return *reinterpret_cast<const float2*>(p + 2 * k);
-  }
-}
+// Fixed part of the main kernel's shared memory; the row-block scales of
+// the CTA's rows (r, alpha), the trace's previous alphas and the staged rows
+// follow it.
+template <int G>
+struct BcdSmem {
+  using S = SolverShape<G>;
+  float part[S::NW * 2 * G];   // per-warp column partials [warp][octet][16]; the exact
+                               // column pass reuses it as doubles [warp][octet][4]
+  double cpart[2][2 * G];      // this CTA's column totals, cluster-visible, double-buffered
+  float c_s[G], b_s[G];        // current c and beta = fl(1/c)
+  float b_old[G];              // beta before the column update (exact column pass)
+  float rtab[128], atab[128];  // NVFP4: r and alpha of every scale byte
+};
 
-// STG: 0 rows stream through the read-only global path, 1 rows staged in
-// shared memory as WT, 2 rows staged as fp32 (no unpacking in the passes).
-template <int F, int G, typename WT, int STG, bool TRACE>
-__global__ void __launch_bounds__(SolverShape<G>::NT, 2048 / SolverShape<G>::NT / 2)
+template <int F, int G, typename WT, bool STAGED, bool TRACE>
+__global__ void __launch_bounds__(SolverShape<G>::NT, 1)
 solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   using S = SolverShape<G>;
+  constexpr uint32_t FULL = 0xffffffffu;
   const int64_t n = bt.item[blockIdx.z].n;
   if ((int64_t)blockIdx.y >= n / G) return;   // whole clusters (they span x only)
   const WT* __restrict__ W = reinterpret_cast<const WT*>(bt.item[blockIdx.z].W);
@@ -438,24 +389,18 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   float* sT_io = bt.item[blockIdx.z].sT;
   SolverWs* ws = bt.item[blockIdx.z].ws;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  SolverSmem<G>& sm = *reinterpret_cast<SolverSmem<G>*>(smem_raw);
-  float* r_s = reinterpret_cast<float*>(smem_raw + sizeof(SolverSmem<G>));
-  float* a_s = r_s + (size_t)steps * S::RPS;
-  float* rtab = a_s + (size_t)steps * S::RPS;       // NVFP4: r and alpha of every scale byte
-  float* atab = rtab + 128;
-  constexpr bool WSMEM = STG != 0;
-  using ST = typename std::conditional<STG == 2, float, WT>::type;  // staged element type
-  ST* wch = reinterpret_cast<ST*>(atab + 128);      // staged rows
-  // TRACE: alpha of the previous round per row-step (code-change trace)
-  float* ap_s = reinterpret_cast<float*>(wch + (WSMEM ? (size_t)steps * S::RPS * G : 0));
+  BcdSmem<G>& sm = *reinterpret_cast<BcdSmem<G>*>(smem_raw);
+  const int rows_cta = steps * S::RPS;
+  float2* ra_s = reinterpret_cast<float2*>(smem_raw + ((sizeof(BcdSmem<G>) + 15) & ~(size_t)15));
+  float* ap_s = reinterpret_cast<float*>(ra_s + rows_cta);        // TRACE only
+  WT* wch = reinterpret_cast<WT*>(ap_s + (TRACE ? rows_cta : 0));  // staged rows
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int oct = lane % S::OPB, rslot = warp * S::RPW + lane / S::OPB;
+  const int oct = lane % S::OPB, rr = lane / S::OPB, rslot = warp * S::RPW + rr;
   const uint32_t rank = cluster_ctarank(), C = gridDim.x;
   const int64_t b = blockIdx.y, nb = n / G;
   const int64_t col0 = b * G + oct * 8;
-  const int64_t row0 = (int64_t)rank * steps * S::RPS;
-  const int rows_cta = steps * S::RPS;
+  const int64_t row0 = (int64_t)rank * rows_cta;
 
   const bool alpha_only = o.flags & SOLVE_ALPHA_ONLY, beta_only = o.flags & SOLVE_BETA_ONLY;
   const bool keep_s = F == NVFP4 && (o.flags & SOLVE_KEEP_S);
@@ -469,60 +414,56 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
     }
     if (tid < 128) {
       float rv = __fmul_rn(sT, ue4m3_value(tid ? (uint32_t)tid : 1u));
-      rtab[tid] = rv;
-      atab[tid] = __frcp_rn(rv);
+      sm.rtab[tid] = rv;
+      sm.atab[tid] = __frcp_rn(rv);
     }
   }
   if (rank == 0 && b == 0 && tid == 0 && !keep_s) *sT_io = sT;
   const float inv_sT = __frcp_rn(sT);
 
-  if constexpr (STG == 2) {
-    // stage rows [row0, row0 + rows_cta) x columns [b*G, b*G+G) (zeros past
-    // m) as fp32, so the passes below read values without unpacking
-    constexpr int PPR = G / 8;                        // 8-element pieces per row
+  if constexpr (STAGED) {
+    // rows [row0, row0 + rows_cta) x columns [b*G, b*G + G), zeros past m,
+    // in 16-byte pieces.  bf16: row-major.  fp32: two planes (elements 0-3
+    // and 4-7 of every octet), so that a warp's 16-byte reads are contiguous.
+    constexpr int PPR = G * (int)sizeof(WT) / 16;     // pieces per row
     for (int p = tid; p < rows_cta * PPR; p += S::NT) {
       const int lr = p / PPR, pc = p % PPR;
       const int64_t i = row0 + lr;
-      float2 v[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                     make_float2(0.f, 0.f)};
-      if (i < m) unpack8_global<WT>(W + i * n + b * G + pc * 8, v);
-      float4* dst = reinterpret_cast<float4*>(wch + (size_t)lr * G + pc * 8);
-      dst[0] = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
-      dst[1] = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
-    }
-    __syncthreads();
-  } else if constexpr (STG == 1) {
-    // stage the rows in their own type (16-byte pieces, zeros past m)
-    constexpr int V = 16 / sizeof(WT);
-    constexpr int PPR = G / V;
-    for (int p = tid; p < rows_cta * PPR; p += S::NT) {
-      const int lr = p / PPR, pc = p % PPR;
-      const int64_t i = row0 + lr;
-      uint4 v = make_uint4(0, 0, 0, 0);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (i < m) v = __ldg(reinterpret_cast<const uint4*>(W + i * n + b * G) + pc);
-      reinterpret_cast<uint4*>(wch + (size_t)lr * G)[pc] = v;
+      if constexpr (sizeof(WT) == 2)
+        reinterpret_cast<uint4*>(wch)[p] = v;
+      else
+        reinterpret_cast<uint4*>(wch)[(pc & 1) * rows_cta * S::OPB + lr * S::OPB + (pc >> 1)] = v;
     }
-    __syncthreads();
   }
-  // this thread's row-steps s cover rows row0 + s*RPS + rslot; those below m
-  // are s < s_end.  Per-thread bases and constant strides for the hot loops.
-  const int64_t first_row = row0 + rslot;
-  const int s_end = first_row >= m ? 0
-                    : (int)((m - first_row + S::RPS - 1) / S::RPS) < steps
-                          ? (int)((m - first_row + S::RPS - 1) / S::RPS)
-                          : steps;
-  const ST* xsm = WSMEM ? wch + (size_t)rslot * G + oct * 8 : nullptr;
-  const WT* xgl = WSMEM ? nullptr : W + first_row * n + col0;
-  constexpr int XSM_STEP = S::RPS * G;
-  const int64_t xgl_step = (int64_t)S::RPS * n;
-  float* rsl = r_s + rslot;
-  float* asl = a_s + rslot;
-  float* apl = ap_s + rslot;
-  const bool trace_codes = TRACE && (o.flags & SOLVE_TRACE_CODES);
-  float2 beta_prev[4];   // TRACE: beta of the previous round
-  auto load_x = [&](int s, float2* x) {
-    if constexpr (WSMEM) unpack8<ST>(xsm + s * XSM_STEP, x);
-    else unpack8_global<WT>(xgl + s * xgl_step, x);
+  // elements 8 oct .. 8 oct + 7 of CTA row lr, as fp32 pairs
+  auto load_x = [&](int lr, float2* x) {
+    if constexpr (STAGED) {
+      if constexpr (sizeof(WT) == 2) {
+        bf16x8_to_f2(reinterpret_cast<const uint4*>(wch)[lr * S::OPB + oct], x);
+      } else {
+        const float4 a = reinterpret_cast<const float4*>(wch)[lr * S::OPB + oct];
+        const float4 c = reinterpret_cast<const float4*>(wch)[rows_cta * S::OPB + lr * S::OPB + oct];
+        x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w);
+        x[2] = make_float2(c.x, c.y); x[3] = make_float2(c.z, c.w);
+      }
+    } else {
+      const int64_t i = row0 + lr;
+      if (i < m) {
+        if constexpr (sizeof(WT) == 2) {
+          bf16x8_to_f2(__ldg(reinterpret_cast<const uint4*>(W + i * n + col0)), x);
+        } else {
+          const float4 a = __ldg(reinterpret_cast<const float4*>(W + i * n + col0));
+          const float4 c = __ldg(reinterpret_cast<const float4*>(W + i * n + col0) + 1);
+          x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w);
+          x[2] = make_float2(c.x, c.y); x[3] = make_float2(c.z, c.w);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = make_float2(0.f, 0.f);
+      }
+    }
   };
 
   float2 cc[4], beta[4];
@@ -531,165 +472,164 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
     cc[k] = make_float2(c_io[col0 + 2 * k], c_io[col0 + 2 * k + 1]);
     beta[k] = make_float2(__frcp_rn(cc[k].x), __frcp_rn(cc[k].y));
   }
-  if (tid < G) {   // the current beta also in shared memory (exact column pass)
+  if (tid < G) {
     sm.c_s[tid] = c_io[b * G + tid];
     sm.b_s[tid] = __frcp_rn(sm.c_s[tid]);
   }
+  __syncthreads();   // staged rows, scale tables
 
   // r0: the caller's scales projected onto F_alpha (rows past m take the
   // projection of 1), or else the format-native absmax scale of
-  // W diag(c0)^-1 per row-block (IEEE arithmetic: the same fp32 decisions
-  // as the oracle's initialisation).  Each r0 entry is read by the thread
-  // that writes the same entry of r at the end (r0 may alias r).
-  if (o.r0 != nullptr) {
-    if (oct == 0)
-      for (int s = 0; s < steps; ++s) {
-        const float u = s < s_end ? o.r0[(first_row + (int64_t)s * S::RPS) * nb + b] : 1.0f;
-        const float rv = proj_alpha<F>(u, sT);
-        rsl[s * S::RPS] = rv;
-        asl[s * S::RPS] = __frcp_rn(rv);
-      }
-  } else
+  // W diag(c0)^-1 per row-block (the same fp32 decisions as the oracle's
+  // initialisation).  Each r0 entry is read by the lane that writes the same
+  // entry of r at the end (r0 may alias r).
   for (int s = 0; s < steps; ++s) {
-    float a = 0.0f;
-    if (s < s_end) {
+    const int lr = s * S::RPS + rslot;
+    const int64_t i = row0 + lr;
+    float rv;
+    if (o.r0 != nullptr) {
+      rv = proj_alpha<F>((oct == 0 && i < m) ? o.r0[i * nb + b] : 1.0f, sT);
+    } else {
       float2 x[4];
-      load_x(s, x);
+      load_x(lr, x);
+      float a = 0.0f;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        float2 p = __fmul2_rn(x[k], beta[k]);
+        const float2 p = __fmul2_rn(x[k], beta[k]);
         a = fmaxf(a, fmaxf(fabsf(p.x), fabsf(p.y)));
       }
-    }
 #pragma unroll
-    for (int o = 1; o < S::OPB; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if (oct == 0) {
-      float r0 = rtn_block_scale<F>(a, sT);
-      rsl[s * S::RPS] = r0;
-      asl[s * S::RPS] = __frcp_rn(r0);
+      for (int d = 1; d < S::OPB; d <<= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, d));
+      rv = rtn_block_scale<F>(a, sT);
     }
+    if (oct == 0) ra_s[lr] = make_float2(rv, __frcp_rn(rv));
   }
   __syncwarp();
 
-  int xb = 0;  // exchange buffer of the next column exchange
-  // column window: 2 * steps + 4 ulps, + 4 for S = r q rounded to fp32
-  const uint32_t col_win = 2u * (uint32_t)steps + 8u;
+  int xb = 0;  // exchange buffer of the next cluster exchange
+  // column window: the per-thread fp32 chain (steps terms) and the fp32
+  // reduce-scatter levels, 2 * depth + 4 ulps, + 4 for S = r q in fp32
+  const uint32_t col_win = 2u * (uint32_t)(steps + S::LV) + 8u;
+  const bool trace_codes = TRACE && (o.flags & SOLVE_TRACE_CODES);
+  float2 beta_prev[4];   // TRACE: beta of the previous round
+#pragma unroll
+  for (int k = 0; k < 4; ++k) beta_prev[k] = beta[k];
   for (int t = 0; t <= T; ++t) {
-    // ---- row half-step (t < T) / error at the current scales ----
+    const bool do_row = t < T && !beta_only;
+    const bool do_col = t < T && !alpha_only;
+    if (!do_row && !do_col && !TRACE) break;
     float e_acc = 0.0f;
     float2 qn2 = make_float2(0.f, 0.f), qd2 = qn2;   // TRACE: code-change sums
-    bool any_tie = false;
-    if ((t < T && !beta_only) || TRACE) {
-      for (int s = 0; s < steps; ++s) {
-        const bool valid = s < s_end;
+    float2 accn[4], accd[4];                          // column partials (num, den) per pair
+#pragma unroll
+    for (int k = 0; k < 4; ++k) accn[k] = accd[k] = make_float2(0.f, 0.f);
+
+    for (int s = 0; s < steps; ++s) {
+      const int lr = s * S::RPS + rslot;
+      float2 x[4], y[4];
+      load_x(lr, x);
+      const float2 ra = ra_s[lr];
+      float rn = ra.x, an = ra.y;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) y[k] = __fmul2_rn(x[k], beta[k]);
+      if (do_row || TRACE) {
+        // ---- row half-step at the current scales (and the error there) ----
+        const float2 a2 = make_float2(ra.y, ra.y);
         float2 num2 = make_float2(0.f, 0.f), den2 = num2, err2 = num2;
-        const float rr = rsl[s * S::RPS], alpha = asl[s * S::RPS];
-        const float alpha_prev = (TRACE && t > 0) ? apl[s * S::RPS] : 0.0f;
-        if (valid) {
-          float2 x[4], z[4], q[4];
-          load_x(s, x);
-          const float2 a2 = make_float2(alpha, alpha);
+        float2 R[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) z[k] = __fmul2_rn(__fmul2_rn(x[k], beta[k]), a2);
-          grid8_packed<F>(z, q);
+        for (int k = 0; k < 4; ++k) R[k] = __fmul2_rn(grid2_packed<F>(__fmul2_rn(y[k], a2)), cc[k]);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float2 R = __fmul2_rn(q[k], cc[k]);
-            num2 = __ffma2_rn(x[k], R, num2);
-            den2 = __ffma2_rn(R, R, den2);
-            if constexpr (TRACE) {
-              float2 d = __ffma2_rn(make_float2(-rr, -rr), R, x[k]);
-              err2 = __ffma2_rn(d, d, err2);
-            }
-          }
+        for (int k = 0; k < 4; ++k) {
+          num2 = __ffma2_rn(x[k], R[k], num2);
+          den2 = __ffma2_rn(R[k], R[k], den2);
           if constexpr (TRACE) {
-            // Qhat(t) - Qhat(t-1): the codes at the previous round's scales
-            if (trace_codes && t > 0) {
-              const float2 ap2 = make_float2(alpha_prev, alpha_prev);
+            const float2 d = __ffma2_rn(make_float2(-ra.x, -ra.x), R[k], x[k]);
+            err2 = __ffma2_rn(d, d, err2);
+          }
+        }
+        if constexpr (TRACE) {
+          // Qhat(t) - Qhat(t-1): the codes at the previous round's scales
+          if (trace_codes && t > 0) {
+            const float ap = ap_s[lr];
+            const float2 ap2 = make_float2(ap, ap);
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const float2 qp = grid2_packed<F>(__fmul2_rn(__fmul2_rn(x[k], beta_prev[k]), ap2));
-                const float2 d = make_float2(q[k].x - qp.x, q[k].y - qp.y);
-                qn2 = __ffma2_rn(d, d, qn2);
-                qd2 = __ffma2_rn(qp, qp, qd2);
-              }
+            for (int k = 0; k < 4; ++k) {
+              const float2 q = grid2_packed<F>(__fmul2_rn(y[k], a2));
+              const float2 qp = grid2_packed<F>(__fmul2_rn(__fmul2_rn(x[k], beta_prev[k]), ap2));
+              const float2 d = make_float2(q.x - qp.x, q.y - qp.y);
+              qn2 = __ffma2_rn(d, d, qn2);
+              qd2 = __ffma2_rn(qp, qp, qd2);
             }
           }
         }
         float num = num2.x + num2.y, den = den2.x + den2.y, err = err2.x + err2.y;
 #pragma unroll
-        for (int o = 1; o < S::OPB; o <<= 1) {
-          num += __shfl_xor_sync(0xffffffffu, num, o);
-          den += __shfl_xor_sync(0xffffffffu, den, o);
-          if constexpr (TRACE) err += __shfl_xor_sync(0xffffffffu, err, o);
+        for (int d = 1; d < S::OPB; d <<= 1) {
+          num += __shfl_xor_sync(FULL, num, d);
+          den += __shfl_xor_sync(FULL, den, d);
+          if constexpr (TRACE) err += __shfl_xor_sync(FULL, err, d);
         }
-        if (TRACE && oct == 0) e_acc += err;
-        // the alpha these codes were taken with serves the next round's trace
-        if (TRACE && trace_codes && oct == 0) apl[s * S::RPS] = alpha;
-        if (t < T && !beta_only) {
+        if constexpr (TRACE) {
+          if (oct == 0) e_acc += err;
+          if (trace_codes) {   // the alpha these codes were taken with serves the next round
+            __syncwarp();
+            if (oct == 0) ap_s[lr] = ra.y;
+          }
+        }
+        if (do_row) {
           const float u = den > 0.0f ? __fdividef(num, den) : 1.0f;
           // all lanes of a row-block hold the same sums, hence the same flag
-          const bool tie = den > 0.0f && near_tie_alpha<F>(u, inv_sT, ROW_TIE_WIN);  // den = 0 past m
-          any_tie |= tie;
-          if (oct == 0 && valid) {
-            float rn, an;
-            RowProj<F>::apply(u, inv_sT, rtab, atab, sT, rn, an);
-            // exact update pending: r holds -alpha (the alpha it needs)
-            rsl[s * S::RPS] = tie ? -alpha : rn;
-            asl[s * S::RPS] = an;
-          }
-        }
-      }
-      // rare: row-blocks whose update lies near a projection boundary get it
-      // from exact sums -- <W_i, R_i> and ||R_i||^2 in fp64 (x * R is exact
-      // in fp64, R = q * c exact in fp32), the quotient rounded once to fp32
-      if (t < T && !beta_only && __any_sync(0xffffffffu, any_tie)) {
-        __syncwarp();
-        for (int s = 0; s < steps; ++s) {
-          const bool need = rsl[s * S::RPS] < 0.0f;   // the same word for the whole row-block
-          if (!__any_sync(0xffffffffu, need)) continue;
-          double dn = 0.0, dd = 0.0;
-          if (need) {   // one column pair at a time (few live registers)
-            const float alpha = -rsl[s * S::RPS];
-            const float2 a2 = make_float2(alpha, alpha);
+          const bool tie = den > 0.0f && near_tie_alpha<F>(u, inv_sT, ROW_TIE_WIN);
+          RowProj<F>::apply(u, inv_sT, sm.rtab, sm.atab, sT, rn, an);
+          if (__any_sync(FULL, tie)) {
+            // rare: the update lies near a projection boundary -- take it from
+            // exact sums, <W_i, R_i> and ||R_i||^2 in fp64 (x R is exact in
+            // fp64, R = q c exact in fp32), the quotient rounded once to fp32
+            double dn = 0.0, dd = 0.0;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              float2 xp;
-              if constexpr (WSMEM) xp = load_pair<ST>(xsm + s * XSM_STEP, k);
-              else xp = load_pair<WT>(xgl + s * xgl_step, k);
-              const float2 q = grid2_packed<F>(__fmul2_rn(__fmul2_rn(xp, beta[k]), a2));
-              const float2 R = __fmul2_rn(q, cc[k]);
-              dn = fma((double)xp.x, (double)R.x, dn);
-              dn = fma((double)xp.y, (double)R.y, dn);
-              dd = fma((double)R.x, (double)R.x, dd);
-              dd = fma((double)R.y, (double)R.y, dd);
+              const float2 Rk = __fmul2_rn(grid2_packed<F>(__fmul2_rn(y[k], a2)), cc[k]);
+              dn = fma((double)x[k].x, (double)Rk.x, dn);
+              dn = fma((double)x[k].y, (double)Rk.y, dn);
+              dd = fma((double)Rk.x, (double)Rk.x, dd);
+              dd = fma((double)Rk.y, (double)Rk.y, dd);
+            }
+#pragma unroll
+            for (int d = 1; d < S::OPB; d <<= 1) {
+              dn += __shfl_xor_sync(FULL, dn, d);
+              dd += __shfl_xor_sync(FULL, dd, d);
+            }
+            if (tie) {
+              rn = proj_alpha<F>((float)(dn / dd), sT);
+              an = __frcp_rn(rn);
             }
           }
+          if (oct == 0) ra_s[lr] = make_float2(rn, an);
+        }
+      }
+      if (do_col) {
+        // ---- column partials with the new row scale ----
+        const float2 a2 = make_float2(an, an), r2 = make_float2(rn, rn);
 #pragma unroll
-          for (int o = 1; o < S::OPB; o <<= 1) {
-            dn += __shfl_xor_sync(0xffffffffu, dn, o);
-            dd += __shfl_xor_sync(0xffffffffu, dd, o);
-          }
-          __syncwarp();
-          if (need && oct == 0) {
-            const float rn = proj_alpha<F>((float)(dn / dd), sT);
-            rsl[s * S::RPS] = rn;
-            asl[s * S::RPS] = __frcp_rn(rn);
-          }
+        for (int k = 0; k < 4; ++k) {
+          const float2 Sv = __fmul2_rn(r2, grid2_packed<F>(__fmul2_rn(y[k], a2)));
+          accn[k] = __ffma2_rn(Sv, x[k], accn[k]);
+          accd[k] = __ffma2_rn(Sv, Sv, accd[k]);
         }
       }
     }
     if constexpr (TRACE) {
 #pragma unroll
-      for (int o = 16; o; o >>= 1) e_acc += __shfl_xor_sync(0xffffffffu, e_acc, o);
+      for (int d = 16; d; d >>= 1) e_acc += __shfl_xor_sync(FULL, e_acc, d);
       if (lane == 0) atomicAdd(&ws->err[t], (double)e_acc);
       if (trace_codes) {
         // sums of this warp; qnum / qden follow err[T+1] in the workspace
         float qn = qn2.x + qn2.y, qd = qd2.x + qd2.y;
 #pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          qn += __shfl_xor_sync(0xffffffffu, qn, o);
-          qd += __shfl_xor_sync(0xffffffffu, qd, o);
+        for (int d = 16; d; d >>= 1) {
+          qn += __shfl_xor_sync(FULL, qn, d);
+          qd += __shfl_xor_sync(FULL, qd, d);
         }
         if (lane == 0 && t > 0) {
           atomicAdd(&ws->err[(T + 1) + t], (double)qn);
@@ -699,73 +639,86 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
         for (int k = 0; k < 4; ++k) beta_prev[k] = beta[k];
       }
     }
-    if (t == T) break;
-    __syncwarp();
-    if (alpha_only) continue;
+    if (!do_col) continue;
 
-    // ---- column half-step: re-quantise with the new r, update c ----
-    float2 acc[8];
-#pragma unroll
-    for (int v = 0; v < 8; ++v) acc[v] = make_float2(0.f, 0.f);
-    for (int s = 0; s < s_end; ++s) {
-      {
-        const float rr = rsl[s * S::RPS], alpha = asl[s * S::RPS];
-        float2 x[4], z[4], q[4];
-        load_x(s, x);
-        const float2 a2 = make_float2(alpha, alpha), r2 = make_float2(rr, rr);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) z[k] = __fmul2_rn(__fmul2_rn(x[k], beta[k]), a2);
-        grid8_packed<F>(z, q);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          float2 Sv = __fmul2_rn(r2, q[k]);
-          acc[2 * k] = __ffma2_rn(Sv, x[k], acc[2 * k]);        // (num_j, num_j+1)
-          acc[2 * k + 1] = __ffma2_rn(Sv, Sv, acc[2 * k + 1]);  // (den_j, den_j+1)
-        }
-      }
-    }
-    // reorder to [column][num, den] for the reduction
-    float accv[16];
+    // ---- column half-step: c_j <- Pi(<S_j, W_j> / ||S_j||^2) ----
+    // v[2c], v[2c+1] = (num, den) of column c of the octet; reduce-scatter
+    // over the RPW lanes sharing the octet: after LV levels each lane holds
+    // the warp's sums of VPL of the 16 values, starting at `base`
+    float v[16];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      accv[4 * k + 0] = acc[2 * k].x;       // num of column 2k
-      accv[4 * k + 1] = acc[2 * k + 1].x;   // den of column 2k
-      accv[4 * k + 2] = acc[2 * k].y;       // num of column 2k+1
-      accv[4 * k + 3] = acc[2 * k + 1].y;   // den of column 2k+1
+      v[4 * k + 0] = accn[k].x;
+      v[4 * k + 1] = accd[k].x;
+      v[4 * k + 2] = accn[k].y;
+      v[4 * k + 3] = accd[k].y;
     }
-    // the exchange buffer alternates with every exchange: a CTA writes
-    // buffer xb only after all peers passed the barrier that follows their
-    // last reads of it
-    cta_octet_reduce<G, 16>(accv, sm.scr, sm.part, sm.cpart[xb]);
-    cluster_sync_all();
-    // column j's total (num, den) over the cluster, summed in rank order;
-    // four CTAs' partials in flight at a time
-    auto cluster_sum = [&](int j, double& sn, double& sd) {
-      const int o = j >> 3, k = j & 7;
-      sn = 0.0;
-      sd = 0.0;
-      for (int q0 = 0; q0 < (int)C; q0 += 4) {
-        double pn[4], pd[4];
+    int base = 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (q0 + u < (int)C) {
-            pn[u] = ld_dsmem_f64(&sm.cpart[xb][o * 16 + 2 * k], (uint32_t)(q0 + u));
-            pd[u] = ld_dsmem_f64(&sm.cpart[xb][o * 16 + 2 * k + 1], (uint32_t)(q0 + u));
-          }
+    for (int l = 0; l < S::LV; ++l) {
+      const int half = 16 >> (l + 1);
+      const bool up = (lane & (S::OPB << l)) != 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (q0 + u < (int)C) {
-            sn += pn[u];
-            sd += pd[u];
-          }
+      for (int i = 0; i < half; ++i) {
+        const float send = up ? v[i] : v[i + half];
+        const float keep = up ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, S::OPB << l);
       }
-    };
-    // projected update, written at once; a column near a projection
-    // boundary is redone below from exact sums
+      base += up ? half : 0;
+    }
+#pragma unroll
+    for (int i = 0; i < S::VPL; ++i) sm.part[(warp * S::OPB + oct) * 16 + base + i] = v[i];
+    __syncthreads();
+    double sn = 0.0, sd = 0.0;
+    if (tid < G) {   // column tid: its warps' sums in fp64, warp order
+      const float* p = sm.part + (tid >> 3) * 16 + 2 * (tid & 7);
+      float pn[S::NW], pd[S::NW];
+#pragma unroll
+      for (int w = 0; w < S::NW; ++w) {
+        pn[w] = p[w * 2 * G];
+        pd[w] = p[w * 2 * G + 1];
+      }
+#pragma unroll
+      for (int w = 0; w < S::NW; ++w) {
+        sn += (double)pn[w];
+        sd += (double)pd[w];
+      }
+    }
+    if (C > 1) {
+      // the CTA totals go to the cluster; every CTA sums all of them in rank
+      // order (identical c in every CTA).  The buffer alternates with every
+      // exchange: a CTA writes buffer xb only after all peers passed the
+      // barrier that follows their last reads of it.
+      if (tid < G) {
+        sm.cpart[xb][2 * tid] = sn;
+        sm.cpart[xb][2 * tid + 1] = sd;
+      }
+      cluster_sync_all();
+      if (tid < G) {
+        sn = 0.0;
+        sd = 0.0;
+        for (int q0 = 0; q0 < (int)C; q0 += 4) {
+          double pn[4], pd[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (q0 + u < (int)C) {
+              pn[u] = ld_dsmem_f64(&sm.cpart[xb][2 * tid], (uint32_t)(q0 + u));
+              pd[u] = ld_dsmem_f64(&sm.cpart[xb][2 * tid + 1], (uint32_t)(q0 + u));
+            }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (q0 + u < (int)C) {
+              sn += pn[u];
+              sd += pd[u];
+            }
+        }
+      }
+      xb ^= 1;
+    }
+    // projected update; a column near a projection boundary is redone below
+    // from exact sums
     bool ctie = false;
     if (tid < G) {
-      double sn, sd;
-      cluster_sum(tid, sn, sd);
       const float cu = (sd > 0.0) ? (float)(sn / sd) : 1.0f;
       ctie = sd > 0.0 && near_tie_beta<F>(cu, col_win);
       const float cn = proj_beta<F>(cu);
@@ -773,50 +726,63 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
       sm.c_s[tid] = cn;
       sm.b_s[tid] = __frcp_rn(cn);
     }
-    xb ^= 1;
-    // every CTA of the cluster sums the same partials in the same order, so
-    // the flag is cluster-uniform and the exact pass below (with its cluster
+    // every CTA of the cluster sums the same totals in the same order, so the
+    // flag is cluster-uniform and the exact pass below (with its cluster
     // barrier) runs in all of them or in none
     if (__syncthreads_or(ctie)) {
-      // rare: exact fp64 column sums of the tile
-      // -- per thread <S_j, W_j> and ||S_j||^2 for one column pair of its
-      // octet at a time, S = r q formed in fp64 (exact) and S * S rounded
-      // once as in a plain fp64 loop, reduced over the CTA in fp64 into the
-      // exchange layout of the fast pass (the old beta from shared memory,
-      // the pair loaded on its own: no register array is indexed by kp)
+      // rare: exact fp64 column sums of the tile -- per thread <S_j, W_j> and
+      // ||S_j||^2 for one column pair of its octet at a time, S = r q formed
+      // in fp64 (exact) and S * S rounded once as in a plain fp64 loop, then
+      // over the octet's lanes, the warps (warp order) and the CTAs (rank order)
+      double* xpart = reinterpret_cast<double*>(sm.part);   // [warp][octet][4]
 #pragma unroll 1
       for (int kp = 0; kp < 4; ++kp) {
         double a4[4] = {0.0, 0.0, 0.0, 0.0};
         const float2 bp = make_float2(sm.b_old[oct * 8 + 2 * kp], sm.b_old[oct * 8 + 2 * kp + 1]);
-        for (int s = 0; s < s_end; ++s) {
-          const float rr = rsl[s * S::RPS], alpha = asl[s * S::RPS];
-          float2 xp;
-          if constexpr (WSMEM) xp = load_pair<ST>(xsm + s * XSM_STEP, kp);
-          else xp = load_pair<WT>(xgl + s * xgl_step, kp);
-          const float2 q = grid2_packed<F>(__fmul2_rn(__fmul2_rn(xp, bp), make_float2(alpha, alpha)));
-          const double s0 = (double)rr * (double)q.x, s1 = (double)rr * (double)q.y;
+        for (int s = 0; s < steps; ++s) {
+          const int lr = s * S::RPS + rslot;
+          const float2 ra = ra_s[lr];
+          float2 x[4];
+          load_x(lr, x);
+          float2 xp = x[0];
+#pragma unroll
+          for (int k = 1; k < 4; ++k) xp = (k == kp) ? x[k] : xp;
+          const float2 q = grid2_packed<F>(__fmul2_rn(__fmul2_rn(xp, bp), make_float2(ra.y, ra.y)));
+          const double s0 = (double)ra.x * (double)q.x, s1 = (double)ra.x * (double)q.y;
           a4[0] = __dadd_rn(a4[0], __dmul_rn(s0, (double)xp.x));
           a4[1] = __dadd_rn(a4[1], __dmul_rn(s0, s0));
           a4[2] = __dadd_rn(a4[2], __dmul_rn(s1, (double)xp.y));
           a4[3] = __dadd_rn(a4[3], __dmul_rn(s1, s1));
         }
-        cta_octet_reduce_f64<G, 4>(a4, reinterpret_cast<double*>(sm.scr), sm.part, sm.l1);
-        if (tid < S::OPB * 4) sm.cpart[xb][(tid >> 2) * 16 + 4 * kp + (tid & 3)] = sm.l1[tid];
+#pragma unroll
+        for (int l = 0; l < S::LV; ++l)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a4[i] += __shfl_xor_sync(FULL, a4[i], S::OPB << l);
+        if (rr == 0)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xpart[(warp * S::OPB + oct) * 4 + i] = a4[i];
+        __syncthreads();
+        if (tid < S::OPB * 4) {
+          double acc = 0.0;
+          for (int w = 0; w < S::NW; ++w) acc += xpart[(w * S::OPB + (tid >> 2)) * 4 + (tid & 3)];
+          // value i of the pair: (num, den) of column 2 kp, then of 2 kp + 1
+          const int j = (tid >> 2) * 8 + 2 * kp + ((tid & 3) >> 1);
+          sm.cpart[xb][2 * j + (tid & 1)] = acc;
+        }
         __syncthreads();
       }
-      cluster_sync_all();
+      if (C > 1) cluster_sync_all();
       if (ctie) {   // rank order, one CTA at a time (rare path)
-        const int o = tid >> 3, k = tid & 7;
-        double sn = 0.0, sd = 0.0;
+        double en = 0.0, ed = 0.0;
         for (uint32_t q = 0; q < C; ++q) {
-          sn += ld_dsmem_f64(&sm.cpart[xb][o * 16 + 2 * k], q);
-          sd += ld_dsmem_f64(&sm.cpart[xb][o * 16 + 2 * k + 1], q);
+          en += ld_dsmem_f64(&sm.cpart[xb][2 * tid], q);
+          ed += ld_dsmem_f64(&sm.cpart[xb][2 * tid + 1], q);
         }
-        const float cn = proj_beta<F>((float)(sn / sd));
+        const float cn = proj_beta<F>((float)(en / ed));
         sm.c_s[tid] = cn;
         sm.b_s[tid] = __frcp_rn(cn);
       }
-      xb ^= 1;
+      if (C > 1) xb ^= 1;
       __syncthreads();
     }
 #pragma unroll
@@ -827,10 +793,12 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   }
 
   // outputs
-  for (int s = 0; s < s_end; ++s)
-    if (oct == 0) r_out[(first_row + (int64_t)s * S::RPS) * nb + b] = rsl[s * S::RPS];
+  for (int s = 0; s < steps; ++s) {
+    const int lr = s * S::RPS + rslot;
+    if (oct == 0 && row0 + lr < m) r_out[(row0 + lr) * nb + b] = ra_s[lr].x;
+  }
   if (rank == 0 && tid < G && T > 0 && !alpha_only) c_io[b * G + tid] = sm.c_s[tid];
-  cluster_sync_all();  // no CTA leaves while a peer may still read its cpart
+  if (C > 1) cluster_sync_all();  // no CTA leaves while a peer may still read its cpart
 }
 
 // mse_trace[t] = err[t] / ||W||^2; with the code-change trace also
@@ -850,41 +818,36 @@ __global__ void solve_finalize_kernel(const SolverWs* ws, int T, double* mse_tra
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-// trace: one more float per row-step (the previous round's alpha, for the
-// code-change trace), after the staged rows.
+constexpr size_t SOLVER_SMEM_MAX = 227 * 1024;
+
+// Dynamic shared memory of the main kernel: the fixed part, (r, alpha) per
+// row, the previous alpha per row (trace), and the staged rows
+// (elem_bytes = 0: streamed).
 template <int G>
-static size_t solver_smem_bytes(int steps, size_t staged_elem_bytes, bool trace = false) {
+static size_t solver_smem_bytes(int steps, size_t elem_bytes, bool trace) {
   const size_t rows = (size_t)steps * SolverShape<G>::RPS;
-  return sizeof(SolverSmem<G>) + 2 * sizeof(float) * rows + 2 * 128 * sizeof(float) +
-         rows * G * staged_elem_bytes + (trace ? sizeof(float) * rows : 0);
+  return ((sizeof(BcdSmem<G>) + 15) & ~(size_t)15) + rows * 8 + (trace ? rows * 4 : 0) +
+         rows * G * elem_bytes;
 }
 
 // Launch geometry: the tile's rows are split over C CTAs of one cluster,
-// `steps` row-steps of RPS rows per CTA.  Prefer clusters of 8, staging the
-// CTA's rows in shared memory as fp32, else in the weight's own type
-// (<= 96 KB of rows); otherwise, for G = 16 only, clusters of 16 with the
-// same staging; otherwise stream the rows through the read-only global
-// path with clusters of 8.  stg: 2 fp32, 1 own type, 0 global.
-// Measured (B200, T = 50, bf16): 14336 x 4096 NVFP4 6.1 ms with fp32 rows
-// in 16 CTAs, 4.1 ms with bf16 rows in 8; 14336 x 4096 MXFP4 5.0 ms staged
-// in 16 CTAs, 4.0 ms streamed by 8; 27648 x 5120 NVFP4 12.0 ms staged in 16,
-// 13.2 ms streamed by 8.  Larger staging at one CTA per SM was slower in
-// every case.
+// `steps` row-steps of RPS rows per CTA.  The fewest CTAs whose rows fit in
+// shared memory in the weight's own type (one CTA per SM, so a tile that fits
+// one SM needs no cluster exchange); tiles taller than 16 CTAs hold stream
+// their rows through the read-only global path with clusters of up to 8.
+// The sizes are those of the traced variant, so that a trace never changes
+// the geometry.
 template <int G, typename WT>
 static void solver_geometry(int64_t m, int& steps, int& C, int& stg) {
   using S = SolverShape<G>;
-  for (int cmax : {8, 16}) {
-    if (cmax == 16 && G != 16) break;
-    for (int s_try : {2, 1}) {
-      const size_t row_bytes = (size_t)G * (s_try == 2 ? sizeof(float) : sizeof(WT));
-      int st = (int)((m + (int64_t)S::RPS * cmax - 1) / ((int64_t)S::RPS * cmax));
-      if (st < 1) st = 1;
-      if ((size_t)st * S::RPS * row_bytes <= 96 * 1024) {
-        steps = st;
-        C = (int)((m + (int64_t)S::RPS * st - 1) / ((int64_t)S::RPS * st));
-        stg = s_try;
-        return;
-      }
+  for (int c = 1; c <= 16; ++c) {
+    const int64_t rows = (m + c - 1) / c;
+    const int st = (int)((rows + S::RPS - 1) / S::RPS);
+    if (solver_smem_bytes<G>(st, sizeof(WT), true) <= SOLVER_SMEM_MAX) {
+      steps = st;
+      C = (int)((m + (int64_t)S::RPS * st - 1) / ((int64_t)S::RPS * st));
+      stg = 1;
+      return;
     }
   }
   steps = (int)((m + (int64_t)S::RPS * 8 - 1) / ((int64_t)S::RPS * 8));
@@ -912,9 +875,8 @@ static int launch_solver(const SolveBatch& bt, int count, int64_t m, int T, cons
     any_trace = any_trace || (traces && traces[i]);
   }
   const size_t sm_init = sizeof(SolverSmem<G>),
-               sm_main = solver_smem_bytes<G>(
-                   steps, stg == 2 ? sizeof(float) : (stg == 1 ? sizeof(WT) : 0), any_trace);
-  if (sm_main > 227 * 1024) return DQ_ERR_UNSUPPORTED;
+               sm_main = solver_smem_bytes<G>(steps, stg ? sizeof(WT) : 0, any_trace);
+  if (sm_main > SOLVER_SMEM_MAX) return DQ_ERR_UNSUPPORTED;
   if (tiles > 65535) return DQ_ERR_UNSUPPORTED;
 
   cudaLaunchAttribute attr[1];
@@ -936,18 +898,16 @@ static int launch_solver(const SolveBatch& bt, int count, int64_t m, int T, cons
 
   cfg.dynamicSmemBytes = sm_main;
   cudaError_t e;
-#define DQ_MAIN(WS, TR)                                                                     \
+#define DQ_MAIN(STAGED, TR)                                                                 \
   {                                                                                         \
-    auto km = solve_bcd_kernel<F, G, WT, WS, TR>;                                          \
+    auto km = solve_bcd_kernel<F, G, WT, STAGED, TR>;                                      \
     if (!allow_big_cluster(km, sm_main)) return DQ_ERR_CUDA;                               \
     e = cudaLaunchKernelEx(&cfg, km, bt, m, steps, T, o);                                   \
   }
-  if (stg == 2) {
-    if (any_trace) DQ_MAIN(2, true) else DQ_MAIN(2, false)
-  } else if (stg == 1) {
-    if (any_trace) DQ_MAIN(1, true) else DQ_MAIN(1, false)
+  if (stg) {
+    if (any_trace) DQ_MAIN(true, true) else DQ_MAIN(true, false)
   } else {
-    if (any_trace) DQ_MAIN(0, true) else DQ_MAIN(0, false)
+    if (any_trace) DQ_MAIN(false, true) else DQ_MAIN(false, false)
   }
 #undef DQ_MAIN
   if (e != cudaSuccess) return DQ_ERR_CUDA;
@@ -966,9 +926,8 @@ template <int G, typename WT>
 static int solver_supported(int64_t m, int64_t n) {
   int steps, C, stg;
   solver_geometry<G, WT>(m, steps, C, stg);
-  const size_t sm_main =   // with the trace array: the largest variant
-      solver_smem_bytes<G>(steps, stg == 2 ? sizeof(float) : (stg == 1 ? sizeof(WT) : 0), true);
-  return (sm_main > 227 * 1024 || n / G > 65535) ? DQ_ERR_UNSUPPORTED : DQ_OK;
+  const size_t sm_main = solver_smem_bytes<G>(steps, stg ? sizeof(WT) : 0, true);
+  return (sm_main > SOLVER_SMEM_MAX || n / G > 65535) ? DQ_ERR_UNSUPPORTED : DQ_OK;
 }
 
 template <typename WT>
