@@ -1,23 +1,27 @@
 #!/usr/bin/env python
 """Benchmark of the DualQuant dual-scale W4A4 hot path on B200.
 
-One step = the whole path over the Llama-3.1-8B-shaped attention workload
-(weights 4096x4096 and 1024x4096 bf16, NVFP4, 50 BCD rounds; activations
-M in {1, 16, 256, 4096} x 4096 bf16 with 1 % outlier channels x50):
-    for each weight : dq_solve_scales (T = 50) -> dq_quantize_weight
+Headline workload (qwen32b_mlp_nvfp4): the Qwen-32B-shaped MLP weights
+27648x5120 and 5120x27648 bf16 (Student-t), NVFP4, 50 BCD rounds;
+activations M x K bf16 with 1 % outlier channels x100, M = 8192 (prefill)
+and M in {1, 8, 64} (decode).  One step is the whole path:
     for each M, each weight : dq_quantize_act -> dq_w4a4_linear
-Inputs are resident in HBM before timing; L2 (126 MB) is flushed between
-steps by writing a 256 MiB buffer outside the timed events.
+    for each weight         : dq_solve_scales (T = 50) -> dq_quantize_weight
+The linears run first in the step, on the weights packed by the previous
+step, right after an L2 flush (a 256 MiB write outside the timed events), so
+they read their weights cold.  Inputs are resident in HBM before timing.
 
-`value` = W4A4 linear TFLOP/s of the inference part of the step (act quant
-+ GEMM, 2*M*N*K summed over the 8 linears, divided by their device time).
-The solver is reported beside it as effective streaming GB/s
-(T * bytes(W) / time) and its own time; ms_per_step covers everything.
-Inside the timed steps events sit only around each step, each solver call
-and the linear part (an event record costs the GPU microseconds).  The
-per-kernel figures (per_M_us, the GEMM and quantiser rooflines) are taken
-after the timed steps from launches back to back on copies of the inputs
-that together exceed L2.
+`value` = W4A4 linear TFLOP/s of the prefill linears (M = 8192, both
+weights, activation quantiser + GEMM: 2 M N K over their device time).  The
+solver, the decode linears and the packer are reported beside it, each with
+its own roofline fraction; ms_per_step covers the whole step.  Events sit
+only around the prefill linears, the decode linears and each solver call (an
+event record costs the GPU microseconds).  Per-kernel figures are taken
+after the timed steps from launches back to back on copies of their inputs
+that together exceed L2.  The other workloads (the Llama-3.1-8B-shaped
+attention and MX MLP layers, the tiny layer, the 224-weight sweep in four
+formats) and the MXFP8 linear are measured after that and reported under
+`configs` / `mxfp8`.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -36,7 +40,7 @@ sys.path.insert(0, ROOT)
 
 from w4a4_post_quantization_dual_b200 import dist, synth  # noqa: E402
 
-WORKLOAD = "llama8b_attn_nvfp4"
+WORKLOAD = "qwen32b_mlp_nvfp4"
 METRIC = "W4A4 linear TFLOP/s & % of FP4 peak; BCD solver GB/s & % HBM peak"
 FMT_NAME = "nvfp4"
 
@@ -64,14 +68,6 @@ def measured_traffic(key, files):
     for f in files:
         h.update(open(os.path.join(ROOT, "w4a4_post_quantization_dual_b200", "csrc", f), "rb").read())
     return rec["dram_bytes"] if h.hexdigest()[:16] == rec["source_hash"] else None
-
-
-def workload_inputs():
-    wl = synth.WORKLOADS[WORKLOAD]
-    Ws = [synth.weight(WORKLOAD, i)[0] for i in range(len(wl["weights"]))]
-    K = Ws[0].shape[1]
-    Xs = {M: synth.acts(WORKLOAD, M, K)[0] for M in wl["M"]}
-    return wl, Ws, Xs
 
 
 class ClockSampler:
@@ -132,13 +128,147 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# Inputs
+# ---------------------------------------------------------------------------
+def workload_inputs(name, fmt_name=None):
+    """Host inputs of a workload: weights and, per weight, its activations
+    for every M of the workload (K = the weight's input width)."""
+    wl = synth.WORKLOADS[name]
+    Ws = [synth.weight(name, i)[0] for i in range(len(wl["weights"]))]
+    Xs = {}
+    for j, W in enumerate(Ws):
+        K = W.shape[1]
+        for M in wl["M"]:
+            Xs[(M, j)] = synth.acts(name, M, K, index=j)[0]
+    return wl, Ws, Xs
+
+
+def ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def per_launch_us(fn_of_copy, n_copies, reps=2):
+    """Average duration of fn_of_copy(i) launched back to back between two
+    events (i cycling over n_copies input copies, so that the launches read
+    cold data when the copies together exceed L2)."""
+    st = torch.cuda.current_stream()
+    for i in range(n_copies):
+        fn_of_copy(i)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(60_000 * reps * n_copies)  # the launches queue up behind it
+    k0, k1 = ev(), ev()
+    k0.record(st)
+    for _ in range(reps):
+        for i in range(n_copies):
+            fn_of_copy(i)
+    k1.record(st)
+    torch.cuda.synchronize()
+    return 1e3 * k0.elapsed_time(k1) / (reps * n_copies)
+
+
+def n_copies(nbytes, lo=2, hi=64):
+    """Copies of an input whose total exceeds twice L2."""
+    return int(max(lo, min(hi, -(-2 * L2_BYTES // max(nbytes, 1)))))
+
+
+def act_bytes(M, K, fmt, G):
+    """Algorithmic bytes of one activation rescale+quantise: bf16 in, codes,
+    block scales (and the fp32 per-token scale for NVFP4) out."""
+    from w4a4_post_quantization_dual_b200 import dq
+    code = 1.0 if dq._fmt(fmt) in dq.EIGHT_BIT else 0.5
+    return M * K * (2 + code + 1.0 / G) + (4 * M if dq._fmt(fmt) == dq.DQ_NVFP4 else 0)
+
+
+def decode_bytes(M, N, K, G):
+    """Algorithmic bytes of a 4-bit linear at small M (weight-bandwidth bound):
+    weight codes + block scales, activation codes + scales + per-token
+    scales, bf16 output."""
+    return N * K / 2 + N * K / G + M * K / 2 + M * K / G + 4 * M + 2 * M * N
+
+
+class Layer:
+    """Device buffers of one weight: the weight, its scales, its packed form."""
+
+    def __init__(self, W, fmt, G, dev):
+        from w4a4_post_quantization_dual_b200 import dq
+        self.W = W
+        m, n = W.shape
+        eight = dq._fmt(fmt) in dq.EIGHT_BIT
+        self.r = torch.empty((m, n // G), dtype=torch.float32, device=dev)
+        self.c = torch.empty(n, dtype=torch.float32, device=dev)
+        self.sT = torch.empty(1, dtype=torch.float32, device=dev)
+        self.codes = torch.empty((m, n if eight else n // 2), dtype=torch.uint8, device=dev)
+        self.scales = torch.empty(dq.scales_bytes(m, n, fmt, G), dtype=torch.uint8, device=dev)
+
+    def solve(self, fmt, T, ws, G):
+        from w4a4_post_quantization_dual_b200 import dq
+        dq.dq_solve_scales(self.W, fmt, T, self.r, self.c, self.sT, None, ws, group=G)
+
+    def pack(self, fmt, G):
+        from w4a4_post_quantization_dual_b200 import dq
+        dq.dq_quantize_weight(self.W, fmt, self.r, self.c, self.sT, self.codes, self.scales,
+                              group=G)
+
+
+class Act:
+    """Device buffers of one activation and its quantised form."""
+
+    def __init__(self, X, fmt, G, N, dev):
+        from w4a4_post_quantization_dual_b200 import dq
+        M, K = X.shape
+        eight = dq._fmt(fmt) in dq.EIGHT_BIT
+        self.X = X
+        self.A = torch.empty((M, K if eight else K // 2), dtype=torch.uint8, device=dev)
+        self.sA = torch.empty(dq.scales_bytes(M, K, fmt, G), dtype=torch.uint8, device=dev)
+        self.st = (torch.empty(M, dtype=torch.float32, device=dev)
+                   if dq._fmt(fmt) == dq.DQ_NVFP4 else None)
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+    def linear(self, L, fmt, G, X=None):
+        from w4a4_post_quantization_dual_b200 import dq
+        dq.dq_quantize_act(self.X if X is None else X, fmt, L.c, self.A, self.sA, self.st, group=G)
+        dq.dq_w4a4_linear(self.A, self.sA, self.st, L.codes, L.scales, L.sT, self.Y, fmt)
+
+    def gemm(self, fmt, codes, scales, sT):
+        from w4a4_post_quantization_dual_b200 import dq
+        dq.dq_w4a4_linear(self.A, self.sA, self.st, codes, scales, sT, self.Y, fmt)
+
+
+def time_linear(L, a, fmt, G, peak_tf):
+    """Activation quantiser and GEMM of one (activation, weight) pair, each
+    launched back to back on cold copies of its input (activations for the
+    quantiser, packed weights for the GEMM)."""
+    M, K = a.X.shape
+    N = L.W.shape[0]
+    from w4a4_post_quantization_dual_b200 import dq
+    nx = n_copies(a.X.numel() * 2, hi=16)
+    Xc = [a.X.clone() for _ in range(nx)]
+    t_act = per_launch_us(lambda i: dq.dq_quantize_act(Xc[i], fmt, L.c, a.A, a.sA, a.st,
+                                                       group=G), nx)
+    del Xc
+    a.linear(L, fmt, G)
+    nw = n_copies(L.codes.numel() + L.scales.numel())
+    Bc = [(L.codes.clone(), L.scales.clone()) for _ in range(nw)]
+    t_gemm = per_launch_us(lambda i: a.gemm(fmt, Bc[i][0], Bc[i][1], L.sT), nw)
+    del Bc
+    fl = 2.0 * M * N * K
+    ab = act_bytes(M, K, fmt, G)
+    return {"M": M, "N": N, "K": K, "act_us": t_act, "gemm_us": t_gemm,
+            "gemm_tflops": fl / (t_gemm * 1e-6) / 1e12, "gemm_frac": fl / (t_gemm * 1e-6) / 1e12 / peak_tf,
+            "act_gbs": ab / (t_act * 1e-6) / 1e9, "linear_tflops": fl / ((t_act + t_gemm) * 1e-6) / 1e12}
+
+
+# ---------------------------------------------------------------------------
 # Reference arm / CPU baseline: the oracle as it stands, on host cores.
 # ---------------------------------------------------------------------------
 _ORACLE_PACKED = {}
 
 
-def oracle_prepare(wl, Ws):
-    """Offline part for the oracle legs: Algorithm 1 initial scales of every
+def oracle_prepare(Ws):
+    """Offline part for the oracle legs: Algorithm 1's initial scales of every
     tile (T = 0) and the packed weights, computed once and cached."""
     import oracle as O
     if not _ORACLE_PACKED:
@@ -149,38 +279,62 @@ def oracle_prepare(wl, Ws):
     return _ORACLE_PACKED
 
 
-def oracle_linear_sample(wl, Ws, Xs, rows):
-    """The oracle's inference path -- activation rescale+quantise and the
-    dequantised fp64 matmul -- on `rows` token rows of the M=4096 activations,
-    for both weights.  Returns (TFLOP/s, seconds)."""
+SAMPLE_COLS = 2048
+
+
+def oracle_linear_sample(Ws, Xs, M, rows):
+    """The oracle's inference path on a bounded sample of the prefill
+    linears: activation rescale+quantise of `rows` token rows, then the
+    dequantised fp64 matmul for SAMPLE_COLS seeded output columns, for both
+    weights.  Returns (TFLOP/s of the sampled outputs, seconds)."""
     import oracle as O
-    packed = oracle_prepare(wl, Ws)
-    X = Xs[max(Xs)][:rows]
+    packed = oracle_prepare(Ws)
     flops, t0 = 0.0, time.perf_counter()
-    for i, W in enumerate(Ws):
+    for j, W in enumerate(Ws):
         N, K = W.shape
-        res, B, sB = packed[i]
+        res, B, sB = packed[j]
+        X = Xs[(M, j)][:rows]
         A, sA, st = O.quantize_act(X, res["c"], O.NVFP4, 16)
-        O.linear(A, sA, st, B, sB, res["s_T"], rows, N, K, O.NVFP4)
-        flops += 2.0 * rows * N * K
+        cols = np.random.default_rng(j).choice(N, size=min(SAMPLE_COLS, N), replace=False)
+        O.linear_rows(A, sA, st, B, sB, res["s_T"], np.arange(rows), rows, N, K, O.NVFP4,
+                      cols=cols)
+        flops += 2.0 * rows * len(cols) * K
     dt = time.perf_counter() - t0
     return flops / dt / 1e12, dt
 
 
-def oracle_solver_sample(wl, Ws):
-    """Algorithm 1 (T = 50) on one 4096 x 16 tile of the first weight.
-    Returns effective GB/s (T * tile bytes / time) and seconds."""
+LINEAR_SAMPLE_DESC = ("oracle (C + numpy fp64): activation rescale+quantise of {rows} of the "
+                      "{M} prefill token rows and the dequantised fp64 matmul for " +
+                      str(SAMPLE_COLS) + " sampled output columns, both weights (weights "
+                      "packed once beforehand, outside the timing)")
+
+
+def _oracle_tile(args):
     import oracle as O
-    W, T = Ws[0], wl["T"]
+    Wt, T = args
     t0 = time.perf_counter()
-    O.solve(W, O.NVFP4, 16, T, tiles=[0])
-    dt = time.perf_counter() - t0
-    return T * W.shape[0] * 16 * 2.0 / dt / 1e9, dt
+    O.solve(Wt, O.NVFP4, 16, T)
+    return time.perf_counter() - t0
 
 
-LINEAR_SAMPLE_DESC = ("oracle (C + numpy fp64): activation rescale+quantise and dequantised "
-                      "matmul on {rows} of the 4096 token rows, both weights (weights packed once "
-                      "beforehand, outside the timing)")
+def oracle_solver_sample(W, T, procs):
+    """Algorithm 1 (T rounds) on whole m x 16 column tiles of the weight:
+    one tile on one core, then one tile per process on `procs` host cores
+    (spawned processes).  Each tile is solved on its own columns (its
+    initial scales and tensor scale from those columns).  Returns effective
+    GB/s (T * tile bytes / time) for both and the seconds."""
+    import multiprocessing as mp
+    m = W.shape[0]
+    tile = lambda b: np.ascontiguousarray(W[:, 16 * b:16 * b + 16])
+    one = _oracle_tile((tile(0), T))
+    ctx = mp.get_context("spawn")
+    t0 = time.perf_counter()
+    with ctx.Pool(procs) as pool:
+        pool.map(_oracle_tile, [(tile(b), T) for b in range(procs)])
+    wall = time.perf_counter() - t0
+    tb = T * m * 16 * 2.0
+    return {"one_core_gbs": tb / one / 1e9, "one_core_s": one,
+            "all_cores_gbs": procs * tb / wall / 1e9, "all_cores_s": wall, "cores": procs}
 
 
 def blas_threads():
@@ -194,23 +348,25 @@ def blas_threads():
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    wl, Ws, Xs = workload_inputs()
-    oracle_prepare(wl, Ws)
+    wl, Ws, Xs = workload_inputs(WORKLOAD)
+    M = max(wl["M"])
+    oracle_prepare(Ws)
     for _ in range(args.warmup):
-        oracle_linear_sample(wl, Ws, Xs, rows=16)
+        oracle_linear_sample(Ws, Xs, M, rows=16)
     flops_t, dt = 0.0, 0.0
     for _ in range(args.steps):
-        v, d = oracle_linear_sample(wl, Ws, Xs, rows=16)
+        v, d = oracle_linear_sample(Ws, Xs, M, rows=16)
         flops_t += v * d
         dt += d
     value = flops_t / dt
-    desc = LINEAR_SAMPLE_DESC.format(rows=16)
+    desc = LINEAR_SAMPLE_DESC.format(rows=16, M=M)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / max(args.steps, 1) * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "format": FMT_NAME, "sample_rows": 16},
+        "config": {"workload": WORKLOAD, "format": FMT_NAME, "M": M, "sample_rows": 16,
+                   "sample_cols": SAMPLE_COLS},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -222,82 +378,95 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 # Our arm
 # ---------------------------------------------------------------------------
-def run_ours(args, rank, world, local_rank):
+def side_config(name, fmts, dev, ws_T, ws, peaks_):
+    """Solver time and linear throughput of another workload (not timed in the
+    step): per format, each weight solved (T rounds) and packed, then the
+    activation quantiser and GEMM of every M of the workload."""
     from w4a4_post_quantization_dual_b200 import dq
+    hbm, fp4_peak, fp8_peak, alu_peak = peaks_
+    wl, Ws, Xs = workload_inputs(name)
+    T = wl["T"]
+    Wd = [torch.from_numpy(W).to(torch.bfloat16).to(dev) for W in Ws]
+    out = {"weights": [list(W.shape) for W in Ws], "M": wl["M"], "T": T}
+    for f in fmts:
+        fmt = dq.FORMATS[f]
+        G = dq.native_group(fmt)
+        peak = fp8_peak if f in ("mxint4", "mxfp8") else fp4_peak
+        res = {"solver": {}, "linear": {}}
+        Ls = [Layer(W, fmt, G, dev) for W in Wd]
+        for L in Ls:
+            ms = 1e-3 * per_launch_us(lambda i: L.solve(fmt, T, ws, G), 2)
+            m_, n_ = L.W.shape
+            tops = 12.0 * m_ * n_ * T / (ms * 1e-3) / 1e12
+            res["solver"][f"{m_}x{n_}"] = {"ms": ms, "tops": tops, "frac_alu": tops / alu_peak}
+            L.pack(fmt, G)
+        for (M, j), X in Xs.items():
+            a = Act(torch.from_numpy(X).to(torch.bfloat16).to(dev), fmt, G, Ls[j].W.shape[0], dev)
+            res["linear"][f"M{M}_N{Ls[j].W.shape[0]}_K{Ls[j].W.shape[1]}"] = time_linear(
+                Ls[j], a, fmt, G, peak)
+            del a
+        res["peak_tflops"] = peak
+        out[f] = res
+        del Ls
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    from w4a4_post_quantization_dual_b200 import dq, sweep
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     dq.lib()
-    wl, Ws, Xs = workload_inputs()
+    wl, Ws, Xs = workload_inputs(WORKLOAD)
     fmt, T = dq.DQ_NVFP4, wl["T"]
     G = dq.native_group(fmt)
     st = torch.cuda.current_stream()
+    Mp = max(wl["M"])                     # prefill
+    Mds = sorted(M for M in wl["M"] if M != Mp)  # decode
 
-    # device-resident inputs and outputs
-    Wd = [torch.from_numpy(W).to(torch.bfloat16).to(dev) for W in Ws]
-    Xd = {M: torch.from_numpy(X).to(torch.bfloat16).to(dev) for M, X in Xs.items()}
-    ws = torch.empty(dq.solve_workspace_size(T), dtype=torch.uint8, device=dev)
-    Wbuf = []
-    for W in Wd:
-        m, n = W.shape
-        Wbuf.append(dict(
-            r=torch.empty((m, n // G), dtype=torch.float32, device=dev),
-            c=torch.empty(n, dtype=torch.float32, device=dev),
-            sT=torch.empty(1, dtype=torch.float32, device=dev),
-            codes=torch.empty((m, n // 2), dtype=torch.uint8, device=dev),
-            scales=torch.empty(dq.scales_bytes(m, n, fmt, G), dtype=torch.uint8, device=dev)))
-    Abuf = {}
-    for M, X in Xd.items():
-        K = X.shape[1]
-        Abuf[M] = dict(A=torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
-                       sA=torch.empty(dq.scales_bytes(M, K, fmt, G), dtype=torch.uint8, device=dev),
-                       st=torch.empty(M, dtype=torch.float32, device=dev),
-                       Y=[torch.empty((M, W.shape[0]), dtype=torch.bfloat16, device=dev) for W in Wd])
+    Ls = [Layer(torch.from_numpy(W).to(torch.bfloat16).to(dev), fmt, G, dev) for W in Ws]
+    acts = {(M, j): Act(torch.from_numpy(X).to(torch.bfloat16).to(dev), fmt, G,
+                        Ls[j].W.shape[0], dev) for (M, j), X in Xs.items()}
+    ws = torch.empty(dq.solve_workspace_size(max(T, 64)), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    lin_flops = sum(2.0 * M * W.shape[0] * W.shape[1] for M in Xd for W in Wd)
-    prefill_M = max(Xd)
-    launches_per_step = 2 * len(Wd) + len(Wd) + 2 * len(Wd) * len(Xd)
-
-    def ev():
-        return torch.cuda.Event(enable_timing=True)
-
-    def linears():
-        for M, X in Xd.items():
-            a = Abuf[M]
-            for j, (W, b) in enumerate(zip(Wd, Wbuf)):
-                dq.dq_quantize_act(X, fmt, b["c"], a["A"], a["sA"], a["st"], group=G)
-                dq.dq_w4a4_linear(a["A"], a["sA"], a["st"], b["codes"], b["scales"], b["sT"],
-                                  a["Y"][j], fmt)
+    flops_p = sum(2.0 * Mp * L.W.shape[0] * L.W.shape[1] for L in Ls)
+    launches_per_step = 2 * len(Ls) * len(wl["M"]) + 3 * len(Ls)
 
     def step(rec):
-        # events only around the step, its solver calls and its linear part:
-        # an event record costs the GPU microseconds, so none sits between
-        # the short inference kernels
-        e0, e1, e2 = ev(), ev(), ev()
+        # linears first, on the weights the previous step packed, right after
+        # the L2 flush (cold weights); events only around the prefill
+        # linears, the decode linears and each solver call
+        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
         e0.record(st)
-        for W, b in zip(Wd, Wbuf):
+        for j, L in enumerate(Ls):
+            acts[(Mp, j)].linear(L, fmt, G)
+        e1.record(st)
+        for M in Mds:
+            for j, L in enumerate(Ls):
+                acts[(M, j)].linear(L, fmt, G)
+        e2.record(st)
+        for L in Ls:
             s0, s1 = ev(), ev()
             s0.record(st)
-            dq.dq_solve_scales(W, fmt, T, b["r"], b["c"], b["sT"], None, ws, group=G)
+            L.solve(fmt, T, ws, G)
             s1.record(st)
-            dq.dq_quantize_weight(W, fmt, b["r"], b["c"], b["sT"], b["codes"], b["scales"], group=G)
-            rec["solve"].append((s0, s1, W.numel()))
-        e1.record(st)
-        linears()
-        e2.record(st)
-        rec["step"].append((e0, e2))
-        rec["lin"].append((e1, e2))
+            L.pack(fmt, G)
+            rec["solve"].append((s0, s1))
+        e3.record(st)
+        rec["step"].append((e0, e3))
+        rec["prefill"].append((e0, e1))
+        rec["decode"].append((e1, e2))
 
     dist.barrier()
     for _ in range(args.warmup):
         flush.fill_(1)
-        step({"solve": [], "step": [], "lin": []})
+        step({"solve": [], "step": [], "prefill": [], "decode": []})
     torch.cuda.synchronize()
     dist.barrier()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    rec = {"solve": [], "step": [], "lin": []}
+    rec = {"solve": [], "step": [], "prefill": [], "decode": []}
     for _ in range(args.steps):
         flush.fill_(rank + 1)      # L2 flush, outside the timed events
         step(rec)
@@ -310,278 +479,251 @@ def run_ours(args, rank, world, local_rank):
 
     el = lambda p: p[0].elapsed_time(p[1])  # ms
     step_ms = sum(el(p) for p in rec["step"])
-    lin_ms = sum(el(p) for p in rec["lin"])
-    solve_ms = sum(el(p[:2]) for p in rec["solve"])
-    big = max(p[2] for p in rec["solve"])
-    solve_big = [el(p[:2]) for p in rec["solve"] if p[2] == big]
-    step_ms, lin_ms, solve_ms = dist.max_over_ranks([step_ms, lin_ms, solve_ms], device=dev)
+    pre_ms = sum(el(p) for p in rec["prefill"])
+    dec_ms = sum(el(p) for p in rec["decode"])
+    solve_each = [el(p) for p in rec["solve"]]
+    solve_ms = sum(solve_each)
+    step_ms, pre_ms, dec_ms, solve_ms = dist.max_over_ranks([step_ms, pre_ms, dec_ms, solve_ms],
+                                                            device=dev)
+    # whole-job throughput: every rank runs the same per-GPU workload (weak
+    # scaling); the time is the slowest rank's
+    value = world * flops_p * args.steps / (pre_ms * 1e-3) / 1e12
 
-    # ---- per-kernel durations (after the timed steps): R launches back to
-    # back between two events, each on its own copy of the inputs, the copies
-    # together larger than L2 so that every launch reads cold data
-    def per_launch_us(fn_of_copy, n_copies, reps=2):
-        for i in range(n_copies):
-            fn_of_copy(i)
-        torch.cuda.synchronize()
-        torch.cuda._sleep(60_000 * reps * n_copies)  # the launches queue up behind it
-        k0, k1 = ev(), ev()
-        k0.record(st)
-        for _ in range(reps):
-            for i in range(n_copies):
-                fn_of_copy(i)
-        k1.record(st)
-        torch.cuda.synchronize()
-        return 1e3 * k0.elapsed_time(k1) / (reps * n_copies)
+    hbm, bf16_tf, bf16_sus, sm_max, peak_kind = peaks()
+    fp4_peak = 4.0 * bf16_tf            # nominal fp4 : bf16 dense ratio 9 : 2.25
+    fp8_peak = 2.0 * bf16_tf            # nominal fp8 : bf16 dense ratio 4.5 : 2.25
+    # solver: 12 algorithmic fp32 ops per element per round (two
+    # quantisations, two scale products, four reduction FMAs); ALU peak =
+    # 148 SMs x 128 fp32 lanes x max SM clock (derived, not measured)
+    alu_peak = 148 * 128 * sm_max * 1e6 / 1e12  # T lane-ops/s
 
-    L2_BYTES = 126 * 1024 * 1024
-    per_m = {}
-    kt = {}
-    for M, X in Xd.items():
-        K = X.shape[1]
-        nx = max(2, min(16, -(-2 * L2_BYTES // (X.numel() * 2))))
-        Xc = [X.clone() for _ in range(nx)]
-        a = Abuf[M]
-        per_m[str(M)] = {}
-        for j, (W, b) in enumerate(zip(Wd, Wbuf)):
-            wbytes = b["codes"].numel() + b["scales"].numel()
-            nw = max(2, min(128, -(-2 * L2_BYTES // wbytes)))
-            Bc = [(b["codes"].clone(), b["scales"].clone()) for _ in range(nw)]
-            t_act = per_launch_us(lambda i: dq.dq_quantize_act(
-                Xc[i % nx], fmt, b["c"], a["A"], a["sA"], a["st"], group=G), nx)
-            t_gemm = per_launch_us(lambda i: dq.dq_w4a4_linear(
-                a["A"], a["sA"], a["st"], Bc[i][0], Bc[i][1], b["sT"], a["Y"][j], fmt), nw)
-            per_m[str(M)][f"N{W.shape[0]}"] = {"act_quant": t_act, "gemm": t_gemm}
-            kt[(M, j)] = (t_act, t_gemm)
+    # ---- per-kernel durations (after the timed steps)
+    solver = {}
+    for j, L in enumerate(Ls):
+        m_, n_ = L.W.shape
+        ms = float(np.mean(solve_each[j::len(Ls)]))
+        tops = 12.0 * m_ * n_ * T / (ms * 1e-3) / 1e12
+        gbs = T * m_ * n_ * 2.0 / (ms * 1e-3) / 1e9
+        solver[f"{m_}x{n_}"] = {"ms": ms, "tops": tops, "frac_alu": tops / alu_peak,
+                                "gbs_effective": gbs, "frac_hbm_effective": gbs / hbm}
+    prefill = {f"N{L.W.shape[0]}_K{L.W.shape[1]}": time_linear(L, acts[(Mp, j)], fmt, G, fp4_peak)
+               for j, L in enumerate(Ls)}
+    decode = {}
+    for M in Mds:
+        for j, L in enumerate(Ls):
+            a = acts[(M, j)]
+            N, K = L.W.shape
+            nw = n_copies(L.codes.numel() + L.scales.numel())
+            Bc = [(L.codes.clone(), L.scales.clone()) for _ in range(nw)]
+            a.linear(L, fmt, G)
+            t_gemm = per_launch_us(lambda i: a.gemm(fmt, Bc[i][0], Bc[i][1], L.sT), nw)
+
+            def pair(i):
+                dq.dq_quantize_act(a.X, fmt, L.c, a.A, a.sA, a.st, group=G)
+                a.gemm(fmt, Bc[i][0], Bc[i][1], L.sT)
+
+            def fused(i):
+                dq.dq_w4a4_linear_fused(a.X, L.c, Bc[i][0], Bc[i][1], L.sT, a.Y, fmt)
+
+            t_pair = per_launch_us(pair, nw)
+            try:    # the fused kernel takes the shapes whose K split fits its stages
+                t_fused = per_launch_us(fused, nw)
+            except dq.DQError:
+                t_fused = None
             del Bc
-        del Xc
-    # ---- solver ablation modes (Table 4 arms) on the largest weight: both
-    # scales, alpha-only, beta-only; each mode is one dq_solve_scales_ex call
-    jb = max(range(len(Wd)), key=lambda j: Wd[j].numel())
-    Wb, bb = Wd[jb], Wbuf[jb]
+            b_ = decode_bytes(M, N, K, G)
+            decode[f"M{M}_N{N}_K{K}"] = {
+                "gemm_us": t_gemm, "act_plus_gemm_us": t_pair, "fused_us": t_fused,
+                "algorithmic_bytes": b_, "gemm_gbs": b_ / (t_gemm * 1e-6) / 1e9,
+                "gemm_frac_hbm": b_ / (t_gemm * 1e-6) / 1e9 / hbm,
+                "pair_gbs": b_ / (t_pair * 1e-6) / 1e9,
+                "fused_gbs": b_ / (t_fused * 1e-6) / 1e9 if t_fused else None,
+                "fused_frac_hbm": b_ / (t_fused * 1e-6) / 1e9 / hbm if t_fused else None}
+    pack = {}
+    for L in Ls:
+        m_, n_ = L.W.shape
+        t = per_launch_us(lambda i: L.pack(fmt, G), 2)
+        b_ = m_ * n_ * (2 + 0.5 + 1.0 / G)
+        pack[f"{m_}x{n_}"] = {"us": t, "gbs": b_ / (t * 1e-6) / 1e9,
+                              "frac_hbm": b_ / (t * 1e-6) / 1e9 / hbm}
+
+    # ---- solver ablation modes (Table 4 arms) on the first weight
+    L0 = Ls[0]
     modes = {"both": 0, "alpha_only": dq.DQ_SOLVE_ALPHA_ONLY, "beta_only": dq.DQ_SOLVE_BETA_ONLY}
-    mode_ms = {}
-    for name, flags in modes.items():
-        mode_ms[name] = 1e-3 * per_launch_us(lambda i: dq.dq_solve_scales_ex(
-            Wb, fmt, T, bb["r"], bb["c"], bb["sT"], flags=flags, workspace=ws, group=G), 3)
-    # restore the step's scales of that weight (the last mode overwrote them)
-    dq.dq_solve_scales(Wb, fmt, T, bb["r"], bb["c"], bb["sT"], None, ws, group=G)
-    # batched solver entry on the seven projections of one Llama-3.1-8B layer
-    # (q, k, v, o, gate, up, down; random bf16 weights, same format and T):
-    # separate calls vs one dq_solve_scales_batched call
-    lshapes = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (14336, 4096),
-               (14336, 4096), (4096, 14336)]
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(7)
-    LW = [(torch.randn(m_, n_, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
-          for m_, n_ in lshapes]
-    Lr = [torch.empty((m_, n_ // G), device=dev) for m_, n_ in lshapes]
-    Lc = [torch.empty(n_, device=dev) for _, n_ in lshapes]
-    Ls = [torch.empty(1, device=dev) for _ in lshapes]
-    Lws = torch.empty(dq.solve_batched_workspace_size(len(LW), T), dtype=torch.uint8, device=dev)
+    mode_ms = {name: 1e-3 * per_launch_us(lambda i: dq.dq_solve_scales_ex(
+        L0.W, fmt, T, L0.r, L0.c, L0.sT, flags=flags, workspace=ws, group=G), 2)
+        for name, flags in modes.items()}
+    L0.solve(fmt, T, ws, G)   # restore the step's scales of that weight
+    L0.pack(fmt, G)
 
-    def layer_separate(_):
-        for W_, r_, c_, s_ in zip(LW, Lr, Lc, Ls):
-            dq.dq_solve_scales(W_, fmt, T, r_, c_, s_, None, ws, group=G)
-
-    def layer_batched(_):
-        dq.dq_solve_scales_batched(LW, fmt, T, Lr, Lc, Ls, None, Lws, group=G)
-
-    batched_ms = {"separate": 1e-3 * per_launch_us(layer_separate, 1),
-                  "batched": 1e-3 * per_launch_us(layer_batched, 1)}
-    del LW, Lr, Lc, Ls, Lws
-    # activation SQNR of the prefill activations with each weight's column
-    # scales (beta) and without them (Appendix E, Table 6)
+    # ---- activation SQNR of the prefill activations with each weight's
+    # column scales (beta) and without them (Appendix E, Table 6)
     act_sqnr = {}
-    for W, b in zip(Wd, Wbuf):
-        key = f"N{W.shape[0]}"
-        act_sqnr[key] = {"with_beta_db": dq.act_sqnr_db(Xd[prefill_M], fmt, b["c"], group=G)}
-    no_beta = dq.act_sqnr_db(Xd[prefill_M], fmt, None, group=G)
-    for v in act_sqnr.values():
-        v["without_beta_db"] = no_beta
-        v["delta_db"] = v["with_beta_db"] - no_beta
+    for j, L in enumerate(Ls):
+        X = acts[(Mp, j)].X
+        w_ = dq.act_sqnr_db(X, fmt, L.c, group=G)
+        wo = dq.act_sqnr_db(X, fmt, None, group=G)
+        act_sqnr[f"K{X.shape[1]}"] = {"with_beta_db": w_, "without_beta_db": wo,
+                                      "delta_db": w_ - wo}
     torch.cuda.synchronize()
     if dq.dq_device_error(clear=True) != 0:
         raise RuntimeError("device error word set during the per-kernel timing")
 
-    # ---- e2e through the public API with host buffers (pinned), prefill linears
-    e2e = None
-    if rank == 0 or world > 1:
-        Xh = torch.from_numpy(Xs[prefill_M]).to(torch.bfloat16).pin_memory()
-        Yh = [torch.empty((prefill_M, W.shape[0]), dtype=torch.bfloat16).pin_memory() for W in Wd]
-        a = Abuf[prefill_M]
-        Xdev = torch.empty_like(Xd[prefill_M])
-
-        def e2e_step():
-            Xdev.copy_(Xh, non_blocking=True)
-            for j, (W, b) in enumerate(zip(Wd, Wbuf)):
-                dq.dq_quantize_act(Xdev, fmt, b["c"], a["A"], a["sA"], a["st"], group=G)
-                dq.dq_w4a4_linear(a["A"], a["sA"], a["st"], b["codes"], b["scales"], b["sT"],
-                                  a["Y"][j], fmt)
-                Yh[j].copy_(a["Y"][j], non_blocking=True)
-
-        for _ in range(3):
-            e2e_step()
+    # ---- the other workloads (reported beside the headline, not in the step)
+    peaks_ = (hbm, fp4_peak, fp8_peak, alu_peak)
+    configs = {}
+    if rank == 0 and not args.headline_only:
+        configs["llama8b_attn_nvfp4"] = side_config("llama8b_attn_nvfp4", ["nvfp4"], dev, T, ws,
+                                                    peaks_)
+        configs["llama8b_mlp_mx"] = side_config("llama8b_mlp_mx", ["mxfp4", "mxint4"], dev, T,
+                                                ws, peaks_)
+        configs["tiny_layer_256"] = side_config("tiny_layer_256", ["nvfp4"], dev, T, ws, peaks_)
+        # whole-model sweep: the 224 linears of a Llama-3.1-8B-shaped model,
+        # random bf16 Student-t weights, solved (T = 50) and packed per format
+        lin = sweep.llama8b_linears()
+        SW = [sweep.student_t_weight(m_, n_, 10_000 + i, dev) for i, (_, m_, n_) in enumerate(lin)]
+        sw = {"weights": len(SW), "params": int(sum(W.numel() for W in SW)), "T": 50}
+        for f, g in (("int4", 128), ("mxint4", 0), ("mxfp4", 0), ("nvfp4", 0)):
+            torch.cuda.synchronize()
+            s0, s1 = ev(), ev()
+            s0.record(st)
+            qs = sweep.solve_and_pack(SW, dq.FORMATS[f], 50, group=g)
+            s1.record(st)
+            torch.cuda.synchronize()
+            sec = 1e-3 * s0.elapsed_time(s1)
+            sw[f] = {"group": g or dq.native_group(dq.FORMATS[f]), "seconds": sec,
+                     "weights_per_s": len(SW) / sec,
+                     "packed_bytes": int(sum(q.codes.numel() + q.scales.numel() for q in qs))}
+            del qs
+        del SW
+        configs["llama8b_sweep_224"] = sw
         torch.cuda.synchronize()
-        tot = 0.0
-        for _ in range(max(args.steps, 5)):
-            flush.fill_(2)
-            x0, x1 = ev(), ev()
-            x0.record(st)
-            e2e_step()
-            x1.record(st)
-            x1.synchronize()
-            tot += x0.elapsed_time(x1)
-        n_e2e = max(args.steps, 5)
-        fl = sum(2.0 * prefill_M * W.shape[0] * W.shape[1] for W in Wd)
-        e2e = {"value": fl * n_e2e / (tot * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": Xh.numel() * 2,
-               "d2h_bytes_per_step": sum(y.numel() * 2 for y in Yh),
-               "what": f"host bf16 X ({prefill_M}x4096) -> device, act quant + GEMM for both "
-                       f"weights, bf16 Y -> host; prefill M={prefill_M}"}
+        if dq.dq_device_error(clear=True) != 0:
+            raise RuntimeError("device error word set during the side configurations")
+
+    # ---- 8-bit variant (Appendix G.2): MXFP8 linear at the prefill shape of
+    # the first weight.  Auxiliary: an error is reported, not raised.
+    mxfp8 = None
+    if rank == 0 and not args.headline_only:
+        try:
+            L8 = Layer(Ls[0].W, dq.DQ_MXFP8, 32, dev)
+            L8.solve(dq.DQ_MXFP8, T, ws, 32)
+            L8.pack(dq.DQ_MXFP8, 32)
+            a8 = Act(acts[(Mp, 0)].X, dq.DQ_MXFP8, 32, L8.W.shape[0], dev)
+            mxfp8 = time_linear(L8, a8, dq.DQ_MXFP8, 32, fp8_peak)
+            mxfp8["peak_tflops"] = fp8_peak
+            mxfp8["device_error"] = dq.dq_device_error(clear=True)
+            del L8, a8
+        except Exception as ex:  # auxiliary measurement: report, do not fail the bench line
+            mxfp8 = {"error": str(ex)[:300]}
+
+    # ---- e2e through the public API with host buffers (pinned): the prefill
+    # linears of both weights, X host -> device, Y device -> host, every step
+    e2e = None
+    Xh = [torch.from_numpy(Xs[(Mp, j)]).to(torch.bfloat16).pin_memory() for j in range(len(Ls))]
+    Yh = [torch.empty((Mp, L.W.shape[0]), dtype=torch.bfloat16).pin_memory() for L in Ls]
+    Xdev = [torch.empty_like(acts[(Mp, j)].X) for j in range(len(Ls))]
+
+    def e2e_step():
+        for j, L in enumerate(Ls):
+            Xdev[j].copy_(Xh[j], non_blocking=True)
+            acts[(Mp, j)].linear(L, fmt, G, X=Xdev[j])
+            Yh[j].copy_(acts[(Mp, j)].Y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    tot = 0.0
+    n_e2e = max(min(args.steps, 10), 3)
+    for _ in range(n_e2e):
+        flush.fill_(2)
+        x0, x1 = ev(), ev()
+        x0.record(st)
+        e2e_step()
+        x1.record(st)
+        x1.synchronize()
+        tot += x0.elapsed_time(x1)
+    tot = dist.max_over_ranks([tot], device=dev)[0]
+    e2e = {"value": world * flops_p * n_e2e / (tot * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(sum(x.numel() * 2 for x in Xh)),
+           "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in Yh)),
+           "what": f"host bf16 X -> device, act quant + GEMM, bf16 Y -> host, both weights, "
+                   f"prefill M={Mp}"}
 
     if rank != 0:
         return
-    hbm, bf16_tf, bf16_sus, sm_max, peak_kind = peaks()
-    fp4_peak = 4.0 * bf16_tf            # nominal fp4 : bf16 dense ratio 9 : 2.25
-    # solver roofline on the largest weight (one dq_solve_scales call: init +
-    # BCD launches).  Algorithmic work = 12 fp32 ops per element per round
-    # (two quantisations, two scale products, four reduction FMAs); ALU peak =
-    # 148 SMs x 128 fp32 lanes x max SM clock.
-    alu_peak = 148 * 128 * sm_max * 1e6 / 1e12  # T lane-ops/s
-    big_ms = sum(solve_big) / len(solve_big)
-    solver_alu = 12.0 * big * T / (big_ms * 1e-3) / 1e12
-    solver_gbs = T * sum(W.numel() * 2 for W in Wd) * args.steps / (solve_ms * 1e-3) / 1e9
-    # GEMM and activation quantiser rooflines on the prefill shape (M=4096,
-    # N=4096, K=4096), durations from the back-to-back per-kernel timing
-    K0 = Wd[0].shape[1]
-    j0 = max(range(len(Wd)), key=lambda j: Wd[j].shape[0])
-    t_act, t_gemm = kt[(prefill_M, j0)]
-    gemm_tf = 2.0 * prefill_M * Wd[j0].shape[0] * K0 / (t_gemm * 1e-6) / 1e12
-    a_bytes = prefill_M * K0 * (2 + 0.5 + 1.0 / 16) + prefill_M * 4
-    act_gbs = a_bytes / (t_act * 1e-6) / 1e9
-    # decode GEMM (M = 1, the largest weight): weight-bandwidth bound; bytes =
-    # codes N*K/2 + scales N*K/16 + A M*K/2 + A scales + Y 2*M*N
-    Md = min(Xd)
-    t_dec = kt[(Md, j0)][1]
-    Nd = Wd[j0].shape[0]
-    dec_bytes = Nd * K0 / 2 + Nd * K0 / 16 + Md * K0 / 2 + Md * K0 / 16 + 4 * Md + 2 * Md * Nd
-    dec_gbs = dec_bytes / (t_dec * 1e-6) / 1e9
-    # whole-job throughput: every rank runs the same per-GPU workload (weak
-    # scaling); the time is the slowest rank's
-    value = world * lin_flops * args.steps / (lin_ms * 1e-3) / 1e12
-
-    # 8-bit variant (Appendix G.2): the MXFP8 linear on the largest weight at
-    # the prefill shape -- solve, pack, then the activation quantiser and the
-    # GEMM timed like the others.  Auxiliary: an error is reported, not raised.
-    mxfp8 = None
-    try:
-        Wm = Wd[j0]
-        N8, K8 = Wm.shape
-        r8 = torch.empty((N8, K8 // 32), device=dev)
-        c8 = torch.empty(K8, device=dev)
-        s8 = torch.empty(1, device=dev)
-        dq.dq_solve_scales(Wm, dq.DQ_MXFP8, T, r8, c8, s8, None, ws, group=32)
-        B8 = torch.empty((N8, K8), dtype=torch.uint8, device=dev)
-        sB8 = torch.empty(dq.scales_bytes(N8, K8, dq.DQ_MXFP8, 32), dtype=torch.uint8, device=dev)
-        dq.dq_quantize_weight(Wm, dq.DQ_MXFP8, r8, c8, s8, B8, sB8, group=32)
-        X8 = Xd[prefill_M]
-        A8 = torch.empty((prefill_M, K8), dtype=torch.uint8, device=dev)
-        sA8 = torch.empty(dq.scales_bytes(prefill_M, K8, dq.DQ_MXFP8, 32), dtype=torch.uint8,
-                          device=dev)
-        Y8 = torch.empty((prefill_M, N8), dtype=torch.bfloat16, device=dev)
-        nx8 = max(2, min(16, -(-2 * L2_BYTES // (X8.numel() * 2))))
-        Xc8 = [X8.clone() for _ in range(nx8)]
-        t_act8 = per_launch_us(lambda i: dq.dq_quantize_act(
-            Xc8[i % nx8], dq.DQ_MXFP8, c8, A8, sA8, None, group=32), nx8)
-        nb8 = max(2, min(64, -(-2 * L2_BYTES // (B8.numel() + sB8.numel()))))
-        Bc8 = [(B8.clone(), sB8.clone()) for _ in range(nb8)]
-        t_gemm8 = per_launch_us(lambda i: dq.dq_w4a4_linear(
-            A8, sA8, None, Bc8[i][0], Bc8[i][1], None, Y8, dq.DQ_MXFP8), nb8)
-        err8 = dq.dq_device_error(clear=True)
-        fl8 = 2.0 * prefill_M * N8 * K8 / (t_gemm8 * 1e-6) / 1e12
-        a8_bytes = prefill_M * K8 * (2 + 1 + 1.0 / 32)
-        mxfp8 = {"shape": f"M={prefill_M} x N={N8} x K={K8}", "T": T,
-                 "gemm": {"kernel": "w4a4_gemm_mxint4_kernel<FP8>", "us_per_launch": t_gemm8,
-                          "achieved": fl8, "peak": 2.0 * bf16_tf, "unit": "TFLOP/s",
-                          "frac": fl8 / (2.0 * bf16_tf),
-                          "peak_kind": f"{peak_kind} bf16 burst x 2 (nominal fp8:bf16)"},
-                 "act_quant": {"us_per_launch": t_act8, "achieved": a8_bytes / (t_act8 * 1e-6) / 1e9,
-                               "peak": hbm, "unit": "GB/s",
-                               "frac": a8_bytes / (t_act8 * 1e-6) / 1e9 / hbm},
-                 "device_error": err8}
-        del Xc8, Bc8
-    except Exception as ex:  # auxiliary measurement: report, do not fail the bench line
-        mxfp8 = {"error": str(ex)[:300]}
-
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        oracle_prepare(wl, Ws)
-        v, secs = oracle_linear_sample(wl, Ws, Xs, rows=64)
-        sgbs, ssecs = oracle_solver_sample(wl, Ws)
+        oracle_prepare(Ws)
+        v, secs = oracle_linear_sample(Ws, Xs, Mp, rows=64)
+        procs = max(1, min(os.cpu_count() or 1, 32))
+        sol = oracle_solver_sample(Ws[0], T, procs)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": LINEAR_SAMPLE_DESC.format(rows=64), "seconds": secs,
-               "solver": {"gbs_effective": sgbs, "seconds": ssecs,
-                          "sample": "Algorithm 1, T=50, one 4096x16 tile, single thread"}}
+               "sample": LINEAR_SAMPLE_DESC.format(rows=64, M=Mp), "seconds": secs,
+               "solver": dict(sol, sample=f"Algorithm 1, T={T}, whole {Ws[0].shape[0]}x16 "
+                                          f"column tiles of the first weight: one tile on one "
+                                          f"core, one tile per process on {procs} processes")}
 
+    # dominant kernel of the step by device time: the solver
+    big = max(solver, key=lambda k: solver[k]["ms"])
+    m_, n_ = (int(v) for v in big.split("x"))
+    sb = solver[big]
+    first = f"N{Ls[0].W.shape[0]}_K{Ls[0].W.shape[1]}"
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4(e2m1)",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "format": FMT_NAME, "weights": [list(W.shape) for W in Ws],
-                   "M": sorted(Xd), "T": T, "l2": "flushed between steps (256 MiB write)",
+        "config": {"workload": WORKLOAD, "format": FMT_NAME,
+                   "weights": [list(L.W.shape) for L in Ls], "M_prefill": Mp, "M_decode": Mds,
+                   "T": T, "l2": "flushed before every step (256 MiB write, outside the timed "
+                                 "events); the linears run first in the step",
+                   "value": "prefill linears (act quant + GEMM), both weights",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "solve_bcd_kernel (+ solve_init_kernel), 4096x4096 bf16, T=50",
-                     "bound": "alu", "achieved": solver_alu, "peak": alu_peak, "unit": "Tops/s",
-                     "frac": solver_alu / alu_peak, "ms_per_launch": big_ms,
-                     "traffic": measured_traffic("solver_4096x4096_nvfp4_T50",
+        "roofline": {"kernel": f"solve_bcd_kernel (+ solve_init_kernel), {big} bf16, T={T}",
+                     "bound": "alu", "achieved": sb["tops"], "peak": alu_peak, "unit": "Tops/s",
+                     "frac": sb["frac_alu"], "ms_per_launch": sb["ms"],
+                     "share_of_step": solve_ms / step_ms,
+                     "traffic": measured_traffic(f"solver_{big}_nvfp4_T50",
                                                  ["dq_solver.cu", "dq_device.cuh"]),
-                     "algorithmic_bytes": big * 2 + big // 16 * 4 + 4096 * 4,
-                     "note": "12 algorithmic fp32 ops / element / round; peak = 148 SM x 128 "
-                             "fp32 lanes x max SM clock (derived, not measured)"},
-        "roofline_gemm": {"kernel": "w4a4_gemm_kernel", "bound": "tensor", "achieved": gemm_tf,
-                          "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
-                          "us_per_launch": t_gemm,
-                          "traffic": measured_traffic("gemm_nvfp4_4096x4096x4096",
+                     "algorithmic_bytes": m_ * n_ * 2 + m_ * n_ // 16 * 4 + n_ * 4,
+                     "peak_kind": "derived: 148 SM x 128 fp32 lanes x max SM clock",
+                     "note": "12 algorithmic fp32 ops / element / round"},
+        "roofline_gemm": {"kernel": "w4a4_gemm", "bound": "tensor",
+                          "achieved": prefill[first]["gemm_tflops"], "peak": fp4_peak,
+                          "unit": "TFLOP/s", "frac": prefill[first]["gemm_frac"],
+                          "us_per_launch": prefill[first]["gemm_us"],
+                          "shape": f"M={Mp} x N={Ls[0].W.shape[0]} x K={Ls[0].W.shape[1]}",
+                          "traffic": measured_traffic(f"gemm_nvfp4_{Mp}x{Ls[0].W.shape[0]}x"
+                                                      f"{Ls[0].W.shape[1]}",
                                                       ["dq_gemm.cu", "dq_device.cuh"]),
-                          "shape": f"M={prefill_M} x N={Wd[j0].shape[0]} x K={K0}",
                           "peak_kind": f"{peak_kind} bf16 burst x 4 (nominal fp4:bf16)"},
-        "roofline_act": {"kernel": "quantize_act_ring_kernel", "bound": "hbm",
-                         "achieved": act_gbs, "peak": hbm, "unit": "GB/s", "frac": act_gbs / hbm,
-                         "us_per_launch": t_act, "algorithmic_bytes": a_bytes,
-                         "traffic": measured_traffic("act_nvfp4_4096x4096",
-                                                     ["dq_quant.cu", "dq_device.cuh"]),
-                         "shape": f"M={prefill_M} x K=4096"},
-        "roofline_decode": {"kernel": "w4a4_gemm_splitk_kernel", "bound": "hbm",
-                            "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
-                            "frac": dec_gbs / hbm, "us_per_launch": t_dec,
-                            "algorithmic_bytes": dec_bytes,
-                            "shape": f"M={Md} x N={Nd} x K={K0}"},
-        "per_M_us": per_m,
+        "roofline_act": {"kernel": "quantize_act", "bound": "hbm",
+                         "achieved": prefill[first]["act_gbs"], "peak": hbm, "unit": "GB/s",
+                         "frac": prefill[first]["act_gbs"] / hbm,
+                         "us_per_launch": prefill[first]["act_us"],
+                         "algorithmic_bytes": act_bytes(Mp, Ls[0].W.shape[1], fmt, G),
+                         "shape": f"M={Mp} x K={Ls[0].W.shape[1]}",
+                         "traffic": measured_traffic(f"act_nvfp4_{Mp}x{Ls[0].W.shape[1]}",
+                                                     ["dq_quant.cu", "dq_device.cuh"])},
+        "solver": solver, "prefill": prefill, "decode": decode, "pack": pack,
         "per_kernel_timing": "after the timed steps: launches back to back between two events, "
-                             "each on its own copy of the inputs (copies > 2x L2)",
+                             "each on its own copy of its input (copies > 2x L2)",
+        "step_ms": {"prefill_linears": pre_ms / args.steps, "decode_linears": dec_ms / args.steps,
+                    "solve": solve_ms / args.steps},
         "solver_modes": {
-            "weight": list(Wb.shape), "T": T, "ms_per_call": mode_ms,
-            "achieved_tops": {k: (12.0 if k == "both" else 6.0) * Wb.numel() * T
-                              / (v * 1e-3) / 1e12 for k, v in mode_ms.items()},
-            "frac_alu": {k: (12.0 if k == "both" else 6.0) * Wb.numel() * T
+            "weight": list(L0.W.shape), "T": T, "ms_per_call": mode_ms,
+            "frac_alu": {k: (12.0 if k == "both" else 6.0) * L0.W.numel() * T
                          / (v * 1e-3) / 1e12 / alu_peak for k, v in mode_ms.items()},
             "note": "Table 4 arms through dq_solve_scales_ex; algorithmic fp32 ops per "
                     "element per round: 12 (both half-steps), 6 (one half-step)"},
-        "solver_batched": {"ms_per_layer": batched_ms, "T": T,
-                           "weights": "q, k, v, o 4096/1024 x 4096; gate, up 14336 x 4096; "
-                                      "down 4096 x 14336 (one Llama-3.1-8B layer)",
-                           "launches": {"separate": 14, "batched": 6}},
+        "configs": configs,
         "mxfp8": mxfp8,
-        "act_sqnr": {"per_weight": act_sqnr, "rows": prefill_M,
+        "act_sqnr": {"per_weight": act_sqnr, "rows": Mp,
                      "note": "SQNR of the dequantised activations mapped back by 1/c vs X, "
-                             "measured on the device (dq_act_quant_error); synthetic "
-                             "activations and weights, so the sign of the delta is not the "
-                             "paper's model result"},
-        "solver": {"gbs_effective": solver_gbs, "frac_hbm": solver_gbs / hbm,
-                   "ms_per_weight_set": solve_ms / args.steps,
-                   "definition": "T * bytes(W bf16) / solver time (tile stays on chip)"},
-        "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16_tf, "kind": peak_kind},
+                             "measured on the device (dq_act_quant_error); synthetic inputs"},
+        "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16_tf, "fp4_tflops": fp4_peak,
+                  "fp8_tflops": fp8_peak, "alu_tops": alu_peak, "kind": peak_kind},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "e2e": e2e,
@@ -593,10 +735,12 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the other workloads and the MXFP8 line")
     args = ap.parse_args()
     rank, world, local_rank = dist.env_ranks()
     if args.warmup < 3 and args.impl == "ours":

@@ -357,6 +357,18 @@ DQ_API int dq_solve_scales_noalloc(const void* W, dq_dtype wt, int64_t m, int64_
  * (0 = none).  Synchronises the current device; clear != 0 resets it. */
 DQ_API int dq_device_error(int clear);
 
+/* Time limit, in nanoseconds, of the bounded waits inside the GEMM and
+ * activation-quantiser pipelines on the current device (default 2 s; ns = 0
+ * restores the default).  Diagnostic: the paper has no counterpart.  A wait
+ * that runs out sets the device error word to DQ_ERR_DEVICE_TIMEOUT and the
+ * kernel unwinds -- every role first waits, with a fixed 2 s limit, for the
+ * copies and tensor-core work it has already issued, then the CTA releases
+ * its tensor memory and exits; the outputs of that call are undefined.  A
+ * very small limit makes the waits of a normal call expire, which is how the
+ * unwinding is tested.  Synchronises the device; do not call it while
+ * another thread has work of this library in flight. */
+DQ_API int dq_set_wait_limit(uint64_t ns);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 DQ_API int dq_version(void);
 

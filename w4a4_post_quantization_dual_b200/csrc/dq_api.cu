@@ -246,4 +246,11 @@ int dq_w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, cons
 
 int dq_device_error(int clear) { return dq::read_device_error(clear); }
 
+int dq_set_wait_limit(uint64_t ns) {
+  const unsigned long long v = ns ? (unsigned long long)ns : 2000000000ull;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DQ_ERR_CUDA;
+  const int a = dq::set_gemm_wait_limit(v), b = dq::set_quant_wait_limit(v);
+  return a != DQ_OK ? a : b;
+}
+
 }  // extern "C"

@@ -36,6 +36,10 @@
 namespace dq {
 
 __device__ int g_dq_device_error = 0;
+// Time limit of the bounded mbarrier waits of the pipelines, in ns: 2 s by
+// default, far beyond any legitimate wait.  dq_set_wait_limit changes it
+// (a test makes the waits expire to exercise the unwinding below).
+__device__ unsigned long long g_dq_wait_limit_ns = 2000000000ull;
 
 namespace gemm {
 
@@ -49,7 +53,10 @@ constexpr int NUM_THREADS = 320;
 // (6..9) therefore share each stage's scale atoms round-robin.
 constexpr int COPIERS = 4;
 constexpr int FIRST_COPIER = 6;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
+// Limit of the waits that unwind a CTA after an expiry: fixed, whatever the
+// pipeline limit, because they only wait for work that was issued and will
+// complete on its own.
+constexpr uint64_t DRAIN_LIMIT_NS = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -79,18 +86,68 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait: returns false (and raises the abort flag) if the phase does
-// not complete within WAIT_LIMIT_NS or another role already aborted.
+// not complete within the pipeline limit or another role already aborted.
 __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t lim = *reinterpret_cast<volatile unsigned long long*>(&g_dq_wait_limit_ns);
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+    if (globaltimer() - t0 > lim) {
       *abort_flag = 1;
       atomicExch(&g_dq_device_error, DQ_ERR_DEVICE_TIMEOUT);
       return false;
     }
+  }
+}
+// Bounded wait with the fixed limit that ignores the abort flag: a role
+// whose progress must not depend on another role's abort (the producers of
+// the paired-SM kernel, whose loads are counted on one CTA's barrier).
+__device__ __noinline__ bool mbar_wait_fixed(uint64_t* bar, uint32_t parity,
+                                             volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > DRAIN_LIMIT_NS) {
+      *abort_flag = 1;
+      atomicExch(&g_dq_device_error, DQ_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+// Unwinding wait: for a phase that work already issued will complete (loads
+// that landed or are in flight, a commit after issued tensor-core work).
+// Ignores the abort flag; bounded by the fixed limit.
+__device__ __noinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > DRAIN_LIMIT_NS) {
+      atomicExch(&g_dq_device_error, DQ_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+// A producer's unwinding: wait until the loads of the last `issued` stages
+// (at most STAGES) before ring position (stage, phase) -- the next slot it
+// would have filled -- have landed, on `full` (and `full2`, nullable).  A
+// stage filled at phase p completes its barrier's phase of parity p, and no
+// later fill of the stage was issued, so the wait is unambiguous.
+template <int STAGES>
+__device__ __forceinline__ void drain_loads(uint64_t* full, uint64_t* full2, int stage,
+                                            uint32_t phase, int issued) {
+  for (int i = 0; i < issued && i < STAGES; ++i) {
+    if (stage == 0) {
+      stage = STAGES - 1;
+      phase ^= 1u;
+    } else {
+      --stage;
+    }
+    mbar_drain(&full[stage], phase);
+    if (full2) mbar_drain(&full2[stage], phase);
   }
 }
 
@@ -194,7 +251,7 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = (227 * 1024 - 1024 - 256 - RESERVE) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + RESERVE;
-  static_assert(4 * STAGES * 8 + 32 <= 256, "barrier area");
+  static_assert(4 * STAGES * 8 + 40 <= 256, "barrier area");
   // tensor-memory columns: accumulator, then one scale slot per stage
   // (SFA: 4 columns per atom; SFB: 4 columns per atom and 128-row group)
   static constexpr int SF_COLS = 4 * SF_ATOMS * (1 + BN / 128);
@@ -265,6 +322,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+  uint64_t* drain = acc_empty + 2;   // tensor-core work of the MMA and copier threads done
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -285,6 +343,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
+    mbar_init(drain, 1 + COPIERS);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -333,6 +392,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       uint32_t phase = 0;
       bool ok = true;
       bool first = true;
+      int issued = 0;   // stages whose loads were all issued
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, first = false) {
         const int tm = tile % tiles_m, tn = tile / tiles_m;
         const int m0 = tm * BM, n0 = tn * BN;
@@ -347,16 +407,22 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     sfA + ((size_t)(m0 / 128) * S4 + (size_t)kt * C::SF_ATOMS) * 512,
                     C::SFA_BYTES, &sffull[stage]);
           tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kt * BKB, m0);
+          ++issued;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
-      // drain: every issued stage must land before the CTA may exit
+      // every stage consumed by the MMAs (normal end) ...
+      const int stage_end = stage;
+      const uint32_t phase_end = phase;
       if (ok) {
         for (int s = 0; s < C::STAGES; ++s) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // ... and, whatever happened, every issued load landed before the CTA
+      // may exit (an expired wait leaves stages unconsumed)
+      drain_loads<C::STAGES>(full, sffull, stage_end, phase_end, issued);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -402,6 +468,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (!ok) break;
         mma_commit(acc_full);
       }
+      // the MMAs issued so far have completed before the CTA may exit
+      mma_commit(drain);
+      mbar_drain(drain, 0);
     }
   } else if (warp >= FIRST_COPIER && warp < FIRST_COPIER + COPIERS) {
     // ------------------------------------------------------------ scale copiers
@@ -434,6 +503,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      mma_commit(drain);   // this copier's scale copies have completed
+      mbar_drain(drain, 0);
     }
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue
@@ -576,6 +647,7 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
   uint64_t* acc_full = sfready + C::STAGES;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+  uint64_t* drain = acc_full + 2;  // tensor-core work of the MMA and copier threads done
   __shared__ float s_rs[BM];       // per-row output scale
   __shared__ float s_rr[SK_BN];    // per-output-column factor of this tile
   __shared__ float s_pamax[FUSED ? BM : 1];   // FUSED: this CTA's row maxima of |x c|
@@ -599,6 +671,7 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
       mbar_init(&sfready[s], COPIERS);
     }
     mbar_init(acc_full, 1);
+    mbar_init(drain, 1 + COPIERS);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -677,6 +750,7 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
       pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
+      int issued = 0;
       for (int kt = 0; kt < kt_per_slice; ++kt) {
         if (kt >= pre) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
@@ -687,12 +761,22 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
         bulk_load(sSFA + stage * C::SFA_BYTES,
                   sfA + ((size_t)(m0 / 128) * S4 + (size_t)(kt0 + kt) * C::SF_ATOMS) * 512,
                   C::SFA_BYTES, &full[stage]);
+        ++issued;
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
-      for (int s = 0; s < C::STAGES; ++s) {  // drain: every issued stage lands before exit
+      const int stage_end = stage;
+      const uint32_t phase_end = phase;
+      for (int s = 0; s < C::STAGES; ++s) {  // every issued stage consumed (normal end)
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
+      // every issued load landed before the CTA may exit
+      drain_loads<C::STAGES>(full, nullptr, stage_end, phase_end, issued);
+    }
+    if (FUSED && lane == 0) {
+      // the weights of every k-tile were issued up front; full[kt] also
+      // counts the A-producer warps, which never wait on a limit
+      for (int kt = 0; kt < kt_per_slice; ++kt) mbar_drain(&full[kt], 0);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -730,6 +814,8 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
       if (ok) mma_commit(acc_full);
+      mma_commit(drain);   // the MMAs issued so far have completed before exit
+      mbar_drain(drain, 0);
     }
   } else {
     // warps 2..5 and the copier warps 6..9 drain the partial tile after the
@@ -756,6 +842,8 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
         mma_commit(&sfready[stage]);
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
+      mma_commit(drain);   // this copier's scale copies have completed
+      mbar_drain(drain, 0);
     }
     __syncwarp();
     const int quad = warp & 3;
@@ -923,7 +1011,7 @@ struct Cfg2 {
   static constexpr int TMEM_COLS = 512;
   static constexpr int K_STEPS = BK / 64;
   static_assert(SF_BASE + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
-  static_assert(4 * STAGES * 8 + 32 <= 256, "barrier area");
+  static_assert(4 * STAGES * 8 + 40 <= 256, "barrier area");
   static_assert(STAGES >= 3, "pipeline depth");
 };
 
@@ -996,10 +1084,11 @@ __device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity)
 __device__ __noinline__ bool wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t lim = *reinterpret_cast<volatile unsigned long long*>(&g_dq_wait_limit_ns);
   while (true) {
     if (try_wait_cluster(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+    if (globaltimer() - t0 > lim) {
       *abort_flag = 1;
       atomicExch(&g_dq_device_error, DQ_ERR_DEVICE_TIMEOUT);
       return false;
@@ -1036,6 +1125,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+  uint64_t* drain = acc_empty + 2;   // leader: its tensor-core work done
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();            // 0: leader, 1: peer
@@ -1059,6 +1149,7 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);                       // 4 epilogue warps in each CTA
+    mbar_init(drain, 1 + COPIERS);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1098,13 +1189,19 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       uint32_t phase = 0;
       bool ok = true;
       bool first = true;
+      int issued = 0;
       for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs, first = false) {
         const int tm = tile % tiles_m, tn = tile / tiles_m;
         const int m_own = tm * 256 + (int)rank * 128;
         for (int kt = 0; kt < KT; ++kt) {
           const uint32_t bar = pair::mapa(smem_u32(&full[stage]), 0);
           if (!(first && kt < pre)) {
-            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+            // both producers see the same phases of their empty barriers (the
+            // leader's commits arrive on both at once) and give up only on the
+            // fixed limit, never on an abort flag: so the two CTAs always fill
+            // the same stages, and the leader's barrier, which counts both
+            // CTAs' bytes, completes for every stage either of them filled
+            if (!mbar_wait_fixed(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
             if (leader) mbar_expect_tx(&full[stage], TX);
             load_b(stage, tn, kt);
           }
@@ -1112,9 +1209,13 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           // scale atoms as rows of 256 bytes: atom a of row block rb is rows 2a, 2a + 1
           pair::tma_load_2d_pair(sSFA + stage * C::SFA_BYTES, &tmSFA, bar, 0,
                                  2 * ((m_own / 128) * S4 + kt * C::SF_ATOMS));
+          ++issued;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // the leader waits until both CTAs' loads of every filled stage have
+      // landed; the peer leaves only after the cluster barrier at the end
+      if (leader) drain_loads<C::STAGES>(full, nullptr, stage, phase, issued);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
@@ -1159,6 +1260,10 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         if (!ok) break;
         pair::commit_both(acc_full);
       }
+      // the MMAs issued into both CTAs' tensor memory have completed before
+      // either CTA leaves (the peer waits at the cluster barrier)
+      pair::commit_leader(drain);
+      mbar_drain(drain, 0);
     }
   } else if (warp >= FIRST_COPIER && warp < FIRST_COPIER + COPIERS) {
     // ------------------------------------------------------------ scale copiers (leader)
@@ -1189,6 +1294,8 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      pair::commit_leader(drain);   // this copier's scale copies have completed
+      mbar_drain(drain, 0);
     }
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue (both)
@@ -1380,6 +1487,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+  uint64_t* drain = acc_empty + 2;   // tensor-core work of the MMA and copier threads done
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (M + BM - 1) / BM, tiles_n = N / BN, num_tiles = tiles_m * tiles_n;
@@ -1397,6 +1505,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
+    mbar_init(drain, 2);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1417,10 +1526,12 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int issued = 0;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          ++issued;   // every load of the stage is issued below, with no wait in between
           if constexpr (I8) {          // int8 staging, 64 bytes per row; no scale copies
             mbar_expect_tx(&full[stage], STG_A + STG_B);
             tma_load_2d(stA + stage * STG_A, &tmA, &full[stage], kt * KTE, m0);
@@ -1443,11 +1554,15 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      const int stage_end = stage;
+      const uint32_t phase_end = phase;
       if (ok)
         for (int s = 0; s < STAGES; ++s) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
+      // every issued load landed before the CTA may exit
+      drain_loads<STAGES>(full, nullptr, stage_end, phase_end, issued);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -1499,12 +1614,14 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
         if (!ok) break;
         mma_commit(acc_full);
       }
+      mma_commit(drain);   // the MMAs issued so far have completed before exit
+      mbar_drain(drain, 0);
     }
   } else if (warp == 6) {
-    if (lane == 0 && !I8) {
+    if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < num_tiles && !I8; tile += gridDim.x) {
         bool ok = true;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
@@ -1517,6 +1634,8 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         if (!ok) break;
       }
+      mma_commit(drain);   // the scale copies have completed (none for MXINT8)
+      mbar_drain(drain, 0);
     }
   } else if (warp >= 7) {
     if constexpr (I8) {
@@ -1973,6 +2092,11 @@ int w4a4_linear_fused(const void* X, const float* c, const uint8_t* B, const uin
   const __nv_bfloat16* Xb = reinterpret_cast<const __nv_bfloat16*>(X);
   return yt == 1 ? gemm::launch_splitk_fused<1>(Xb, c, B, sB, s_w, r_row, Y, M, N, K, S, st)
                  : gemm::launch_splitk_fused<0>(Xb, c, B, sB, s_w, r_row, Y, M, N, K, S, st);
+}
+
+int set_gemm_wait_limit(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_dq_wait_limit_ns, &ns, sizeof(ns)) == cudaSuccess ? DQ_OK
+                                                                                 : DQ_ERR_CUDA;
 }
 
 int read_device_error(int clear) {

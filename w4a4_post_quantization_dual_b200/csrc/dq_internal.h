@@ -81,5 +81,8 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 // (one per translation unit); read_device_error combines them.
 int read_device_error(int clear);
 int read_quant_error(int clear);
+// Time limits of the bounded waits (ns) of the GEMM and quantiser kernels.
+int set_gemm_wait_limit(unsigned long long ns);
+int set_quant_wait_limit(unsigned long long ns);
 
 }  // namespace dq

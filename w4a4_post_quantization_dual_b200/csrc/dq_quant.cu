@@ -354,25 +354,45 @@ quantize_act_rows_kernel(const XT* __restrict__ X, int64_t M, int64_t Mpad, int6
 // on it) and the packed code words are rotated back before the store.
 // ---------------------------------------------------------------------------
 __device__ int g_dq_quant_error = 0;
+// Time limit of the ring's bounded waits, in ns (2 s by default, far beyond
+// any legitimate wait; dq_set_wait_limit changes it for testing).  The waits
+// that unwind a CTA after an expiry keep the fixed 2 s.
+__device__ unsigned long long g_dq_quant_wait_limit_ns = 2000000000ull;
 
 namespace aq {
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
-__device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity) {
-  const uint64_t limit = 2000000000ull;  // 2 s, far beyond any legitimate wait
-  uint64_t t0 = 0;
-  for (int i = 0;; ++i) {
-    uint32_t ok;
+__device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity,
+                                            bool fixed_limit = false) {
+  uint32_t ok;
+  // usual case: the stage landed while the previous ones were processed
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  if (ok) return true;
+  const uint64_t limit =
+      fixed_limit ? 2000000000ull
+                  : *reinterpret_cast<volatile unsigned long long*>(&g_dq_quant_wait_limit_ns);
+  // elapsed time: the larger of the global timer (coarse ticks) and the SM
+  // cycle counter at two cycles per ns (resolution for very small limits)
+  uint64_t t0, c0, t, cyc;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  c0 = clock64();
+  while (true) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-    if (ok) return true;
-    uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    if (i == 0) t0 = t;
-    else if (t - t0 > limit) {
+    cyc = (clock64() - c0) >> 1;
+    const uint64_t el = (t - t0) > cyc ? (t - t0) : cyc;
+    // a pipeline wait that outlasted its limit counts as expired even if the
+    // phase completed meanwhile (try_wait may suspend until it does); an
+    // unwinding wait only needs the phase
+    if (ok && (fixed_limit || el <= limit)) return true;
+    if (el > limit) {
       atomicExch(&g_dq_quant_error, DQ_ERR_DEVICE_TIMEOUT);
       return false;
     }
@@ -496,7 +516,38 @@ __device__ __forceinline__ float act_block_load(const unsigned char* bp, const f
   return m[0];
 }
 
-template <int F, int G, int BPT, int MAXT, int MINB>
+// x~ = x*c for one block, the column scales from the shared-memory copy cT:
+// piece q (4 floats) of block s at float4 index q * S + s, so that the lanes
+// of a wavefront (consecutive blocks, in the rotated piece order of x) read
+// disjoint banks.
+template <int G>
+__device__ __forceinline__ float act_block_load_cs(const unsigned char* bp, const float4* cT,
+                                                   int S, int s, int rot, float2* xt) {
+  constexpr int P = G / 8, H = G / 2;
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    const int q = (p + rot) & (P - 1);
+    const uint4 v = *reinterpret_cast<const uint4*>(bp + 16 * q);
+    const float4 c0 = cT[(2 * q) * S + s], c1 = cT[(2 * q + 1) * S + s];
+    xt[4 * p + 0] = __fmul2_rn(aq::bf16pair(v.x), make_float2(c0.x, c0.y));
+    xt[4 * p + 1] = __fmul2_rn(aq::bf16pair(v.y), make_float2(c0.z, c0.w));
+    xt[4 * p + 2] = __fmul2_rn(aq::bf16pair(v.z), make_float2(c1.x, c1.y));
+    xt[4 * p + 3] = __fmul2_rn(aq::bf16pair(v.w), make_float2(c1.z, c1.w));
+  }
+  float m[H / 2];
+#pragma unroll
+  for (int h = 0; h < H / 2; ++h) m[h] = fmaxf(aq::absmax2(xt[2 * h]), aq::absmax2(xt[2 * h + 1]));
+#pragma unroll
+  for (int w = H / 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int h = 0; h < w; ++h) m[h] = fmaxf(m[h], m[h + w]);
+  return m[0];
+}
+
+// CSM: the column scales live in shared memory (loaded once per CTA) instead
+// of registers, so that rows of more blocks keep their rescaled values in
+// registers: long rows (K up to ~28K), one row per stage.
+template <int F, int G, int BPT, int MAXT, int MINB, bool CSM = false>
 __global__ void __launch_bounds__(MAXT, MINB)
 quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t Mpad, int64_t K,
                          const float* __restrict__ c, uint8_t* __restrict__ codes,
@@ -508,7 +559,10 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const uint32_t row_bytes = (uint32_t)K * 2;
   const uint32_t stage_bytes = row_bytes * (uint32_t)RT;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + (size_t)stage_bytes * NST);
+  // CSM: [column scales, K floats][stages]; else [stages]
+  const float4* cT = reinterpret_cast<const float4*>(smem_raw);
+  unsigned char* stages = smem_raw + (CSM ? (size_t)K * 4 : 0);
+  uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)stage_bytes * NST);
   uint32_t* rowmax = reinterpret_cast<uint32_t*>(full + NST);  // [3][16] fp32 bits, >= 0
   volatile int* abort_flag = reinterpret_cast<volatile int*>(rowmax + 48);
 
@@ -539,20 +593,30 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
   // column scales of the owned blocks, in the rotated piece order: c comes
   // from the solver, never from the kernel launched just before this one, so
   // it is read ahead of the dependency wait (X and the outputs after it)
-  float2 cv[BPT][H];
+  float2 cv[CSM ? 1 : BPT][H];
+  if constexpr (CSM) {
+    // column scales into shared memory, piece-transposed (see act_block_load_cs)
+    float4* cw = reinterpret_cast<float4*>(smem_raw);
+    for (int i = tid; i < S * (G / 4); i += blockDim.x) {
+      const int sb = i / (G / 4), q = i % (G / 4);
+      cw[q * S + sb] = c ? __ldg(reinterpret_cast<const float4*>(c) + i)
+                         : make_float4(1.f, 1.f, 1.f, 1.f);
+    }
+  } else {
 #pragma unroll
-  for (int j = 0; j < BPT; ++j) {
-    const int s = tl + j * NTS;
+    for (int j = 0; j < BPT; ++j) {
+      const int s = tl + j * NTS;
 #pragma unroll
-    for (int p = 0; p < P; ++p) {
-      const int q = (p + rot) & (P - 1);
+      for (int p = 0; p < P; ++p) {
+        const int q = (p + rot) & (P - 1);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float4 v = (c && own[j])
-                             ? __ldg(reinterpret_cast<const float4*>(c + (int64_t)s * G + q * 8) + h)
-                             : make_float4(1.f, 1.f, 1.f, 1.f);
-        cv[j][4 * p + 2 * h] = make_float2(v.x, v.y);
-        cv[j][4 * p + 2 * h + 1] = make_float2(v.z, v.w);
+        for (int h = 0; h < 2; ++h) {
+          const float4 v = (c && own[j])
+                               ? __ldg(reinterpret_cast<const float4*>(c + (int64_t)s * G + q * 8) + h)
+                               : make_float4(1.f, 1.f, 1.f, 1.f);
+          cv[j][4 * p + 2 * h] = make_float2(v.x, v.y);
+          cv[j][4 * p + 2 * h + 1] = make_float2(v.z, v.w);
+        }
       }
     }
   }
@@ -569,7 +633,7 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
                        aq::smem_u32(bar)), "r"(bytes) : "memory");
       asm volatile(
           "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-              "r"(aq::smem_u32(smem_raw + (size_t)stg * stage_bytes)),
+              "r"(aq::smem_u32(stages + (size_t)stg * stage_bytes)),
           "l"(X + t0 * K), "r"(bytes), "r"(aq::smem_u32(bar))
           : "memory");
     } else {  // padding rows only: nothing to load
@@ -587,7 +651,7 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
     const int64_t t = t0 + rt;
     const bool rowv = t < M, rowp = t < Mpad;  // both uniform over a warp
     if (!aq::wait_parity(&full[stg], phase)) *abort_flag = 1;
-    const unsigned char* sp = smem_raw + (size_t)stg * stage_bytes;
+    const unsigned char* sp = stages + (size_t)stg * stage_bytes;
     uint8_t* crow = codes + t * (K / 2);
     uint8_t* sfrow = scales + ((((t >> 7) * S4) << 9) + ((t & 31) << 4) + (((t & 127) >> 5) << 2));
 
@@ -599,7 +663,10 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
 #pragma unroll
       for (int j = 0; j < BPT; ++j) {
         ab[j] = 0.0f;
-        if (rowv && own[j]) ab[j] = act_block_load<G>(sp + boff[j], cv[j], rot, xt[j]);
+        if (rowv && own[j]) {
+          if constexpr (CSM) ab[j] = act_block_load_cs<G>(sp + boff[j], cT, S, tl + j * NTS, rot, xt[j]);
+          else ab[j] = act_block_load<G>(sp + boff[j], cv[j], rot, xt[j]);
+        }
         amax = fmaxf(amax, ab[j]);
       }
       // maxima are >= 0, so their bit patterns order like the values
@@ -638,7 +705,9 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
           uint32_t byte = 0;
           if (rowv && own[j]) {
             float2 xt[H];
-            const float ab = act_block_load<G>(sp + boff[j], cv[j], rot, xt);
+            float ab;
+            if constexpr (CSM) ab = act_block_load_cs<G>(sp + boff[j], cT, S, tl + j * NTS, rot, xt);
+            else ab = act_block_load<G>(sp + boff[j], cv[j], rot, xt);
             float inv;
             bool zero;
             act_block_scale<F>(ab, 0.0f, 0.0f, byte, inv, zero);
@@ -663,58 +732,79 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
     for (int k = 0; k < NST; ++k) {
       const int sk = stg + k < NST ? stg + k : stg + k - NST;
       const uint32_t pk = stg + k < NST ? phase : phase ^ 1u;
-      if (t0 + k * step < M) aq::wait_parity(&full[sk], pk);
+      if (t0 + k * step < M) aq::wait_parity(&full[sk], pk, true);
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// Weight packer: one thread per (row, block).
+// Weight packer: one CTA per tile of 128 rows x 32 row-blocks (eight 512-byte
+// scale atoms of the tensor-core layout).  Lane l of each warp takes block l
+// of the tile, so a warp reads and writes one row's 32 consecutive blocks
+// contiguously; the 8 warps step through the 128 rows.  beta = fl(1/c) of
+// the tile's columns is computed once into shared memory (transposed:
+// element k of every lane's block side by side, so the lanes read distinct
+// banks); the quantiser argument is fl(fl(w * beta) * alpha), alpha =
+// fl(1/r).  The scale atoms are assembled in shared memory and stored
+// whole; rows past m and blocks past n/G get zero scale bytes (the layout's
+// padding) and no codes.  INT4 / INT8 scales are bf16, row-major.
 // ---------------------------------------------------------------------------
 template <int F, int G, typename WT>
 __global__ void __launch_bounds__(256)
 pack_weight_kernel(const WT* __restrict__ W, int64_t m, int64_t n, const float* __restrict__ r,
                    const float* __restrict__ c, const float* __restrict__ sTp,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  constexpr int TB = 32;                  // blocks per tile, one per lane
+  constexpr int CH = G < 32 ? G : 32;     // elements per chunk of a block
+  constexpr bool LAYOUT = F != INT4 && F != INT8;
+  __shared__ float beta_t[G * TB];        // [element k of a block][lane]
+  __shared__ __align__(16) uint8_t atoms[LAYOUT ? 8 * 512 : 16];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t nb = n / G;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= m * nb) return;
-  const int64_t i = idx / nb, b = idx % nb;
-  const float rr = r[idx];
-  const float alpha = __frcp_rn(rr);
-  float x[G], z[G];
-  if constexpr (sizeof(WT) == 2) {
+  const int64_t r0 = (int64_t)blockIdx.x * 128, b0 = (int64_t)blockIdx.y * TB;
+  for (int k = tid; k < TB * G; k += 256) {   // k = block-in-tile * G + element
+    const int64_t col = b0 * G + k;
+    beta_t[(k % G) * TB + k / G] = col < n ? __frcp_rn(__ldg(c + col)) : 0.0f;
+  }
+  const float sT = (F == NVFP4) ? *sTp : 1.0f;
+  __syncthreads();
+  const int64_t b = b0 + lane;
+#pragma unroll 1
+  for (int rr = warp; rr < 128; rr += 8) {
+    const int64_t i = r0 + rr;
+    uint32_t byte = 0;
+    if (i < m && b < nb) {
+      const float rv = r[i * nb + b];
+      const float alpha = __frcp_rn(rv);
 #pragma unroll
-    for (int u = 0; u < G / 8; ++u)
-      bf16x8_to_f32(__ldcs(reinterpret_cast<const uint4*>(W + i * n + b * G) + u), x + 8 * u);
-  } else {
+      for (int h = 0; h < G / CH; ++h) {
+        float x[CH], z[CH];
+        load_block<WT, CH>(W + i * n + b * G + h * CH, x);
 #pragma unroll
-    for (int u = 0; u < G / 4; ++u) {
-      float4 v = __ldcs(reinterpret_cast<const float4*>(W + i * n + b * G) + u);
-      x[4 * u] = v.x; x[4 * u + 1] = v.y; x[4 * u + 2] = v.z; x[4 * u + 3] = v.w;
+        for (int k = 0; k < CH; ++k)
+          z[k] = __fmul_rn(__fmul_rn(x[k], beta_t[(h * CH + k) * TB + lane]), alpha);
+        if constexpr (is_8bit(F)) store_codes8<F, CH>(codes + i * n + b * G + h * CH, z);
+        else store_codes<F, CH>(codes + i * (n / 2) + b * (G / 2) + h * (CH / 2), z);
+      }
+      if constexpr (F == NVFP4) {
+        byte = ue4m3_rn(__fdiv_rn(rv, sT));
+      } else if constexpr (is_mx(F)) {
+        const uint32_t e = (__float_as_uint(rv) >> 23) & 0xFFu;  // exponent of a power of two
+        byte = e > 254u ? 254u : e;
+      } else {
+        reinterpret_cast<__nv_bfloat16*>(scales)[i * nb + b] = __float2bfloat16_rn(rv);
+      }
     }
+    // byte (row % 32) * 16 + ((row % 128) / 32) * 4 + (block % 4) of atom block / 4
+    if constexpr (LAYOUT) atoms[(lane >> 2) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (lane & 3)] = (uint8_t)byte;
   }
-#pragma unroll
-  for (int k = 0; k < G; ++k)
-    z[k] = __fmul_rn(__fmul_rn(x[k], __frcp_rn(__ldg(c + b * G + k))), alpha);
-  if constexpr (is_8bit(F)) store_codes8<F, G>(codes + i * n + b * G, z);
-  else store_codes<F, G>(codes + i * (n / 2) + b * (G / 2), z);
-  if constexpr (F == NVFP4) {
-    scales[sf_offset(i, b, nb)] = (uint8_t)ue4m3_rn(__fdiv_rn(rr, *sTp));
-  } else if constexpr (is_mx(F)) {
-    uint32_t e = (__float_as_uint(rr) >> 23) & 0xFFu;  // exponent of a power of two
-    scales[sf_offset(i, b, nb)] = (uint8_t)(e > 254u ? 254u : e);
-  } else {
-    reinterpret_cast<__nv_bfloat16*>(scales)[idx] = __float2bfloat16_rn(rr);
+  if constexpr (LAYOUT) {
+    __syncthreads();
+    const int64_t S4 = (nb + 3) / 4, a = b0 / 4 + (tid >> 5);
+    if (a < S4)
+      reinterpret_cast<uint4*>(scales + ((int64_t)blockIdx.x * S4 + a) * 512)[lane] =
+          reinterpret_cast<const uint4*>(atoms + (tid >> 5) * 512)[lane];
   }
-}
-
-// Zero the padding of a tensor-core scale buffer (rows m..Mpad-1 and the
-// scale columns beyond n/G inside the last atom column).
-__global__ void zero_bytes_kernel(uint8_t* p, int64_t nbytes) {
-  int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 16;
-  if (i + 16 <= nbytes) *reinterpret_cast<uint4*>(p + i) = make_uint4(0, 0, 0, 0);
-  else for (int64_t k = i; k < nbytes; ++k) p[k] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -761,15 +851,35 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
                       s_tok, NTS, RT, NST);
         return e == cudaSuccess ? (int)DQ_OK : (int)DQ_ERR_CUDA;
       };
+      // long rows: column scales in shared memory, one row per stage, up to
+      // BPT2 blocks per thread in registers (at most 512 threads)
+      auto ring_long = [&](auto kern, int bpt2) -> int {
+        const int NTS = (int)((S + bpt2 - 1) / bpt2 + 31) / 32 * 32;
+        const size_t stage = (size_t)K * sizeof(XT), cbytes = (size_t)K * 4;
+        if (NTS > 512 || cbytes + 2 * stage + 8 * 8 + 48 * 4 + 16 > 227 * 1024) return -1;
+        int NST = (int)((227 * 1024 - cbytes - 8 * 8 - 48 * 4 - 16) / stage);
+        NST = NST > 8 ? 8 : NST;
+        const size_t smem = cbytes + stage * NST + 8 * NST + 48 * 4 + 16;
+        int64_t grid = Mpad;
+        if (grid > (int64_t)num_sms()) grid = num_sms();
+        if (!ensure_kernel_attrs((const void*)kern, (int)smem, false)) return (int)DQ_ERR_CUDA;
+        const cudaError_t e =
+            launch_ex(kern, dim3((unsigned)grid), dim3(NTS), smem, st, 1,
+                      reinterpret_cast<const __nv_bfloat16*>(X), M, Mpad, K, c, codes, scales,
+                      s_tok, NTS, 1, NST);
+        return e == cudaSuccess ? (int)DQ_OK : (int)DQ_ERR_CUDA;
+      };
       int rc = -1;
       if constexpr (F == NVFP4) {
         // two blocks per thread halve the per-row overhead per element once
         // a row has enough blocks to keep 128+ threads busy
         if (S >= 256 && S <= 1024) rc = ring(quantize_act_ring_kernel<F, G, 2, 512, 1>, 2, 512, 1);
         else if (S <= 512) rc = ring(quantize_act_ring_kernel<F, G, 1, 512, 2>, 1, 512, 2);
+        else rc = ring_long(quantize_act_ring_kernel<F, G, 4, 512, 1, true>, 4);
       } else {
         if (S <= 384) rc = ring(quantize_act_ring_kernel<F, G, 1, 384, 2>, 1, 384, 2);
         else if (S <= 512) rc = ring(quantize_act_ring_kernel<F, G, 1, 512, 1>, 1, 512, 1);
+        else rc = ring_long(quantize_act_ring_kernel<F, G, 2, 512, 1, true>, 2);
       }
       if (rc >= 0) return rc;
     }
@@ -836,6 +946,11 @@ int read_quant_error(int clear) {
   return v;
 }
 
+int set_quant_wait_limit(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_dq_quant_wait_limit_ns, &ns, sizeof(ns)) == cudaSuccess ? DQ_OK
+                                                                                       : DQ_ERR_CUDA;
+}
+
 int quantize_act(const void* X, int xt, int64_t M, int64_t K, const float* c, int f, int G,
                  uint8_t* codes, void* scales, float* s_tok, cudaStream_t st) {
   uint8_t* sc = reinterpret_cast<uint8_t*>(scales);
@@ -865,16 +980,11 @@ template <int F, int G, typename WT>
 static int launch_pack(const void* W, int64_t m, int64_t n, const float* r, const float* c,
                        const float* sT, uint8_t* codes, uint8_t* scales, cudaStream_t st) {
   const int64_t nb = n / G;
-  if (F != INT4 && F != INT8) {
-    // padding rows / scale columns of the tensor-core layout are zeroed first
-    int64_t bytes = (int64_t)(((m + 127) / 128) * ((nb + 3) / 4) * 512);
-    if ((m & 127) || (nb & 3)) {
-      zero_bytes_kernel<<<(unsigned)((bytes / 16 + 255) / 256 + 1), 256, 0, st>>>(scales, bytes);
-    }
-  }
-  int64_t total = m * nb;
-  if (!ensure_kernel_attrs((const void*)pack_weight_kernel<F, G, WT>, 0, false)) return DQ_ERR_CUDA;
-  pack_weight_kernel<F, G, WT><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+  const int64_t row_tiles = (m + 127) / 128, col_tiles = (nb + 31) / 32;
+  if (row_tiles > 0x7FFFFFFF || col_tiles > 65535) return DQ_ERR_UNSUPPORTED;
+  auto kern = pack_weight_kernel<F, G, WT>;
+  if (!ensure_kernel_attrs((const void*)kern, 0, false)) return DQ_ERR_CUDA;
+  kern<<<dim3((unsigned)row_tiles, (unsigned)col_tiles), 256, 0, st>>>(
       reinterpret_cast<const WT*>(W), m, n, r, c, sT, codes, scales);
   return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
 }

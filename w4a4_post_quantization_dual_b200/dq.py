@@ -51,6 +51,7 @@ SIGNATURES = {
     "dq_act_quant_error": (_int, [_vp, _int, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp, _vp,
                                   _vp]),
     "dq_device_error": (_int, [_int]),
+    "dq_set_wait_limit": (_int, [ctypes.c_uint64]),
     "dq_version": (_int, []),
 }
 
@@ -227,6 +228,11 @@ def dq_w4a4_linear_fused(X, c, B, sB, s_w, Y, fmt, r_row=None, stream=None):
 
 def dq_device_error(clear=True):
     return lib().dq_device_error(1 if clear else 0)
+
+
+def dq_set_wait_limit(ns=0):
+    """Limit of the device-side bounded waits in ns (0: the 2 s default)."""
+    _check(lib().dq_set_wait_limit(int(ns)), "dq_set_wait_limit")
 
 
 # ----------------------------------------------------------------------------
