@@ -60,8 +60,9 @@ typedef enum {
   DQ_MXFP4 = 2,  /* E2M1, E8M0 block scale, G = 32 (OCP MX)                */
   DQ_NVFP4 = 3   /* E2M1, UE4M3 block scale, G = 16, plus an fp32 per-tensor
                     (weights) or per-token (activations) scale             */,
-  /* 8-bit variants (Appendix G.2, Table 9); dq_solve_scales* only so far,
-     the other entry points return DQ_ERR_UNSUPPORTED for them            */
+  /* 8-bit variants (Appendix G.2, Table 9): the solver, packer, activation
+     quantiser and error measure take all three; dq_w4a4_linear takes
+     MXFP8 and MXINT8 and returns DQ_ERR_UNSUPPORTED for INT8             */
   DQ_INT8 = 4,   /* integers -128..127, bf16 block scale, G in {32, 64, 128} */
   DQ_MXINT8 = 5, /* integers -128..127, E8M0 block scale, G = 32           */
   DQ_MXFP8 = 6   /* FP8 E4M3, E8M0 block scale, G = 32 (OCP MX)            */

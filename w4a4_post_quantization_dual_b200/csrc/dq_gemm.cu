@@ -1860,6 +1860,8 @@ static int launch_splitk(const uint8_t* A, const uint8_t* sA, const float* s_tok
                          const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                          int64_t M, int64_t N, int64_t K, int S, cudaStream_t st) {
   using C = Cfg<FMT, SK_BN, SK_PART_BYTES>;
+  // each CTA owns a column slice of SK_BN / S columns, moved as float4
+  if (S < 1 || S > 8 || SK_BN % (4 * S)) return DQ_ERR_UNSUPPORTED;
   const int a_rows = M < BM ? (int)((M + 15) / 16 * 16) : BM;
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, M, K / 2, a_rows) || !make_map(&tb, B, N, K / 2, SK_BN)) return DQ_ERR_CUDA;
@@ -1881,6 +1883,7 @@ static int launch_splitk_fused(const __nv_bfloat16* X, const float* c, const uin
                                const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                                int64_t M, int64_t N, int64_t K, int S, cudaStream_t st) {
   using C = Cfg<NVFP4, SK_BN, SK_PART_BYTES>;
+  if (S < 1 || S > 8 || SK_BN % (4 * S)) return DQ_ERR_UNSUPPORTED;
   const int a_rows = M < BM ? (int)((M + 15) / 16 * 16) : BM;
   const int kt_per_slice = (int)(K / BK) / S;
   if (kt_per_slice > C::STAGES) return DQ_ERR_UNSUPPORTED;
@@ -1998,16 +2001,22 @@ static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, con
                     const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int64_t M,
                     int64_t N, int64_t K, cudaStream_t st) {
   const int64_t tm = (M + BM - 1) / BM, sms = num_sms();
-  if (N % 256 == 0 && pair_mode() == 2) {
+  // long K with plenty of 256 x 256 tiles: the paired-SM kernel reads 30 %
+  // fewer operand bytes per SM (measured 8192 x 5120 x 27648: 3.88 vs 3.60
+  // PFLOP/s); at K of a few thousand both tile shapes run alike
+  if (N % 256 == 0 && (pair_mode() == 2 || (pair_mode() == 1 && K >= 16384 &&
+                                             ((M + 255) / 256) * (N / 256) >= 2 * sms))) {
     const int max_pairs = pair_max_clusters<FMT, YT>();
     if (max_pairs > 0)
       return launch_pair<FMT, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, max_pairs, st);
   }
   if (N % 256 == 0 && tm * (N / 256) >= sms)
     return launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
-  if (N % 256 == 0 && pair_mode() != 0) {
+  if (N % 256 == 0 && pair_mode() != 0 && (tm > 1 || pair_mode() == 2)) {
     // too few 128 x 256 tiles to fill the SMs: paired-SM 256 x 256 tiles
-    // once they occupy at least half of the SM pairs
+    // once they occupy at least half of the SM pairs (not when one 128-row
+    // tile holds every token: the weight-streaming 128-wide tiles measured
+    // faster there, M = 1 x 27648 x 5120: 30.3 vs 34.9 us)
     const int max_pairs = pair_max_clusters<FMT, YT>();
     const int64_t tiles2 = ((M + 255) / 256) * (N / 256);
     if (max_pairs > 0 && 2 * tiles2 >= max_pairs)
@@ -2017,7 +2026,7 @@ static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, con
   const int KT = (int)(K / BK);
   // largest split whose clusters (one per output tile) all run in one wave
   int S = 1;
-  for (int cand : {8, 4, 2})
+  for (int cand : {8, 4, 2})   // the column slice 128 / S must stay a multiple of 4
     if (S == 1 && KT % cand == 0 && t128 * cand <= sms &&
         t128 <= splitk_max_clusters<FMT, YT>(cand))
       S = cand;

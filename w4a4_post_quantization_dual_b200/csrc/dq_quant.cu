@@ -447,11 +447,11 @@ __device__ __forceinline__ void act_block_scale(float ab, float st, float d6, ui
     const float sblk = __fmul_rn(ue4m3_value(byte), st);
     zero = (sblk == 0.0f);
     inv = zero ? 0.0f : __frcp_rn(sblk);
-  } else {  // OCP MX rule: 2^(floor(log2 amax) - 2), E8M0 byte e + 127
+  } else {  // OCP MX rule: 2^(floor(log2 amax) - emax), E8M0 byte e + 127
     int e = -127;
     zero = !(ab > 0.0f);
     if (!zero) {
-      e = ilog2f(ab) - 2;
+      e = ilog2f(ab) - mx_emax(F);
       e = e < -127 ? -127 : (e > 127 ? 127 : e);
     }
     byte = (uint32_t)(e + 127);
@@ -491,6 +491,50 @@ __device__ __forceinline__ void act_block_codes(const float2* xt, float inv, boo
   }
   if constexpr (P == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(wv[0], wv[1]);
   else *reinterpret_cast<uint4*>(dst) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+}
+
+// One-byte codes of one block (values xt in the rotated piece order): MXFP8
+// E4M3 (nearest even, saturating, sign kept) or MXINT8 integers (nearest
+// even, clipped to [-128, 127]); rotated back and stored (G bytes, 16-byte
+// aligned); all-zero codes when the block scale is zero.
+template <int F, int G>
+__device__ __forceinline__ void act_block_codes8(const float2* xt, float inv, bool zero, int rot,
+                                                 uint8_t* dst) {
+  constexpr int P = G / 8;
+  static_assert(P == 4, "one-byte codes: 32-element blocks");
+  const float2 inv2 = make_float2(inv, inv);
+  uint2 wv[P];   // 8 codes per piece
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float2 z0 = __fmul2_rn(xt[4 * p + 2 * h], inv2), z1 = __fmul2_rn(xt[4 * p + 2 * h + 1], inv2);
+      if constexpr (F == MXFP8) {
+        uint16_t lo, hi;   // element 2k in the low byte of each pair
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(lo) : "f"(z0.x), "f"(z0.y));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(hi) : "f"(z1.x), "f"(z1.y));
+        w[h] = (uint32_t)lo | ((uint32_t)hi << 16);
+      } else {
+        const float v[4] = {z0.x, z0.y, z1.x, z1.y};
+        uint32_t b = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          b |= ((uint32_t)(int)rintf(fminf(fmaxf(v[k], -128.0f), 127.0f)) & 0xFFu) << (8 * k);
+        w[h] = b;
+      }
+    }
+    wv[p] = zero ? make_uint2(0u, 0u) : make_uint2(w[0], w[1]);
+  }
+  // undo the piece rotation: output piece q comes from wv[(q - rot) mod P]
+  uint2 o[P];
+#pragma unroll
+  for (int q = 0; q < P; ++q) {
+    const uint2 a0 = wv[q], a1 = wv[(q + 3) & 3], a2 = wv[(q + 2) & 3], a3 = wv[(q + 1) & 3];
+    o[q] = rot == 0 ? a0 : (rot == 1 ? a1 : (rot == 2 ? a2 : a3));
+  }
+  reinterpret_cast<uint4*>(dst)[0] = make_uint4(o[0].x, o[0].y, o[1].x, o[1].y);
+  reinterpret_cast<uint4*>(dst)[1] = make_uint4(o[2].x, o[2].y, o[3].x, o[3].y);
 }
 
 // x~ = x*c for one block read from shared memory, and its absolute maximum.
@@ -579,7 +623,7 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
     const int s = tl + j * NTS;
     own[j] = s < S;
     boff[j] = (uint32_t)rt * row_bytes + (uint32_t)s * (G * 2);
-    coff[j] = (uint32_t)s * (G / 2);
+    coff[j] = (uint32_t)s * (is_8bit(F) ? G : G / 2);
     sfo[j] = ((uint32_t)(s >> 2) << 9) | (uint32_t)(s & 3);
   }
   if (tid < 48) rowmax[tid] = 0u;
@@ -652,7 +696,7 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
     const bool rowv = t < M, rowp = t < Mpad;  // both uniform over a warp
     if (!aq::wait_parity(&full[stg], phase)) *abort_flag = 1;
     const unsigned char* sp = stages + (size_t)stg * stage_bytes;
-    uint8_t* crow = codes + t * (K / 2);
+    uint8_t* crow = codes + t * (is_8bit(F) ? K : K / 2);
     uint8_t* sfrow = scales + ((((t >> 7) * S4) << 9) + ((t & 31) << 4) + (((t & 127) >> 5) << 2));
 
     if constexpr (F == NVFP4) {
@@ -711,7 +755,8 @@ quantize_act_ring_kernel(const __nv_bfloat16* __restrict__ X, int64_t M, int64_t
             float inv;
             bool zero;
             act_block_scale<F>(ab, 0.0f, 0.0f, byte, inv, zero);
-            act_block_codes<F, G>(xt, inv, zero, rot, crow + coff[j]);
+            if constexpr (is_8bit(F)) act_block_codes8<F, G>(xt, inv, zero, rot, crow + coff[j]);
+            else act_block_codes<F, G>(xt, inv, zero, rot, crow + coff[j]);
           }
           if (own[j]) sfrow[sfo[j]] = (uint8_t)byte;
         }
@@ -829,7 +874,7 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
   const int bpt = (int)((S + NT - 1) / NT);
   const int64_t Mpad = (F == INT4 || F == INT8) ? M : ((M + 127) / 128) * 128;
   const XT* Xp = reinterpret_cast<const XT*>(X);
-  if constexpr (F != INT4 && !is_8bit(F)) {
+  if constexpr (F == NVFP4 || is_mx(F)) {
     if constexpr (sizeof(XT) == 2) {
       // ring kernel: NTS threads per row, BPT blocks per thread, at most MAXT
       // threads and MINB CTAs per SM (the register budget of each variant)
@@ -883,6 +928,8 @@ static int launch_act(const void* X, int64_t M, int64_t K, const float* c, uint8
       }
       if (rc >= 0) return rc;
     }
+  }
+  if constexpr (F == NVFP4 || (is_mx(F) && !is_8bit(F))) {
     // rows kernel (fp32 input, or rows too long for the register-resident ring):
     // R rows per CTA iteration, BPT blocks per thread
     constexpr int R = (G == 16) ? 4 : 2;

@@ -526,19 +526,24 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
 
     for (int s = 0; s < steps; ++s) {
       const int lr = s * S::RPS + rslot;
-      float2 x[4], y[4];
+      float2 x[4], q[4];
       load_x(lr, x);
       const float2 ra = ra_s[lr];
       float rn = ra.x, an = ra.y;
+      {
+        // codes at the current scales: the row half-step's, and the column
+        // half-step's too wherever the row scale does not move
+        const float2 a2 = make_float2(ra.y, ra.y);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) y[k] = __fmul2_rn(x[k], beta[k]);
+        for (int k = 0; k < 4; ++k) q[k] = grid2_packed<F>(__fmul2_rn(__fmul2_rn(x[k], beta[k]), a2));
+      }
       if (do_row || TRACE) {
         // ---- row half-step at the current scales (and the error there) ----
         const float2 a2 = make_float2(ra.y, ra.y);
         float2 num2 = make_float2(0.f, 0.f), den2 = num2, err2 = num2;
         float2 R[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) R[k] = __fmul2_rn(grid2_packed<F>(__fmul2_rn(y[k], a2)), cc[k]);
+        for (int k = 0; k < 4; ++k) R[k] = __fmul2_rn(q[k], cc[k]);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           num2 = __ffma2_rn(x[k], R[k], num2);
@@ -555,9 +560,8 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
             const float2 ap2 = make_float2(ap, ap);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const float2 q = grid2_packed<F>(__fmul2_rn(y[k], a2));
               const float2 qp = grid2_packed<F>(__fmul2_rn(__fmul2_rn(x[k], beta_prev[k]), ap2));
-              const float2 d = make_float2(q.x - qp.x, q.y - qp.y);
+              const float2 d = make_float2(q[k].x - qp.x, q[k].y - qp.y);
               qn2 = __ffma2_rn(d, d, qn2);
               qd2 = __ffma2_rn(qp, qp, qd2);
             }
@@ -589,7 +593,7 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
             double dn = 0.0, dd = 0.0;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const float2 Rk = __fmul2_rn(grid2_packed<F>(__fmul2_rn(y[k], a2)), cc[k]);
+              const float2 Rk = __fmul2_rn(q[k], cc[k]);
               dn = fma((double)x[k].x, (double)Rk.x, dn);
               dn = fma((double)x[k].y, (double)Rk.y, dn);
               dd = fma((double)Rk.x, (double)Rk.x, dd);
@@ -610,10 +614,17 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
       }
       if (do_col) {
         // ---- column partials with the new row scale ----
-        const float2 a2 = make_float2(an, an), r2 = make_float2(rn, rn);
+        // a row-block whose scale did not move keeps its codes (the same
+        // fp32 products as above); the warp re-quantises only if one moved
+        if (!__all_sync(FULL, an == ra.y)) {
+          const float2 a2 = make_float2(an, an);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) q[k] = grid2_packed<F>(__fmul2_rn(__fmul2_rn(x[k], beta[k]), a2));
+        }
+        const float2 r2 = make_float2(rn, rn);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float2 Sv = __fmul2_rn(r2, grid2_packed<F>(__fmul2_rn(y[k], a2)));
+          const float2 Sv = __fmul2_rn(r2, q[k]);
           accn[k] = __ffma2_rn(Sv, x[k], accn[k]);
           accd[k] = __ffma2_rn(Sv, Sv, accd[k]);
         }
@@ -697,16 +708,17 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
       if (tid < G) {
         sn = 0.0;
         sd = 0.0;
-        for (int q0 = 0; q0 < (int)C; q0 += 4) {
-          double pn[4], pd[4];
+        // eight CTAs' totals in flight at a time: one round trip for C <= 8
+        for (int q0 = 0; q0 < (int)C; q0 += 8) {
+          double pn[8], pd[8];
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
+          for (int u = 0; u < 8; ++u)
             if (q0 + u < (int)C) {
               pn[u] = ld_dsmem_f64(&sm.cpart[xb][2 * tid], (uint32_t)(q0 + u));
               pd[u] = ld_dsmem_f64(&sm.cpart[xb][2 * tid + 1], (uint32_t)(q0 + u));
             }
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
+          for (int u = 0; u < 8; ++u)
             if (q0 + u < (int)C) {
               sn += pn[u];
               sd += pd[u];

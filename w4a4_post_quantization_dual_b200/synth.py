@@ -111,11 +111,15 @@ def weight(workload: str, index: int, shape=None):
 def acts(workload: str, M: int, K: int, index: int = 0, outlier_channels=None):
     """Activations for a workload.  The tiny workload places its outlier
     channels on the first outlier columns of its weight (the paper's premise
-    that weight and activation outliers share channels, Section 4.2)."""
+    that weight and activation outliers share channels, Section 4.2); the
+    other workloads draw theirs with the activation seed."""
     w = WORKLOADS[workload]
     n_out = w.get("x_outliers")
     if n_out is None:
         n_out = int(round(w.get("x_outlier_frac", 0.0) * K))
+    if (outlier_channels is None and w.get("w_outlier_cols", 0) >= (n_out or 0) > 0
+            and K == w["weights"][index][1]):
+        outlier_channels = weight(workload, index)[1][:n_out]
     return activations(M, K, 1000 + w["seed"] + index, outlier_channels=outlier_channels,
                        n_outliers=n_out, outlier_scale=w.get("x_outlier_scale", 1.0),
                        bf16=w["bf16"])
