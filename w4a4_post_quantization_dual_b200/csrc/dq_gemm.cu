@@ -239,19 +239,27 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* v) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-template <int FMT, int BN, int RESERVE = 0>
+// AR: rows of A staged per k-tile.  The MMA always computes 128 rows; with
+// AR < 128 (every token fits in AR rows) it reads the rows past AR from the
+// shared memory that follows the stage, which only feeds accumulator rows
+// that are never stored, and each stage is smaller, so more of the weight
+// stream is in flight.
+template <int FMT, int BN, int RESERVE = 0, int AR = BM>
 struct Cfg {
   static constexpr int G = (FMT == NVFP4) ? 16 : 32;
   static constexpr int SF_PER_ROW = BK / G;                   // scales per row per k-tile
   static constexpr int SF_ATOMS = SF_PER_ROW / 4;             // 512-byte atoms per 128 rows
-  static constexpr int A_BYTES = BM * BKB;                    // 16 KB
+  static constexpr int A_BYTES = AR * BKB;                    // 16 KB for 128 rows
   static constexpr int B_BYTES = BN * BKB;
   static constexpr int SFA_BYTES = SF_ATOMS * 512;
   static constexpr int SFB_BYTES = (BN / 128) * SF_ATOMS * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = (227 * 1024 - 1024 - 256 - RESERVE) / STAGE_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + RESERVE;
-  static_assert(4 * STAGES * 8 + 40 <= 256, "barrier area");
+  static constexpr int STAGES = (227 * 1024 - 1024 - 512 - RESERVE) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/ + RESERVE;
+  static_assert(AR % 32 == 0 && AR <= BM, "staged A rows");
+  static_assert(4 * STAGES * 8 + 40 <= 512, "barrier area");
+  // the MMA's 128-row read of the last A stage stays inside the B stages
+  static_assert((BM - AR) * BKB <= STAGES * B_BYTES, "A read window");
   // tensor-memory columns: accumulator, then one scale slot per stage
   // (SFA: 4 columns per atom; SFB: 4 columns per atom and 128-row group)
   static constexpr int SF_COLS = 4 * SF_ATOMS * (1 + BN / 128);
@@ -299,13 +307,13 @@ __device__ __forceinline__ void epilogue_bf16(uint32_t tmem, int quad, int lane,
   }
 }
 
-template <int FMT, int BN, int YT>
+template <int FMT, int BN, int YT, int AR = BM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const uint8_t* __restrict__ sfA, const uint8_t* __restrict__ sfB,
                  const float* __restrict__ s_tok, const float* __restrict__ s_w,
                  const float* __restrict__ r_row, void* __restrict__ Y, int M, int N, int K) {
-  using C = Cfg<FMT, BN>;
+  using C = Cfg<FMT, BN, 0, AR>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -622,7 +630,7 @@ constexpr int SK_PART_BYTES = BM * SK_BN * 4;
 // scale atoms (UE4M3) of every k-tile of the slice straight into the stage
 // buffers, with the arithmetic of the standalone activation quantiser; TMA
 // brings only the weights.  Requires kt_per_slice <= STAGES.
-template <int FMT, int YT, bool FUSED>
+template <int FMT, int YT, bool FUSED, int AR = BM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const uint8_t* __restrict__ sfA,
@@ -632,7 +640,7 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
                         int a_rows, const __nv_bfloat16* __restrict__ X,
                         const float* __restrict__ cvec) {
   constexpr int BN = SK_BN;
-  using C = Cfg<FMT, BN, SK_PART_BYTES>;
+  using C = Cfg<FMT, BN, SK_PART_BYTES, AR>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -735,7 +743,7 @@ w4a4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA,
     if (lane == 0 && !FUSED) {
       // A tiles carry only the a_rows rows that exist (rounded up to 16): the
       // MMA's other rows feed accumulator rows that are never stored
-      const uint32_t tx = C::STAGE_BYTES - (BM - a_rows) * BKB;
+      const uint32_t tx = C::STAGE_BYTES - (AR - a_rows) * BKB;
       auto load_b = [&](int stage, int kt) {
         tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], (kt0 + kt) * BKB, n0);
         bulk_load(sSFB + stage * C::SFB_BYTES,
@@ -1382,11 +1390,12 @@ w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 // 32 elements (one scale byte per MMA, K = 32) accumulates in tensor memory.
 // Tiles 128 x 128, BK = 128 elements per stage, persistent.
 //   warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, warp 6 scale copies,
-//   warps 7..10 converters.
+//   warps 7..14 converters.
 // ---------------------------------------------------------------------------
 namespace i4 {
 constexpr int BN = 128, BKE = 128;                   // elements per k-tile
-constexpr int THREADS = 352;
+constexpr int CONVERTERS = 8;                  // converter warps (7 .. 14)
+constexpr int THREADS = (7 + CONVERTERS) * 32;
 constexpr int STG_A = BM * BKE / 2, STG_B = BN * BKE / 2;      // packed staging (8 KB each)
 constexpr int OP_A = BM * BKE, OP_B = BN * BKE;                // E4M3 operands (16 KB each)
 constexpr int SF_A = 512, SF_B = 512;                          // one 128 x 4 atom each
@@ -1501,7 +1510,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sfready[s], 1);
-      mbar_init(&conv[s], 4);
+      mbar_init(&conv[s], CONVERTERS);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
@@ -1640,7 +1649,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
   } else if (warp >= 7) {
     if constexpr (I8) {
     // converters: int8 staging x block power of two -> swizzled bf16 operand tiles
-    const int ct = threadIdx.x - 7 * 32;        // 0..127
+    const int ct = threadIdx.x - 7 * 32;        // 0 .. 32 * CONVERTERS - 1
     const int64_t S = K / 32;
     int stage = 0;
     uint32_t phase = 0;
@@ -1654,7 +1663,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
         if (!got) { ok = false; break; }
         // 16-byte int8 chunks: A rows 0..127 (4 chunks each), then B rows
 #pragma unroll 2
-        for (int c = ct; c < (BM + BN) * 4; c += 128) {
+        for (int c = ct; c < (BM + BN) * 4; c += 32 * CONVERTERS) {
           const bool isB = c >= BM * 4;
           const int cc = isB ? c - BM * 4 : c;
           const int r = cc >> 2, kc = cc & 3;
@@ -1679,7 +1688,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     } else if constexpr (!FP8) {
     // converters: packed INT4 staging -> swizzled E4M3 operand tiles
-    const int ct = threadIdx.x - 7 * 32;        // 0..127
+    const int ct = threadIdx.x - 7 * 32;        // 0 .. 32 * CONVERTERS - 1
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -1691,7 +1700,7 @@ w4a4_gemm_mxint4_kernel(const __grid_constant__ CUtensorMap tmA,
         if (!got) { ok = false; break; }
         // 16-byte packed chunks: A rows 0..127 (4 chunks each), then B rows
 #pragma unroll 2
-        for (int c = ct; c < (BM + BN) * 4; c += 128) {
+        for (int c = ct; c < (BM + BN) * 4; c += 32 * CONVERTERS) {
           const bool isB = c >= BM * 4;
           const int cc = isB ? c - BM * 4 : c;
           const int r = cc >> 2, kc = cc & 3;
@@ -1839,14 +1848,15 @@ static int num_sms() {
   return n;
 }
 
-template <int FMT, int BN, int YT>
+template <int FMT, int BN, int YT, int AR = BM>
 static int launch(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                   const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int64_t M,
                   int64_t N, int64_t K, cudaStream_t st) {
-  using C = Cfg<FMT, BN>;
+  using C = Cfg<FMT, BN, 0, AR>;
+  if (AR < BM && M > AR) return DQ_ERR_UNSUPPORTED;
   CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K / 2, BM) || !make_map(&tb, B, N, K / 2, BN)) return DQ_ERR_CUDA;
-  auto kern = w4a4_gemm_kernel<FMT, BN, YT>;
+  if (!make_map(&ta, A, M, K / 2, AR) || !make_map(&tb, B, N, K / 2, BN)) return DQ_ERR_CUDA;
+  auto kern = w4a4_gemm_kernel<FMT, BN, YT, AR>;
   if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
   const int64_t tiles = ((M + BM - 1) / BM) * (N / BN);
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
@@ -1855,17 +1865,18 @@ static int launch(const uint8_t* A, const uint8_t* sA, const float* s_tok, const
   return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
 }
 
-template <int FMT, int YT>
+template <int FMT, int YT, int AR = BM>
 static int launch_splitk(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                          const uint8_t* sB, const float* s_w, const float* r_row, void* Y,
                          int64_t M, int64_t N, int64_t K, int S, cudaStream_t st) {
-  using C = Cfg<FMT, SK_BN, SK_PART_BYTES>;
+  using C = Cfg<FMT, SK_BN, SK_PART_BYTES, AR>;
   // each CTA owns a column slice of SK_BN / S columns, moved as float4
   if (S < 1 || S > 8 || SK_BN % (4 * S)) return DQ_ERR_UNSUPPORTED;
   const int a_rows = M < BM ? (int)((M + 15) / 16 * 16) : BM;
+  if (a_rows > AR) return DQ_ERR_UNSUPPORTED;
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, M, K / 2, a_rows) || !make_map(&tb, B, N, K / 2, SK_BN)) return DQ_ERR_CUDA;
-  auto kern = w4a4_gemm_splitk_kernel<FMT, YT, false>;
+  auto kern = w4a4_gemm_splitk_kernel<FMT, YT, false, AR>;
   if (!ensure_kernel_attrs((const void*)kern, C::SMEM_BYTES, false)) return DQ_ERR_CUDA;
   const int kt_per_slice = (int)(K / BK) / S;
   if (launch_ex(kern, dim3(S, (unsigned)(N / SK_BN), (unsigned)((M + BM - 1) / BM)),
@@ -2030,10 +2041,15 @@ static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, con
     if (S == 1 && KT % cand == 0 && t128 * cand <= sms &&
         t128 <= splitk_max_clusters<FMT, YT>(cand))
       S = cand;
-  if (S > 1) return launch_splitk<FMT, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, S, st);
+  const bool few = M <= 32;   // every token in 32 staged rows
+  if (S > 1)
+    return few ? launch_splitk<FMT, YT, 32>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, S, st)
+               : launch_splitk<FMT, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, S, st);
   if (N % 256 == 0 && tm * (N / 256) * 2 > t128)  // few tiles either way: keep the wide tile
-    return launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
-  return launch<FMT, 128, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
+    return few ? launch<FMT, 256, YT, 32>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
+               : launch<FMT, 256, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
+  return few ? launch<FMT, 128, YT, 32>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st)
+             : launch<FMT, 128, YT>(A, sA, s_tok, B, sB, s_w, r_row, Y, M, N, K, st);
 }
 
 // MODE 1: MXFP8 codes (one byte per element, 128-byte swizzled TMA boxes);

@@ -110,6 +110,14 @@ __device__ __forceinline__ double ld_dsmem_f64(const double* local, uint32_t ran
   asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(ra));
   return v;
 }
+// Two doubles into CTA `rank`'s shared memory (made visible to it by the
+// release / acquire of the next cluster barrier).
+__device__ __forceinline__ void st_dsmem_f64x2(const double* local, uint32_t rank, double a,
+                                               double b) {
+  uint32_t la = (uint32_t)__cvta_generic_to_shared(local), ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(la), "r"(rank));
+  asm volatile("st.shared::cluster.v2.f64 [%0], {%1, %2};" ::"r"(ra), "d"(a), "d"(b) : "memory");
+}
 
 // Reduce V fp64 partials per thread over the CTA's threads that share an
 // octet (initialisation: column l1 norms); scr (the float scratch of
@@ -391,13 +399,17 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BcdSmem<G>& sm = *reinterpret_cast<BcdSmem<G>*>(smem_raw);
   const int rows_cta = steps * S::RPS;
-  float2* ra_s = reinterpret_cast<float2*>(smem_raw + ((sizeof(BcdSmem<G>) + 15) & ~(size_t)15));
+  const uint32_t C = gridDim.x;
+  // cluster receive buffers [2][C][2G] of column totals (C > 1), then
+  // (r, alpha) per row, the trace's previous alphas and the staged rows
+  double* recv = reinterpret_cast<double*>(smem_raw + ((sizeof(BcdSmem<G>) + 15) & ~(size_t)15));
+  float2* ra_s = reinterpret_cast<float2*>(recv + (C > 1 ? 4 * (size_t)C * G : 0));
   float* ap_s = reinterpret_cast<float*>(ra_s + rows_cta);        // TRACE only
   WT* wch = reinterpret_cast<WT*>(ap_s + (TRACE ? rows_cta : 0));  // staged rows
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int oct = lane % S::OPB, rr = lane / S::OPB, rslot = warp * S::RPW + rr;
-  const uint32_t rank = cluster_ctarank(), C = gridDim.x;
+  const uint32_t rank = cluster_ctarank();
   const int64_t b = blockIdx.y, nb = n / G;
   const int64_t col0 = b * G + oct * 8;
   const int64_t row0 = (int64_t)rank * rows_cta;
@@ -506,7 +518,8 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
   }
   __syncwarp();
 
-  int xb = 0;  // exchange buffer of the next cluster exchange
+  int xb = 0;   // buffer of the next exact-pass exchange
+  int xr = 0;   // index of the next column-total exchange (receive buffer xr & 1)
   // column window: the per-thread fp32 chain (steps terms) and the fp32
   // reduce-scatter levels, 2 * depth + 4 ulps, + 4 for S = r q in fp32
   const uint32_t col_win = 2u * (uint32_t)(steps + S::LV) + 8u;
@@ -700,32 +713,21 @@ solve_bcd_kernel(SolveBatch bt, int64_t m, int steps, int T, SolveOpts o) {
       // order (identical c in every CTA).  The buffer alternates with every
       // exchange: a CTA writes buffer xb only after all peers passed the
       // barrier that follows their last reads of it.
-      if (tid < G) {
-        sm.cpart[xb][2 * tid] = sn;
-        sm.cpart[xb][2 * tid + 1] = sd;
-      }
+      // pushed into slot `rank` of every CTA's receive buffer before the
+      // barrier, read locally after it
+      double* rb = recv + (size_t)(xr & 1) * C * 2 * G;
+      if (tid < G)
+        for (uint32_t q = 0; q < C; ++q) st_dsmem_f64x2(rb + rank * 2 * G + 2 * tid, q, sn, sd);
       cluster_sync_all();
       if (tid < G) {
         sn = 0.0;
         sd = 0.0;
-        // eight CTAs' totals in flight at a time: one round trip for C <= 8
-        for (int q0 = 0; q0 < (int)C; q0 += 8) {
-          double pn[8], pd[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (q0 + u < (int)C) {
-              pn[u] = ld_dsmem_f64(&sm.cpart[xb][2 * tid], (uint32_t)(q0 + u));
-              pd[u] = ld_dsmem_f64(&sm.cpart[xb][2 * tid + 1], (uint32_t)(q0 + u));
-            }
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (q0 + u < (int)C) {
-              sn += pn[u];
-              sd += pd[u];
-            }
+        for (uint32_t q = 0; q < C; ++q) {
+          sn += rb[q * 2 * G + 2 * tid];
+          sd += rb[q * 2 * G + 2 * tid + 1];
         }
       }
-      xb ^= 1;
+      ++xr;
     }
     // projected update; a column near a projection boundary is redone below
     // from exact sums
@@ -836,10 +838,10 @@ constexpr size_t SOLVER_SMEM_MAX = 227 * 1024;
 // row, the previous alpha per row (trace), and the staged rows
 // (elem_bytes = 0: streamed).
 template <int G>
-static size_t solver_smem_bytes(int steps, size_t elem_bytes, bool trace) {
+static size_t solver_smem_bytes(int steps, size_t elem_bytes, bool trace, int C) {
   const size_t rows = (size_t)steps * SolverShape<G>::RPS;
-  return ((sizeof(BcdSmem<G>) + 15) & ~(size_t)15) + rows * 8 + (trace ? rows * 4 : 0) +
-         rows * G * elem_bytes;
+  return ((sizeof(BcdSmem<G>) + 15) & ~(size_t)15) + (C > 1 ? 32 * (size_t)C * G : 0) +
+         rows * 8 + (trace ? rows * 4 : 0) + rows * G * elem_bytes;
 }
 
 // Launch geometry: the tile's rows are split over C CTAs of one cluster,
@@ -855,9 +857,10 @@ static void solver_geometry(int64_t m, int& steps, int& C, int& stg) {
   for (int c = 1; c <= 16; ++c) {
     const int64_t rows = (m + c - 1) / c;
     const int st = (int)((rows + S::RPS - 1) / S::RPS);
-    if (solver_smem_bytes<G>(st, sizeof(WT), true) <= SOLVER_SMEM_MAX) {
+    const int cc = (int)((m + (int64_t)S::RPS * st - 1) / ((int64_t)S::RPS * st));
+    if (solver_smem_bytes<G>(st, sizeof(WT), true, cc) <= SOLVER_SMEM_MAX) {
       steps = st;
-      C = (int)((m + (int64_t)S::RPS * st - 1) / ((int64_t)S::RPS * st));
+      C = cc;
       stg = 1;
       return;
     }
@@ -887,7 +890,7 @@ static int launch_solver(const SolveBatch& bt, int count, int64_t m, int T, cons
     any_trace = any_trace || (traces && traces[i]);
   }
   const size_t sm_init = sizeof(SolverSmem<G>),
-               sm_main = solver_smem_bytes<G>(steps, stg ? sizeof(WT) : 0, any_trace);
+               sm_main = solver_smem_bytes<G>(steps, stg ? sizeof(WT) : 0, any_trace, C);
   if (sm_main > SOLVER_SMEM_MAX) return DQ_ERR_UNSUPPORTED;
   if (tiles > 65535) return DQ_ERR_UNSUPPORTED;
 
@@ -938,7 +941,7 @@ template <int G, typename WT>
 static int solver_supported(int64_t m, int64_t n) {
   int steps, C, stg;
   solver_geometry<G, WT>(m, steps, C, stg);
-  const size_t sm_main = solver_smem_bytes<G>(steps, stg ? sizeof(WT) : 0, true);
+  const size_t sm_main = solver_smem_bytes<G>(steps, stg ? sizeof(WT) : 0, true, C);
   return (sm_main > SOLVER_SMEM_MAX || n / G > 65535) ? DQ_ERR_UNSUPPORTED : DQ_OK;
 }
 
