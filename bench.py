@@ -348,7 +348,7 @@ def blas_threads():
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    wl, Ws, Xs = workload_inputs(WORKLOAD)
+    wl, Ws, Xs = workload_inputs(args.workload)
     M = max(wl["M"])
     oracle_prepare(Ws)
     for _ in range(args.warmup):
@@ -365,7 +365,7 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / max(args.steps, 1) * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "format": FMT_NAME, "M": M, "sample_rows": 16,
+        "config": {"workload": args.workload, "format": FMT_NAME, "M": M, "sample_rows": 16,
                    "sample_cols": SAMPLE_COLS},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": desc},
@@ -416,7 +416,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     dq.lib()
-    wl, Ws, Xs = workload_inputs(WORKLOAD)
+    wl, Ws, Xs = workload_inputs(args.workload)
     fmt, T = dq.DQ_NVFP4, wl["T"]
     G = dq.native_group(fmt)
     st = torch.cuda.current_stream()
@@ -533,6 +533,8 @@ def run_ours(args, rank, world, local_rank):
             del Bc
             b_ = decode_bytes(M, N, K, G)
             decode[f"M{M}_N{N}_K{K}"] = {
+                "kernel": ("w4a4_gemv_kernel (CUDA cores)" if M == 1 and K % 1024 == 0 and
+                           fmt in (dq.DQ_NVFP4, dq.DQ_MXFP4) else "tcgen05 GEMM"),
                 "gemm_us": t_gemm, "act_plus_gemm_us": t_pair, "fused_us": t_fused,
                 "algorithmic_bytes": b_, "gemm_gbs": b_ / (t_gemm * 1e-6) / 1e9,
                 "gemm_frac_hbm": b_ / (t_gemm * 1e-6) / 1e9 / hbm,
@@ -674,7 +676,7 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4(e2m1)",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "format": FMT_NAME,
+        "config": {"workload": args.workload, "format": FMT_NAME,
                    "weights": [list(L.W.shape) for L in Ls], "M_prefill": Mp, "M_decode": Mds,
                    "T": T, "l2": "flushed before every step (256 MiB write, outside the timed "
                                  "events); the linears run first in the step",
@@ -739,6 +741,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "llama8b_attn_nvfp4"],
+                    help="the NVFP4 layer the step runs (prefill + decode linears, solve + pack)")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the other workloads and the MXFP8 line")
     args = ap.parse_args()

@@ -245,7 +245,10 @@ DQ_API int dq_quantize_act(const void* X, dq_dtype xt, int64_t M, int64_t K, con
  * DQ_INT4 returns DQ_ERR_UNSUPPORTED (bf16 group scales have no
  * block-scaled tensor-core form on sm_100a).
  * Sizes: M >= 1, N % 128 == 0, K % 256 == 0; A, B, sA, sB 16-byte aligned.
- * FP32 accumulation in tensor memory.
+ * FP32 accumulation in tensor memory.  With M == 1 (NVFP4, MXFP4, K a
+ * multiple of 1024) the call runs on the CUDA cores instead: a weight
+ * stream with exact integer block dot products and fp32 accumulation,
+ * summed in a fixed order (the same bits on every call).
  * Ordering: stream-ordered.  The inference kernels use programmatic
  * dependent launch and read the weight operand (B, sB) before waiting for
  * the kernel launched just before them in the stream; B and sB must

@@ -2005,12 +2005,17 @@ static int splitk_max_clusters(int S) {
   return n > 0 ? n : 0;
 }
 
-// Tile-shape policy: 128 x 256 persistent tiles when they fill the machine,
-// else 128 x 128 persistent tiles, else split-K over a cluster of S CTAs.
+// Tile-shape policy: up to four tokens on the CUDA cores (dq_gemv.cu); 128 x
+// 256 persistent tiles when they fill the machine, else 128 x 128 persistent
+// tiles, else split-K over a cluster of S CTAs.
 template <int FMT, int YT>
 static int dispatch(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                     const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int64_t M,
                     int64_t N, int64_t K, cudaStream_t st) {
+  if (M <= GEMV_MAX_TOKENS) {   // a weight stream: the CUDA-core kernel of dq_gemv.cu
+    const int rc = w4a4_gemv(A, sA, s_tok, B, sB, s_w, r_row, Y, YT, M, N, K, FMT, st);
+    if (rc != DQ_ERR_UNSUPPORTED) return rc;
+  }
   const int64_t tm = (M + BM - 1) / BM, sms = num_sms();
   // long K with plenty of 256 x 256 tiles: the paired-SM kernel reads 30 %
   // fewer operand bytes per SM (measured 8192 x 5120 x 27648: 3.88 vs 3.60

@@ -32,6 +32,13 @@ int quantize_weight(const void* W, int wt, int64_t m, int64_t n, int f, int G, c
 int w4a4_linear(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
                 const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int yt,
                 int64_t M, int64_t N, int64_t K, int f, cudaStream_t st);
+// The linear for at most GEMV_MAX_TOKENS tokens on the CUDA cores (NVFP4,
+// MXFP4, K % 1024 == 0); DQ_ERR_UNSUPPORTED when it does not apply, and the
+// caller takes the tensor-core kernels.
+constexpr int GEMV_MAX_TOKENS = 1;
+int w4a4_gemv(const uint8_t* A, const uint8_t* sA, const float* s_tok, const uint8_t* B,
+              const uint8_t* sB, const float* s_w, const float* r_row, void* Y, int yt, int64_t M,
+              int64_t N, int64_t K, int f, cudaStream_t st);
 
 // Set the function attributes a launch needs (dynamic shared memory bytes,
 // the all-shared L1 carveout, and optionally non-portable cluster sizes)
