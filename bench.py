@@ -257,8 +257,11 @@ def time_linear(L, a, fmt, G, peak_tf):
     fl = 2.0 * M * N * K
     ab = act_bytes(M, K, fmt, G)
     return {"M": M, "N": N, "K": K, "act_us": t_act, "gemm_us": t_gemm,
-            "gemm_traffic": measured_traffic(f"gemm_nvfp4_{M}x{N}x{K}", ["dq_gemm.cu", "dq_device.cuh"]),
-            "act_traffic": measured_traffic(f"act_nvfp4_{M}x{K}", ["dq_quant.cu", "dq_device.cuh"]),
+            # the captures are of the NVFP4 kernels
+            "gemm_traffic": (measured_traffic(f"gemm_nvfp4_{M}x{N}x{K}", ["dq_gemm.cu", "dq_device.cuh"])
+                             if dq._fmt(fmt) == dq.DQ_NVFP4 else None),
+            "act_traffic": (measured_traffic(f"act_nvfp4_{M}x{K}", ["dq_quant.cu", "dq_device.cuh"])
+                            if dq._fmt(fmt) == dq.DQ_NVFP4 else None),
             "gemm_tflops": fl / (t_gemm * 1e-6) / 1e12, "gemm_frac": fl / (t_gemm * 1e-6) / 1e12 / peak_tf,
             "act_gbs": ab / (t_act * 1e-6) / 1e9, "linear_tflops": fl / ((t_act + t_gemm) * 1e-6) / 1e12}
 
@@ -539,7 +542,7 @@ def run_ours(args, rank, world, local_rank):
                            fmt in (dq.DQ_NVFP4, dq.DQ_MXFP4) else "tcgen05 GEMM"),
                 "gemm_us": t_gemm, "act_plus_gemm_us": t_pair, "fused_us": t_fused,
                 "gemm_traffic": (measured_traffic(f"gemv_nvfp4_{M}x{N}x{K}", ["dq_gemv.cu", "dq_device.cuh"])
-                                 if M == 1 else None),
+                                 if M == 1 and dq._fmt(fmt) == dq.DQ_NVFP4 else None),
                 "algorithmic_bytes": b_, "gemm_gbs": b_ / (t_gemm * 1e-6) / 1e9,
                 "gemm_frac_hbm": b_ / (t_gemm * 1e-6) / 1e9 / hbm,
                 "pair_gbs": b_ / (t_pair * 1e-6) / 1e9,
