@@ -142,73 +142,38 @@ w4a4_gemv_kernel(const uint8_t* __restrict__ A, const uint8_t* __restrict__ sA,
   for (int i = tid; i < rows * WARPS * MT; i += THREADS) part[i] = 0.0f;
   // the quads' scale pieces: 16 bytes per (quad, atom) = the four quarters'
   // 4 scale bytes of row d % 32; consecutive quads are consecutive pieces
-  // (four loads in flight per thread: the loops below are latency-bound)
-  for (int i0s = tid; i0s < nq * S4; i0s += 4 * THREADS) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0s + u * THREADS;
-      if (i < nq * S4) {
-        const int ql = i % nq, at = i / nq;
-        const int64_t d = q0 + ql;
-        v[u] = __ldg(reinterpret_cast<const uint4*>(sB + ((((d >> 5) * S4) + at) << 9) +
-                                                    ((d & 31) << 4)));
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0s + u * THREADS;
-      if (i < nq * S4) {
-        const int ql = i % nq, at = i / nq;
-        *reinterpret_cast<uint4*>(scs + ((size_t)ql * S4 + at) * 16) = v[u];
-      }
-    }
+  for (int i = tid; i < nq * S4; i += THREADS) {
+    const int ql = i % nq, at = i / nq;
+    const int64_t d = q0 + ql;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+        sB + ((((d >> 5) * S4) + at) << 9) + ((d & 31) << 4)));
+    *reinterpret_cast<uint4*>(scs + ((size_t)ql * S4 + at) * 16) = v;
   }
 
   pdl_wait();
   // ---- stage the activations (tokens >= M are zeros)
   const int W8 = K >> 3;   // code words (8 elements) per token
-  for (int i0a = tid; i0a < MT * W8; i0a += 4 * THREADS) {
-    uint32_t w[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0a + u * THREADS;
-      const int t = i / W8, jw = i - t * W8;
-      w[u] = (i < MT * W8 && t < M)
-                 ? __ldg(reinterpret_cast<const uint32_t*>(A + (size_t)t * (K >> 1)) + jw)
-                 : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0a + u * THREADS;
-      if (i >= MT * W8) break;
-      const int t = i / W8, jw = i - t * W8;
-      const uint32_t m = w[u] & 0x77777777u;
-      const uint32_t pl = mag_permute(w[u]), ph = mag_permute(w[u] >> 16);
-      const uint32_t ml = mag_permute(m), mh = mag_permute(m >> 16);
-      // per byte 2 pos - mag: +|2a| for positive codes, -|2a| for negative ones
-      const uint32_t lo = __vsub4(pl + pl, ml), hi = __vsub4(ph + ph, mh);
-      const int k = jw << 3;
-      *reinterpret_cast<uint2*>(a8 + (size_t)t * K + ((k >> 10) << 10) + (((k >> 4) & 1) << 9) +
-                                (((k >> 5) & 31) << 4) + (k & 8)) = make_uint2(lo, hi);
-    }
+  for (int i = tid; i < MT * W8; i += THREADS) {
+    const int t = i / W8, jw = i - t * W8;
+    const uint32_t w =
+        t < M ? __ldg(reinterpret_cast<const uint32_t*>(A + (size_t)t * (K >> 1)) + jw) : 0u;
+    const uint32_t m = w & 0x77777777u;
+    const uint32_t pl = mag_permute(w), ph = mag_permute(w >> 16);
+    const uint32_t ml = mag_permute(m), mh = mag_permute(m >> 16);
+    // per byte 2 pos - mag: +|2a| for positive codes, -|2a| for negative ones
+    const uint32_t lo = __vsub4(pl + pl, ml), hi = __vsub4(ph + ph, mh);
+    const int k = jw << 3;
+    *reinterpret_cast<uint2*>(a8 + (size_t)t * K + ((k >> 10) << 10) + (((k >> 4) & 1) << 9) +
+                              (((k >> 5) & 31) << 4) + (k & 8)) = make_uint2(lo, hi);
   }
-  for (int i0s = tid; i0s < MT * S; i0s += 4 * THREADS) {
-    uint32_t b[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0s + u * THREADS;
-      const int t = i / S, sb = i - t * S;
-      b[u] = (i < MT * S && t < M) ? (uint32_t)__ldg(sA + sf_offset(t, sb, S)) : 0xFFFFFFFFu;
+  for (int i = tid; i < MT * S; i += THREADS) {
+    const int t = i / S, sb = i - t * S;
+    float v = 0.0f;
+    if (t < M) {
+      const uint32_t b = __ldg(sA + sf_offset(t, sb, S));
+      v = __fmul_rn(FMT == NVFP4 ? ue4m3_value(b) : e8m0_value(b), 0.25f);
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0s + u * THREADS;
-      if (i >= MT * S) break;
-      asc[i] = b[u] == 0xFFFFFFFFu
-                   ? 0.0f
-                   : __fmul_rn(FMT == NVFP4 ? ue4m3_value(b[u]) : e8m0_value(b[u]), 0.25f);
-    }
+    asc[i] = v;
   }
   __syncthreads();
   pdl_trigger();
